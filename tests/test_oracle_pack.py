@@ -1,0 +1,174 @@
+"""Pins for the oracle's reorder, bit-packing and record layout (CPU only).
+
+Format: FORMAT.md sections 2-4 (PackKV paper page, Figure 2 steps 1 and 2;
+TL;DR: reorder with K and V bound together, light lossless encoding).
+"""
+import os
+import struct
+
+import numpy as np
+import pytest
+
+import oracle as O
+from decode_gemv_packkv_b200 import synth
+
+
+def _lines(path):
+    with open(path) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                yield line
+
+
+def test_pack_unit_hand_words(golden_dir):
+    for line in _lines(os.path.join(golden_dir, "pack_units.txt")):
+        wtxt, rule, words = (t.strip() for t in line.split("|"))
+        w = int(wtxt[2:])
+        offs = np.array([eval(rule, {"j": j}) for j in range(32)], np.int64)  # rule text from the fixture
+        want = [int(t, 16) for t in words.split()]
+        got = O.pack_unit(offs, w)
+        assert [int(x) for x in got] == want, line
+        assert np.array_equal(O.unpack_unit(got, w), offs)
+
+
+@pytest.mark.parametrize("w", [0, 1, 2, 3, 4])
+def test_pack_round_trip_and_size(w):
+    rng = np.random.default_rng(w)
+    for _ in range(200):
+        offs = rng.integers(0, 1 << w, 32) if w else np.zeros(32, np.int64)
+        words = O.pack_unit(offs, w)
+        assert words.shape == (w,)          # exactly w words: 32*w bits, no padding
+        assert np.array_equal(O.unpack_unit(words, w), offs)
+
+
+def test_unit_width_is_minimal():
+    rng = np.random.default_rng(3)
+    for _ in range(2000):
+        codes = rng.integers(0, 16, 32) >> rng.integers(0, 5)
+        codes = codes + rng.integers(0, 3)
+        base, w = O.unit_base_width(codes)
+        offs = codes - base
+        assert base == codes.min()
+        assert offs.max() < (1 << w)
+        assert w == 0 or offs.max() >= (1 << (w - 1))
+
+
+def test_stable_rank_matches_sorted():
+    rng = np.random.default_rng(5)
+    for trial in range(50):
+        keys = rng.integers(0, 6 if trial % 2 else 10**6, 128)
+        rank = O.stable_rank(keys)
+        order = sorted(range(128), key=lambda t: keys[t])   # Python's sort is stable
+        assert sorted(rank.tolist()) == list(range(128))
+        assert [order[r] for r in range(128)] == list(np.argsort(rank))
+        perm = np.empty(128, np.int64)
+        perm[rank] = np.arange(128)
+        assert np.all(np.diff(keys[perm]) >= 0)
+        ties = np.diff(keys[perm]) == 0
+        assert np.all(np.diff(perm)[ties] > 0)                  # ties keep index order
+    assert np.array_equal(O.stable_rank(np.zeros(128, np.int64)), np.arange(128))
+
+
+def _k1_block():
+    k = np.full((128, 128), np.float16(0.5))
+    k[:, 0] = (np.arange(128) % 2).astype(np.float16)
+    return k
+
+
+def _expected_record(spec):
+    f = dict(t.strip().split("=", 1) for t in spec.split("|")[1:])
+    out = bytearray()
+    out += struct.pack("<4H", *[int(x) for x in f["gws"].split(",")])
+    out += struct.pack("<II", int(f["flags"], 16), int(f["total_words"]))
+
+    def expand16(txt):
+        vals = []
+        for item in txt.split(","):
+            v, _, n = item.partition("*")
+            vals += [int(v, 16)] * (int(n) if n else 1)
+        assert len(vals) == 128
+        return struct.pack("<128H", *vals)
+    out += expand16(f["min"]) + expand16(f["scale"])
+    meta = bytearray(512)
+    for item in f["meta"].split(","):
+        where, val = item.split(":")
+        g, c = where[1:].split("c")
+        meta[int(g) * 128 + int(c)] = int(val, 16)
+    out += meta
+    if f["words"]:
+        w, _, n = f["words"].partition("*")
+        out += struct.pack("<I", int(w, 16)) * int(n)
+    out += b"\x00" * (int(f["len"]) - len(out))
+    return bytes(out)
+
+
+def test_records_hand_layout(golden_dir):
+    specs = {line.split("|")[0].strip(): line for line in _lines(os.path.join(golden_dir, "records.txt"))}
+    k = _k1_block()
+    v = np.zeros((128, 128), np.float16)
+    for key_kind, name in ((O.KEY_K_SUM, "K1_key1"), (O.KEY_IDENTITY, "K1_key0")):
+        k_rec, _, perm = O.encode_block(k, v, 4, key_kind)
+        assert k_rec == _expected_record(specs[name]), name
+        if key_kind == O.KEY_K_SUM:
+            assert perm.tolist() == list(range(0, 128, 2)) + list(range(1, 128, 2))
+        else:
+            assert perm.tolist() == list(range(128))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("structured", [False, True])
+def test_record_round_trip(bits, structured):
+    k, v, _ = synth.small_case(40 + bits, 1, 1, 1, 256, structured=structured)
+    for i in range(2):
+        kb, vb = k[0, 0, 128 * i:128 * (i + 1)], v[0, 0, 128 * i:128 * (i + 1)]
+        k_rec, v_rec, perm = O.encode_block(kb, vb, bits)
+        ck, k_mn, k_sc = O.quantize_block_k(kb, bits)
+        cv, v_mn, v_sc = O.quantize_block_v(vb, bits)
+        pk, pv = O.parse_record(k_rec), O.parse_record(v_rec)
+        assert np.array_equal(pk.codes, ck[perm]) and np.array_equal(pv.codes, cv[perm])
+        assert np.array_equal(pk.mn.view(np.uint16), k_mn.view(np.uint16))
+        assert np.array_equal(pv.scale.view(np.uint16), v_sc[perm].view(np.uint16))
+        for rec, p in ((k_rec, pk), (v_rec, pv)):
+            assert len(rec) % 16 == 0
+            assert len(rec) <= O.record_bytes_max(bits)
+            assert p.raw == (len(rec) == O.raw_record_bytes(bits))
+            if not p.raw:
+                assert len(rec) == -(-(1040 + 4 * int(p.width.sum())) // 16) * 16
+                assert len(rec) < O.raw_record_bytes(bits)
+            assert p.is_v == (rec is v_rec)
+        # K-sum key: keys are non-decreasing in storage order
+        keys = ck.astype(np.int64).sum(axis=1)
+        assert np.all(np.diff(keys[perm]) >= 0)
+
+
+def test_random_blocks_fall_back_to_raw():
+    k, v, _ = synth.small_case(9, 1, 1, 1, 128)
+    for bits in (2, 3, 4):
+        k_rec, v_rec, _ = O.encode_block(k[0, 0], v[0, 0], bits)
+        assert len(k_rec) == O.raw_record_bytes(bits) == len(v_rec)
+
+
+def test_cache_append_equals_block_encode():
+    """Growing the cache token by token yields the records of a block encode ([Abs]: growth)."""
+    k, v, _ = synth.small_case(12, 2, 2, 1, 300)
+    a = O.OracleCache(2, 2, 4, 3)
+    a.encode_blocks(k[:, :, :256], v[:, :, :256], 2)
+    for t in range(256, 300):
+        a.append_token(k[:, :, t], v[:, :, t])
+    b = O.OracleCache(2, 2, 4, 3)
+    for t in range(300):
+        b.append_token(k[:, :, t], v[:, :, t])
+    assert a.n_blocks == b.n_blocks == 2 and a.tail_len == b.tail_len == 44
+    for bb in range(2):
+        for h in range(2):
+            for i in range(2):
+                assert a.record("k", bb, h, i) == b.record("k", bb, h, i)
+                assert a.record("v", bb, h, i) == b.record("v", bb, h, i)
+    assert np.array_equal(a.k_tail[:, :, :44], b.k_tail[:, :, :44])
+    # arena layout: ascending (b, h, block) within one encode call, offsets contiguous
+    offs = a.k_index[:, :, :2, 0].reshape(-1)
+    lens = a.k_index[:, :, :2, 1].reshape(-1)
+    assert np.array_equal(a.k_index[:, :, :2, 0].transpose(0, 1, 2).reshape(-1),
+                          np.concatenate([[0], np.cumsum(lens)[:-1]]))
+    assert offs[-1] + lens[-1] == len(a.k_arena) // 16
