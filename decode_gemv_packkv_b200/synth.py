@@ -34,7 +34,7 @@ class Workload:
     seq: int
     bits: tuple
     seed: int
-    decode_steps: int = 0       # streaming-growth workload: tokens appended after the prefill
+    decode_steps: int = 0       # streaming growth: tokens seq .. seq+decode_steps-1 are appended one by one
 
     @property
     def group(self) -> int:
@@ -113,24 +113,6 @@ def timing_probs(w: Workload, tokens: int) -> np.ndarray:
     rng = _slice_rng(w.seed + 2, 0)
     p = rng.random((w.batch, w.q_heads, tokens), dtype=np.float32)
     return (p / p.sum(axis=-1, keepdims=True)).astype(np.float32)
-
-
-def decode_tokens(w: Workload, step: int):
-    """The K, V token appended at decode step `step`: fp16 [B, Hkv, 128] each.
-    Same distributions as the prefill (continues each sequence)."""
-    k = np.empty((w.batch, w.kv_heads, HEAD_DIM), np.float16)
-    v = np.empty_like(k)
-    for b in range(w.batch):
-        for h in range(w.kv_heads):
-            rng = _slice_rng(w.seed, b * w.kv_heads + h)
-            mu = rng.standard_normal(HEAD_DIM, dtype=np.float32)
-            sigma = rng.uniform(0.5, 2.0, HEAD_DIM).astype(np.float32)
-            outliers = rng.choice(HEAD_DIM, 4, replace=False)
-            sigma[outliers] *= np.float32(10.0)
-            r2 = _slice_rng(w.seed + 3, (b * w.kv_heads + h) * (1 << 20) + step)
-            k[b, h] = (mu + sigma * r2.standard_normal(HEAD_DIM, dtype=np.float32)).astype(np.float16)
-            v[b, h] = r2.standard_normal(HEAD_DIM, dtype=np.float32).astype(np.float16)
-    return k, v
 
 
 def small_case(seed: int, batch: int, kv_heads: int, group: int, tokens: int,

@@ -1,0 +1,184 @@
+/*
+ * packkv.h — C ABI of the PackKV decode path for NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the PackKV paper page ("PackKV: Reducing KV Cache
+ * Memory Footprint through LLM-Aware Lossy Compression"):
+ *   - abstract: a KV cache compressed so that it stays compatible with its
+ *     dynamic growth during decoding, and decompression fused into the
+ *     matrix-vector products;
+ *   - Figure 1: each query dots every K vector, softmax, weighted sum of V;
+ *   - Figure 2 and the TL;DR: quantize, reorder the quantized vectors (K and V
+ *     bound together), bit-pack the integer codes along the channel direction;
+ *     decompression inside the matrix-vector multiply, no write-back;
+ *   - Figure 5: token-wise and channel-wise quantization granularity.
+ * Every parameter the pages leave open is fixed by FORMAT.md (version 1).
+ *
+ * Conventions for every call:
+ *   - Pointers named "device" are CUDA device pointers; all must be 16-byte
+ *     aligned.  fp16 data is passed as uint16_t (IEEE binary16 bits).
+ *   - The library never allocates, frees or synchronises memory, except
+ *     packkv_get_status, which synchronises `stream` to read the status word.
+ *     The caller owns every buffer.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     stream-ordered; host-side counters in packkv_cache are updated by the
+ *     calls at enqueue time.
+ *   - Errors found on the host are returned before anything is launched, and
+ *     nothing is written.  Errors found on the device (arena full, non-finite
+ *     input, corrupt index entry, a wait that gave up) set sticky bits in the
+ *     cache's status word; packkv_get_status reads and clears them.
+ *   - Thread safety: calls on one cache must be serialised by the caller.
+ */
+#ifndef PACKKV_H
+#define PACKKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PACKKV_ABI_VERSION 1u
+#define PACKKV_FORMAT_VERSION 1u
+#define PACKKV_BLOCK_TOKENS 128
+#define PACKKV_GROUP_TOKENS 32
+#define PACKKV_HEAD_DIM 128
+
+typedef enum {
+  PACKKV_OK = 0,
+  PACKKV_ERR_INVALID_ARG = 1,  /* bad pointer, alignment, shape or counter */
+  PACKKV_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. q_heads/kv_heads = 3) */
+  PACKKV_ERR_CAPACITY = 3,     /* cache block table full (host) or arena full (device) */
+  PACKKV_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  PACKKV_ERR_DEVICE = 5        /* device-detected error other than capacity */
+} packkv_status;
+
+/* Sticky device status bits (packkv_get_status). */
+#define PACKKV_DEV_CAPACITY 0x1u   /* an encode did not fit in an arena; its blocks are invalid */
+#define PACKKV_DEV_NONFINITE 0x2u  /* an encoded block held a NaN or Inf */
+#define PACKKV_DEV_BAD_RECORD 0x4u /* a GEMV met an invalid index entry; its outputs are NaN/skipped */
+#define PACKKV_DEV_TIMEOUT 0x8u    /* a kernel's bounded wait on an async copy gave up */
+
+/* Reorder keys (FORMAT.md section 2). */
+#define PACKKV_KEY_IDENTITY 0u
+#define PACKKV_KEY_K_SUM 1u
+#define PACKKV_KEY_KV_SUM 2u
+
+typedef struct {
+  uint32_t version;      /* PACKKV_FORMAT_VERSION */
+  uint32_t bits;         /* code width: 2, 3 or 4 */
+  uint32_t block_tokens; /* 128 */
+  uint32_t group_tokens; /* 32 */
+  uint32_t head_dim;     /* 128 */
+  uint32_t reorder_key;  /* PACKKV_KEY_* */
+} packkv_format;
+
+/*
+ * The packed cache of one attention layer: plain data, every pointer owned by
+ * the caller.  Zero ctrl[0..3] and set n_blocks = tail_len = 0 before first
+ * use (packkv_cache_reset does both).
+ */
+typedef struct {
+  packkv_format fmt;
+  int32_t batch;       /* sequences */
+  int32_t kv_heads;    /* KV heads per sequence */
+  int32_t max_blocks;  /* block-table capacity per (sequence, head) */
+  int32_t n_blocks;    /* host counter: packed blocks per (sequence, head), uniform over the batch */
+  int32_t tail_len;    /* host counter: tokens in the uncompressed tail, 0..127 */
+  int32_t reserved0;
+  uint8_t* k_arena;    /* device, arena_bytes: K records (FORMAT.md section 4) */
+  uint8_t* v_arena;    /* device, arena_bytes: V records */
+  uint64_t arena_bytes;/* capacity of EACH arena; multiple of 16, at most 2^36 */
+  uint32_t* k_index;   /* device u32 [batch][kv_heads][max_blocks][2] = {offset16, length16} */
+  uint32_t* v_index;   /* device, same shape */
+  uint16_t* k_tail;    /* device fp16 [batch][kv_heads][128][128], arrival order */
+  uint16_t* v_tail;    /* device fp16, same shape */
+  uint64_t* ctrl;      /* device u64[4]: K arena end (16-B units), V arena end, status bits, scratch */
+  uint8_t* perm;       /* device, optional (NULL): u8 [batch][kv_heads][max_blocks][128],
+                          perm[slot] = token index within the block */
+} packkv_cache;
+
+/* ABI version and sizeof(packkv_cache), for bindings to check their mirror. */
+uint32_t packkv_abi_version(void);
+size_t packkv_cache_struct_size(void);
+const char* packkv_status_string(packkv_status s);
+
+/* Largest record of one block for `bits` (the raw record: 528 + 2048*bits bytes).
+ * Returns 0 for unsupported bits. */
+size_t packkv_record_bytes_max(uint32_t bits);
+
+/* Workspace bytes packkv_pv_gemv needs for any n_blocks <= cache->max_blocks
+ * with `q_heads` query heads (split-K partials).  packkv_qk_gemv needs none. */
+size_t packkv_workspace_bytes(const packkv_cache* cache, int32_t q_heads);
+
+/* Validates the struct (host-side checks only).  Nothing is launched. */
+packkv_status packkv_cache_check(const packkv_cache* cache);
+
+/* Zeroes ctrl[0..3] on `stream` and sets n_blocks = tail_len = 0. */
+packkv_status packkv_cache_reset(packkv_cache* cache, void* stream);
+
+/*
+ * Encode n_blocks full blocks per (sequence, head) and append them to the cache
+ * (quantize, joint token reorder, channel-direction bit-packing: FORMAT.md
+ * sections 1-4; paper page Figures 2 and 5).
+ *   k, v: device fp16 [batch][kv_heads][n_blocks*128][128], row-major.
+ * Records go to the arenas in ascending (sequence, head, block) order.
+ * Requires tail_len == 0 and n_blocks + cache->n_blocks <= max_blocks
+ * (else PACKKV_ERR_INVALID_ARG / PACKKV_ERR_CAPACITY, nothing launched).
+ * On success cache->n_blocks += n_blocks.  If an arena overflows on the device,
+ * PACKKV_DEV_CAPACITY is set, nothing is written to the arenas and the new
+ * index entries are marked invalid.  n_blocks == 0 is a no-op.
+ */
+packkv_status packkv_encode_block(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
+                                  int32_t n_blocks, void* stream);
+
+/*
+ * Append one token per (sequence, head) to the uncompressed tail (the cache's
+ * dynamic growth, paper abstract).  k, v: device fp16 [batch][kv_heads][128].
+ * When the tail reaches 128 tokens it is encoded as one block (as
+ * packkv_encode_block) and tail_len returns to 0.
+ * PACKKV_ERR_CAPACITY if the tail is full-to-be and the block table is full.
+ */
+packkv_status packkv_append_token(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
+                                  void* stream);
+
+/*
+ * scores[b][hq][i] = scale * sum_c q[b][hq][c] * k_hat[b][hq/G][i][c]  (fp32 accumulate)
+ * over the packed blocks in storage order, then the tail in arrival order
+ * (FORMAT.md sections 6-7; paper page Figure 1, Figure 2 fused decompression).
+ *   q:      device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8}.
+ *   scores: device fp32, row (b, hq) starts at (b*q_heads + hq) * ld_scores;
+ *           ld_scores >= T = n_blocks*128 + tail_len, multiple of 4.
+ *   ws, ws_bytes: unused (may be NULL / 0).
+ * The decompressed K is never written to memory.  T == 0 is a no-op.
+ */
+packkv_status packkv_qk_gemv(const packkv_cache* cache, const uint16_t* q, int32_t q_heads,
+                             float scale, float* scores, int64_t ld_scores, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * out[b][hq][c] = sum_i p[b][hq][i] * v_hat[b][hq/G][i][c]  (fp32 accumulate)
+ * with p in the same storage order as the scores.
+ *   p:   device fp32, row (b, hq) at (b*q_heads + hq) * ld_p, ld_p >= T, multiple of 4.
+ *   out: device fp32 [batch][q_heads][128].
+ *   ws:  device, ws_bytes >= packkv_workspace_bytes(cache, q_heads): split-K
+ *        partial sums over the sequence plus one counter per (sequence, kv
+ *        head).  The caller zero-fills ws once before its first use; every
+ *        completed call leaves the counters at zero again.  Partials are
+ *        reduced in a fixed order, so results are deterministic on a given GPU.
+ *        Two calls sharing one ws must not overlap in time.
+ * With T == 0, out is set to zero.
+ */
+packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t ld_p,
+                             int32_t q_heads, float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, returns PACKKV_OK if no device status bit is set,
+ * else PACKKV_ERR_CAPACITY (capacity bit set) or PACKKV_ERR_DEVICE; stores
+ * the bits in *bits_out (if not NULL) and clears them. */
+packkv_status packkv_get_status(const packkv_cache* cache, void* stream, uint32_t* bits_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PACKKV_H */

@@ -359,6 +359,7 @@ class OracleCache:
         self.tail_len = 0
         self.k_tail = np.zeros((batch, kv_heads, BLOCK_TOKENS, HEAD_DIM), np.float16)
         self.v_tail = np.zeros((batch, kv_heads, BLOCK_TOKENS, HEAD_DIM), np.float16)
+        self._decoded = {}      # (tensor, b, h, block) -> fp64 [128, D]; records never change once written
 
     def encode_blocks(self, k: np.ndarray, v: np.ndarray, n_blocks: int, blocks=None):
         """Append n_blocks blocks per (batch, head); k, v: [B, Hkv, n_blocks*128, D] fp16.
@@ -400,8 +401,11 @@ class OracleCache:
         """All tokens of (b, h) in storage order, decoded to fp64 [T, D]: blocks then tail."""
         parts = []
         for i in range(self.n_blocks):
-            rec = parse_record(self.record(which, b, h, i))
-            parts.append(dequant_k(rec) if which == "k" else dequant_v(rec))
+            key = (which, b, h, i)
+            if key not in self._decoded:
+                rec = parse_record(self.record(which, b, h, i))
+                self._decoded[key] = dequant_k(rec) if which == "k" else dequant_v(rec)
+            parts.append(self._decoded[key])
         tail = (self.k_tail if which == "k" else self.v_tail)[b, h, :self.tail_len]
         parts.append(tail.astype(np.float64))
         return np.concatenate(parts, axis=0)

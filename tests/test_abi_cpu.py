@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every symbol its header declares, and
+rejects bad arguments on the host before launching anything (no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(packkv_\w+)\s*\(", text, flags=re.M))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def pk():
+    from decode_gemv_packkv_b200 import build
+    build.build()
+    from decode_gemv_packkv_b200 import packkv
+    return packkv
+
+
+def test_header_declares_the_four_calls():
+    names = _declared_functions()
+    for call in ("packkv_encode_block", "packkv_append_token", "packkv_qk_gemv", "packkv_pv_gemv"):
+        assert call in names
+
+
+def test_library_exports_every_declared_symbol(pk):
+    lib = ctypes.CDLL(pk.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(pk.EXPORTED) <= set(_declared_functions())
+
+
+def test_abi_constants(pk):
+    lib = pk._lib
+    assert lib.packkv_abi_version() == 1
+    assert lib.packkv_cache_struct_size() == ctypes.sizeof(pk.CacheStruct)
+    assert [lib.packkv_record_bytes_max(b) for b in (1, 2, 3, 4, 5)] == [0, 4624, 6672, 8720, 0]
+    assert lib.packkv_status_string(3) == b"capacity exceeded"
+
+
+def _fake_cache(pk, **over):
+    s = pk.CacheStruct()
+    s.fmt = pk.Format(1, 4, 128, 32, 128, 1)
+    s.batch, s.kv_heads, s.max_blocks, s.n_blocks, s.tail_len = 2, 2, 4, 0, 0
+    base = 0x10000000
+    for i, f in enumerate(["k_arena", "v_arena", "k_index", "v_index", "k_tail", "v_tail", "ctrl"]):
+        setattr(s, f, base + i * 0x100000)
+    s.arena_bytes = 1 << 20
+    for k, v in over.items():
+        if k in ("bits", "version", "reorder_key", "head_dim"):
+            setattr(s.fmt, k, v)
+        else:
+            setattr(s, k, v)
+    return s
+
+
+def test_host_checks_reject_before_launch(pk):
+    lib = pk._lib
+    ok = _fake_cache(pk)
+    assert lib.packkv_cache_check(ctypes.byref(ok)) == pk.OK
+    bad_cases = {
+        "bits": (dict(bits=5), pk.ERR_UNSUPPORTED),
+        "version": (dict(version=2), pk.ERR_UNSUPPORTED),
+        "head_dim": (dict(head_dim=64), pk.ERR_UNSUPPORTED),
+        "key": (dict(reorder_key=7), pk.ERR_UNSUPPORTED),
+        "misaligned": (dict(k_arena=0x10000008), pk.ERR_INVALID_ARG),
+        "null": (dict(ctrl=0), pk.ERR_INVALID_ARG),
+        "arena": (dict(arena_bytes=1000), pk.ERR_INVALID_ARG),
+        "tail": (dict(tail_len=128), pk.ERR_INVALID_ARG),
+        "blocks": (dict(n_blocks=5), pk.ERR_INVALID_ARG),
+    }
+    for name, (over, want) in bad_cases.items():
+        s = _fake_cache(pk, **over)
+        assert lib.packkv_cache_check(ctypes.byref(s)) == want, name
+    # call-level checks (all return before any CUDA call)
+    k = ctypes.c_void_p(0x20000000)
+    s = _fake_cache(pk, tail_len=3)
+    assert lib.packkv_encode_block(ctypes.byref(s), k, k, 1, None) == pk.ERR_INVALID_ARG  # tail not empty
+    s = _fake_cache(pk, n_blocks=4)
+    assert lib.packkv_encode_block(ctypes.byref(s), k, k, 1, None) == pk.ERR_CAPACITY
+    s = _fake_cache(pk, n_blocks=4, tail_len=127)
+    assert lib.packkv_append_token(ctypes.byref(s), k, k, None) == pk.ERR_CAPACITY
+    s = _fake_cache(pk)
+    assert lib.packkv_encode_block(ctypes.byref(s), ctypes.c_void_p(0x20000004), k, 1, None) == pk.ERR_INVALID_ARG
+    assert lib.packkv_encode_block(ctypes.byref(s), k, k, 0, None) == pk.OK  # no-op
+    assert s.n_blocks == 0
+    # GEMVs: bad head grouping, bad leading dimension
+    s = _fake_cache(pk, n_blocks=2)
+    assert lib.packkv_qk_gemv(ctypes.byref(s), k, 3, 1.0, k, 256, None, 0, None) == pk.ERR_INVALID_ARG
+    assert lib.packkv_qk_gemv(ctypes.byref(s), k, 6, 1.0, k, 256, None, 0, None) == pk.ERR_UNSUPPORTED
+    assert lib.packkv_qk_gemv(ctypes.byref(s), k, 2, 1.0, k, 255, None, 0, None) == pk.ERR_INVALID_ARG
+    assert lib.packkv_qk_gemv(ctypes.byref(s), k, 2, 1.0, k, 254, None, 0, None) == pk.ERR_INVALID_ARG
+    assert lib.packkv_pv_gemv(ctypes.byref(s), k, 256, 2, k, k, 0, None) == pk.ERR_INVALID_ARG  # ws too small
+    s = _fake_cache(pk)  # empty cache: q·Kᵀ is a no-op
+    assert lib.packkv_qk_gemv(ctypes.byref(s), k, 2, 1.0, k, 0, None, 0, None) == pk.OK

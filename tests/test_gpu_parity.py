@@ -1,0 +1,340 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Encoder: records, index, arena ends and permutations bit-exact.  GEMVs: every
+element within 1e-3 * sum|terms| (FORMAT.md section 7).  Small cases span
+several blocks, pack groups and a ragged tail; the full workload sizes are
+checked in the launch configuration the benchmark times, on sampled blocks the
+oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from decode_gemv_packkv_b200 import synth
+from parity_util import assert_within_terms, compare_encoder, gpu_record, gpu_records, to_dev
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / np.sqrt(128.0)
+
+
+@pytest.fixture(scope="module")
+def pk():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from decode_gemv_packkv_b200 import packkv
+    return packkv
+
+
+def _build(pk, k, v, bits, key=O.KEY_K_SUM, max_blocks=None, keep_perm=True, arena_bytes=None):
+    B, H, T, _ = k.shape
+    nb_total = T // 128
+    mb = max_blocks or max(1, nb_total + 1)
+    cache = pk.PackKVCache(B, H, mb, bits, reorder_key=key, keep_perm=keep_perm, arena_bytes=arena_bytes)
+    pk.prefill(cache, to_dev(k), to_dev(v))
+    ocache = O.OracleCache(B, H, mb, bits, key)
+    ocache.encode_blocks(k[:, :, :nb_total * 128], v[:, :, :nb_total * 128], nb_total)
+    for t in range(nb_total * 128, T):
+        ocache.append_token(k[:, :, t], v[:, :, t])
+    return cache, ocache
+
+
+def _qk(pk, cache, q, ld=None):
+    B, Hq, _ = q.shape
+    ld = ld or ((cache.tokens + 3) // 4 * 4)
+    scores = torch.full((B, Hq, ld), 7.0, dtype=torch.float32, device="cuda")
+    pk.packkv_qk_gemv(cache, to_dev(q), SCALE, scores)
+    torch.cuda.synchronize()
+    return scores.cpu().numpy()
+
+
+def _pv(pk, cache, p):
+    B, Hq, T = p.shape
+    ld = (T + 3) // 4 * 4
+    pd = torch.zeros((B, Hq, ld), dtype=torch.float32, device="cuda")
+    pd[:, :, :T] = to_dev(p.astype(np.float32))
+    out = torch.full((B, Hq, 128), 7.0, dtype=torch.float32, device="cuda")
+    pk.packkv_pv_gemv(cache, pd, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- encoder
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("structured", [False, True])
+@pytest.mark.parametrize("key", [O.KEY_IDENTITY, O.KEY_K_SUM, O.KEY_KV_SUM])
+def test_encoder_bit_exact(pk, bits, structured, key):
+    k, v, _ = synth.small_case(100 + bits + 3 * key, 2, 3, 1, 512, structured=structured)
+    cache, ocache = _build(pk, k, v, bits, key)
+    compare_encoder(cache, ocache)
+    assert pk.packkv_get_status(cache) == 0
+
+
+def test_encoder_two_calls_append_after_arena_end(pk):
+    """A second encode call appends after the first call's records (arena order)."""
+    k, v, _ = synth.small_case(5, 2, 2, 1, 768, structured=True)
+    cache = pk.PackKVCache(2, 2, 8, 3, keep_perm=True)
+    ocache = O.OracleCache(2, 2, 8, 3)
+    for lo, n in ((0, 2), (256, 3), (640, 1)):
+        sl = slice(lo, lo + 128 * n)
+        pk.packkv_encode_block(cache, to_dev(k[:, :, sl].copy()), to_dev(v[:, :, sl].copy()), n)
+        ocache.encode_blocks(k[:, :, sl], v[:, :, sl], n)
+    compare_encoder(cache, ocache)
+
+
+# ----------------------------------------------------------------------------- q·Kᵀ
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("structured", [False, True])
+def test_qk_parity(pk, bits, group, structured):
+    tail = {1: 0, 2: 37, 4: 127, 8: 1}[group]
+    k, v, q = synth.small_case(200 + bits * 10 + group, 2, 2, group, 3 * 128 + tail, structured=structured)
+    cache, ocache = _build(pk, k, v, bits)
+    got = _qk(pk, cache, q)
+    ref, terms = O.cache_qk(ocache, q, SCALE)
+    T = ocache.tokens
+    assert_within_terms(got[:, :, :T], ref, terms, "scores")
+    assert np.all(got[:, :, T:] == 7.0), "wrote past T"
+
+
+def test_qk_leading_dimension_and_tail_only(pk):
+    k, v, q = synth.small_case(9, 1, 2, 2, 77)
+    cache, ocache = _build(pk, k, v, 4)
+    assert cache.n_blocks == 0 and cache.tail_len == 77
+    got = _qk(pk, cache, q, ld=200)
+    ref, terms = O.cache_qk(ocache, q, SCALE)
+    assert_within_terms(got[:, :, :77], ref, terms, "tail scores")
+    assert np.all(got[:, :, 77:] == 7.0)
+
+
+# ----------------------------------------------------------------------------- p·V
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("structured", [False, True])
+def test_pv_parity(pk, bits, group, structured):
+    tail = {1: 5, 2: 0, 4: 64, 8: 127}[group]
+    k, v, q = synth.small_case(300 + bits * 10 + group, 2, 2, group, 5 * 128 + tail, structured=structured)
+    cache, ocache = _build(pk, k, v, bits)
+    scores, _ = O.cache_qk(ocache, q, SCALE)
+    p = O.softmax(scores).astype(np.float32)          # storage order, same fp32 p on both sides
+    got = _pv(pk, cache, p)
+    ref, terms = O.cache_pv(ocache, p)
+    assert_within_terms(got, ref, terms, "p·V (softmax p)")
+    rng = np.random.default_rng(bits + group)
+    p2 = rng.standard_normal(p.shape).astype(np.float32)  # signed weights: cancellation
+    got2 = _pv(pk, cache, p2)
+    ref2, terms2 = O.cache_pv(ocache, p2)
+    assert_within_terms(got2, ref2, terms2, "p·V (signed p)")
+
+
+def test_pv_is_deterministic_and_leaves_workspace_zeroed(pk):
+    k, v, q = synth.small_case(12, 2, 4, 2, 20 * 128 + 3)
+    cache, _ = _build(pk, k, v, 4, keep_perm=False)
+    p = np.random.default_rng(0).random((2, 8, cache.tokens)).astype(np.float32)
+    a = _pv(pk, cache, p)
+    b = _pv(pk, cache, p)
+    assert np.array_equal(a, b)
+    ws = cache.workspace(8).cpu().numpy()
+    assert not ws[:2 * 4 * 4].any(), "counters not reset"
+
+
+def test_empty_cache(pk):
+    cache = pk.PackKVCache(1, 2, 4, 3)
+    out = torch.full((1, 2, 128), 5.0, device="cuda")
+    pk.packkv_pv_gemv(cache, torch.zeros((1, 2, 4), device="cuda"), out)
+    scores = torch.full((1, 2, 4), 5.0, device="cuda")
+    pk.packkv_qk_gemv(cache, torch.zeros((1, 2, 128), dtype=torch.float16, device="cuda"), 1.0, scores)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0) and torch.all(scores == 5.0)
+
+
+# ----------------------------------------------------------------------------- growth
+@pytest.mark.parametrize("bits", [2, 4])
+def test_streaming_append_matches_oracle(pk, bits):
+    """Token-by-token growth across block boundaries ([Abs]: dynamic growth)."""
+    B, H, G = 2, 2, 2
+    k, v, q = synth.small_case(41 + bits, B, H, G, 128 + 300, structured=(bits == 2))
+    cache = pk.PackKVCache(B, H, 4, bits, keep_perm=True)
+    ocache = O.OracleCache(B, H, 4, bits)
+    pk.packkv_encode_block(cache, to_dev(k[:, :, :128].copy()), to_dev(v[:, :, :128].copy()), 1)
+    ocache.encode_blocks(k[:, :, :128], v[:, :, :128], 1)
+    kd, vd = to_dev(k), to_dev(v)
+    for t in range(128, 428):
+        pk.packkv_append_token(cache, kd[:, :, t].contiguous(), vd[:, :, t].contiguous())
+        ocache.append_token(k[:, :, t], v[:, :, t])
+        if t in (128, 254, 255, 256, 383, 384, 427):
+            assert (cache.n_blocks, cache.tail_len) == (ocache.n_blocks, ocache.tail_len)
+            got = _qk(pk, cache, q)
+            ref, terms = O.cache_qk(ocache, q, SCALE)
+            assert_within_terms(got[:, :, :ocache.tokens], ref, terms, f"scores at t={t}")
+            p = O.softmax(ref).astype(np.float32)
+            got_o = _pv(pk, cache, p)
+            ref_o, terms_o = O.cache_pv(ocache, p)
+            assert_within_terms(got_o, ref_o, terms_o, f"out at t={t}")
+    compare_encoder(cache, ocache)
+    with pytest.raises(pk.PackKVError):
+        for t in range(428, 428 + 128):   # the 4th block would exceed max_blocks=4? 3 + 1 fits; a 5th does not
+            pk.packkv_append_token(cache, kd[:, :, 0].contiguous(), vd[:, :, 0].contiguous())
+        for t in range(128):
+            pk.packkv_append_token(cache, kd[:, :, 0].contiguous(), vd[:, :, 0].contiguous())
+
+
+# ----------------------------------------------------------------------------- device-detected errors
+def test_arena_overflow_is_detected_on_device(pk):
+    k, v, q = synth.small_case(77, 1, 2, 1, 256)
+    cache = pk.PackKVCache(1, 2, 4, 4, arena_bytes=3 * 8720)   # room for 3 of the 4 records
+    pk.packkv_encode_block(cache, to_dev(k), to_dev(v), 2)
+    bits = pk.packkv_get_status(cache)
+    assert bits & pk.DEV_CAPACITY
+    assert cache.arena_used() == (0, 0)
+    idx = cache.k_index.cpu().numpy().view(np.uint32)
+    assert np.all(idx[0, :, :2, 0] == 0xFFFFFFFF)
+    scores = torch.zeros((1, 2, 256), device="cuda")
+    pk.packkv_qk_gemv(cache, to_dev(q), 1.0, scores)
+    assert torch.all(torch.isnan(scores))
+    assert pk.packkv_get_status(cache) & pk.DEV_BAD_RECORD
+    assert pk.packkv_get_status(cache) == 0     # read-and-clear
+
+
+def test_nonfinite_input_sets_status(pk):
+    k, v, _ = synth.small_case(78, 1, 1, 1, 128)
+    k[0, 0, 5, 7] = np.inf
+    cache = pk.PackKVCache(1, 1, 2, 4)
+    pk.packkv_encode_block(cache, to_dev(k), to_dev(v), 1)
+    assert pk.packkv_get_status(cache) & pk.DEV_NONFINITE
+
+
+# ----------------------------------------------------------------------------- full workload sizes
+def _upload(w, tokens, structured=False):
+    """K, V on the device for a workload, generated one (b, h) slice at a time."""
+    kd = torch.empty((w.batch, w.kv_heads, tokens, 128), dtype=torch.float16, device="cuda")
+    vd = torch.empty_like(kd)
+    for b in range(w.batch):
+        for h in range(w.kv_heads):
+            ks, vs = synth.kv_slice(w.seed, w.kv_heads, b, h, tokens, structured=structured)
+            kd[b, h].copy_(torch.from_numpy(ks))
+            vd[b, h].copy_(torch.from_numpy(vs))
+    return kd, vd
+
+
+def _sampled_check(pk, w, bits, kd, vd, cache, samples, full_bh):
+    """Encoder records, scores and outputs on sampled blocks (+ one whole sequence)."""
+    q = synth.queries(w)
+    G = w.group
+    T = cache.tokens
+    scores = torch.empty((w.batch, w.q_heads, T), dtype=torch.float32, device="cuda")
+    pk.packkv_qk_gemv(cache, to_dev(q), SCALE, scores)
+    # p nonzero on the sampled blocks only: the oracle needs just those blocks
+    p = np.zeros((w.batch, w.q_heads, T), np.float32)
+    rng = np.random.default_rng(bits)
+    for (b, h, i) in samples:
+        p[b, h * G:(h + 1) * G, i * 128:(i + 1) * 128] = rng.random((G, 128), dtype=np.float32)
+    out = torch.empty((w.batch, w.q_heads, 128), dtype=torch.float32, device="cuda")
+    pk.packkv_pv_gemv(cache, to_dev(p), out)
+    torch.cuda.synchronize()
+    s_np = scores.cpu().numpy()
+    o_np = out.cpu().numpy()
+    karena, kindex = gpu_records(cache, "k")
+    varena, vindex = gpu_records(cache, "v")
+    o_ref = np.zeros_like(o_np, dtype=np.float64)
+    o_terms = np.zeros_like(o_ref)
+    for (b, h, i) in samples:
+        kb = kd[b, h, i * 128:(i + 1) * 128].cpu().numpy()
+        vb = vd[b, h, i * 128:(i + 1) * 128].cpu().numpy()
+        k_rec, v_rec, _ = O.encode_block(kb, vb, bits)
+        assert gpu_record(karena, kindex, b, h, i) == k_rec, f"K record {(b, h, i)}"
+        assert gpu_record(varena, vindex, b, h, i) == v_rec, f"V record {(b, h, i)}"
+        kdec = O.dequant_k(O.parse_record(k_rec))
+        vdec = O.dequant_v(O.parse_record(v_rec))
+        ref, terms = O.qk_scores(q[b, h * G:(h + 1) * G], kdec, SCALE)
+        assert_within_terms(s_np[b, h * G:(h + 1) * G, i * 128:(i + 1) * 128], ref, terms, f"scores {(b, h, i)}")
+        o, t = O.pv_out(p[b, h * G:(h + 1) * G, i * 128:(i + 1) * 128], vdec)
+        o_ref[b, h * G:(h + 1) * G] += o
+        o_terms[b, h * G:(h + 1) * G] += t
+    assert_within_terms(o_np, o_ref, o_terms, "p·V on sampled blocks")
+    # one whole sequence, dense softmax p
+    b, h = full_bh
+    ocache = O.OracleCache(1, 1, cache.n_blocks, bits)
+    nbk = cache.n_blocks
+    ocache.encode_blocks(kd[b:b + 1, h:h + 1, :nbk * 128].cpu().numpy(), vd[b:b + 1, h:h + 1, :nbk * 128].cpu().numpy(),
+                         nbk)
+    ref, terms = O.cache_qk(ocache, q[b:b + 1, h * G:(h + 1) * G], SCALE)
+    assert_within_terms(s_np[b:b + 1, h * G:(h + 1) * G], ref, terms, "scores, whole sequence")
+    pdense = np.zeros((w.batch, w.q_heads, T), np.float32)
+    pdense[b, h * G:(h + 1) * G] = O.softmax(ref[0]).astype(np.float32)
+    pk.packkv_pv_gemv(cache, to_dev(pdense), out)
+    ref_o, terms_o = O.cache_pv(ocache, pdense[b:b + 1, h * G:(h + 1) * G])
+    assert_within_terms(out.cpu().numpy()[b:b + 1, h * G:(h + 1) * G], ref_o, terms_o, "p·V, whole sequence")
+    assert np.all(np.isfinite(s_np))
+    assert pk.packkv_get_status(cache) == 0
+
+
+@pytest.mark.parametrize("wid,bits", [(0, 4), (1, 4), (2, 4), (2, 2), (3, 3)])
+def test_full_workload_sampled(pk, wid, bits):
+    w = synth.WORKLOADS[wid]
+    kd, vd = _upload(w, w.seq)
+    nb = w.seq // 128
+    cache = pk.PackKVCache(w.batch, w.kv_heads, nb, bits)
+    pk.packkv_encode_block(cache, kd, vd, nb)
+    rng = np.random.default_rng(wid)
+    samples = {(int(rng.integers(w.batch)), int(rng.integers(w.kv_heads)), int(rng.integers(nb)))
+               for _ in range(6)}
+    samples |= {(0, 0, 0), (w.batch - 1, w.kv_heads - 1, nb - 1)}
+    _sampled_check(pk, w, bits, kd, vd, cache, sorted(samples), (w.batch - 1, w.kv_heads // 2))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_streaming_workload(pk, bits):
+    """Batch 4 x 32 heads, prefill 8192 then 4096 appended tokens; GEMVs every step,
+    checked against the oracle at steps 0, 1, 127, 128, 129, every 512th and the last
+    on two sequences, and every block encoded during decode checked bit-exact there."""
+    w = synth.WORKLOADS[4]
+    total = w.seq + w.decode_steps
+    kd, vd = _upload(w, total)
+    nb_max = total // 128
+    cache = pk.PackKVCache(w.batch, w.kv_heads, nb_max, bits)
+    pk.packkv_encode_block(cache, kd[:, :, :w.seq].contiguous(), vd[:, :, :w.seq].contiguous(), w.seq // 128)
+    G = w.group
+    check_steps = {0, 1, 127, 128, 129, w.decode_steps - 1} | set(range(0, w.decode_steps, 512))
+    seqs = [(0, 3), (w.batch - 1, w.kv_heads - 1)]
+    oc = {}
+    for (b, h) in seqs:
+        o = O.OracleCache(1, 1, nb_max, bits)
+        o.encode_blocks(kd[b:b + 1, h:h + 1, :w.seq].cpu().numpy(), vd[b:b + 1, h:h + 1, :w.seq].cpu().numpy(),
+                        w.seq // 128)
+        oc[(b, h)] = o
+    k_np = {bh: kd[bh[0], bh[1], w.seq:].cpu().numpy() for bh in seqs}
+    v_np = {bh: vd[bh[0], bh[1], w.seq:].cpu().numpy() for bh in seqs}
+    ld = (total + 3) // 4 * 4
+    scores = torch.empty((w.batch, w.q_heads, ld), dtype=torch.float32, device="cuda")
+    out = torch.empty((w.batch, w.q_heads, 128), dtype=torch.float32, device="cuda")
+    for step in range(w.decode_steps):
+        t = w.seq + step
+        pk.packkv_append_token(cache, kd[:, :, t].contiguous(), vd[:, :, t].contiguous())
+        for bh in seqs:
+            oc[bh].append_token(k_np[bh][step][None, None], v_np[bh][step][None, None])
+        q = synth.queries(w, step)
+        pk.packkv_qk_gemv(cache, to_dev(q), SCALE, scores)
+        T = cache.tokens
+        p = torch.softmax(scores[:, :, :T], dim=-1)
+        pfull = torch.zeros_like(scores)
+        pfull[:, :, :T] = p
+        pk.packkv_pv_gemv(cache, pfull, out)
+        if step in check_steps:
+            s_np = scores.cpu().numpy()
+            p_np = pfull.cpu().numpy()
+            o_np = out.cpu().numpy()
+            for (b, h), o in oc.items():
+                assert o.tokens == T
+                ref, terms = O.cache_qk(o, q[b:b + 1, h * G:(h + 1) * G], SCALE)
+                assert_within_terms(s_np[b:b + 1, h * G:(h + 1) * G, :T], ref, terms, f"scores step {step}")
+                ref_o, terms_o = O.cache_pv(o, p_np[b:b + 1, h * G:(h + 1) * G, :T])
+                assert_within_terms(o_np[b:b + 1, h * G:(h + 1) * G], ref_o, terms_o, f"out step {step}")
+    karena, kindex = gpu_records(cache, "k")
+    varena, vindex = gpu_records(cache, "v")
+    for (b, h), o in oc.items():
+        for i in range(w.seq // 128, o.n_blocks):
+            assert gpu_record(karena, kindex, b, h, i) == o.record("k", 0, 0, i)
+            assert gpu_record(varena, vindex, b, h, i) == o.record("v", 0, 0, i)
+    assert pk.packkv_get_status(cache) == 0
