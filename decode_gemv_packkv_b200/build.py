@@ -29,14 +29,15 @@ def sources():
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 
 
-def build(verbose_ptxas: bool = False, force: bool = False) -> str:
+def build(verbose_ptxas: bool = False, force: bool = False, out: str | None = None, defines=()) -> str:
     srcs = sources()
     deps = srcs + glob.glob(os.path.join(HERE, "csrc", "*.h")) + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) \
         + [os.path.join(ROOT, "include", "packkv.h")]
-    if not force and os.path.exists(LIB) and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in deps):
-        return LIB
+    lib = out or LIB
+    if not force and os.path.exists(lib) and all(os.path.getmtime(lib) >= os.path.getmtime(d) for d in deps):
+        return lib
     cmd = [nvcc(), *ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *srcs]
+           "-I", os.path.join(ROOT, "include"), *[f"-D{d}" for d in defines], "-o", lib + ".tmp", *srcs]
     if verbose_ptxas:
         cmd[1:1] = ["-Xptxas", "-v"]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -45,8 +46,8 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
         raise RuntimeError("nvcc failed building libpackkv.so")
     if verbose_ptxas:
         sys.stderr.write(res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -209,9 +209,7 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
   a.p = p;
   a.ld = ld_p;
   a.out = out;
-  const size_t bh = (size_t)cache->batch * cache->kv_heads;
-  a.counters = reinterpret_cast<uint32_t*>(ws);
-  a.partials = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(ws) + (bh * 4 + 255) / 256 * 256);
+  a.partials = reinterpret_cast<float*>(ws);
   return cuda_status(packkv::launch_pv(a, as_stream(stream)));
 }
 

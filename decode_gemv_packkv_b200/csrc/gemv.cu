@@ -26,9 +26,10 @@
 //  * q·Kᵀ: lanes split (group, token word, channel range); each lane keeps fp32
 //    accumulators for 8 or 16 tokens and a 2- or 4-way shuffle sum finishes.
 //  * p·V: lane = channel; a warp sums its item range into per-channel fp32
-//    partials, writes them to the workspace at every (sequence, head) boundary,
-//    and the last warp to finish a (sequence, head) (atomic counter, no waiting)
-//    adds the partials in warp order: deterministic, no second kernel.
+//    partials and writes them to the workspace at every (sequence, head)
+//    boundary (split-K over the sequence); a second-pass kernel, launched as a
+//    programmatic dependent so its launch overlaps the first, adds the partials
+//    of each (sequence, head) in warp order: deterministic.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -42,7 +43,10 @@ namespace packkv {
 namespace {
 
 constexpr int kWarpsPerCta = 4;
-constexpr int kWarpSmemBudget = 27 * 1024;  // two CTAs of 4 warps per SM
+#ifndef PACKKV_WARP_SMEM_KB
+#define PACKKV_WARP_SMEM_KB 10  // shared memory per warp: one stage, five CTAs of 4 warps per SM
+#endif
+constexpr int kWarpSmemBudget = PACKKV_WARP_SMEM_KB * 1024;
 constexpr uint32_t kMagicBits = 0x4B000000u;
 constexpr float kMagic = 8388608.0f;
 
@@ -52,39 +56,68 @@ __device__ __forceinline__ float mag(uint32_t field_bits) {
   return __uint_as_float(field_bits | kMagicBits) - kMagic;
 }
 
+// (w & mask) | 0x4B000000 in one LOP3: the field lands in the low mantissa bits of 2^23.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t fld(uint32_t w) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(kMagicBits));
+  return d;
+}
+
+// Two magic-number fields -> their exact values, with one packed FP32 add.
+__device__ __forceinline__ float2 pairf(uint32_t a, uint32_t b) {
+  return __fadd2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), make_float2(-kMagic, -kMagic));
+}
+
 // Field position exponents of the in-register decode (value = field * 2^sig).
 __host__ __device__ constexpr int sig4(int i) { return i <= 4 ? 4 * i : 4 * i - 12; }
 __host__ __device__ constexpr int sig2(int i) { return i <= 10 ? 2 * i : 2 * i - 12; }
 __host__ __device__ constexpr float pow2(int e) {
   return e >= 0 ? float(1u << e) : 1.0f / float(1u << (-e));
 }
+// 2^e for a run-time e in [-126, 127], from the exponent bits (no division)
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
 
-// 8 nibbles of a 4-bit slice word: v[i] = field_i * 2^sig4(i)
-__device__ __forceinline__ void dec4(uint32_t w, float (&v)[8]) {
+// 8 nibbles of a 4-bit slice word as 4 pairs: v[p] = (field_2p * 2^sig4(2p), field_2p+1 * 2^sig4(2p+1))
+__device__ __forceinline__ void dec4(uint32_t w, float2 (&v)[4]) {
   const uint32_t h = w >> 12;
-  v[0] = mag(w & 0xFu);
-  v[1] = mag(w & 0xF0u);
-  v[2] = mag(w & 0xF00u);
-  v[3] = mag(w & 0xF000u);
-  v[4] = mag(w & 0xF0000u);
-  v[5] = mag(h & 0xF00u);
-  v[6] = mag(h & 0xF000u);
-  v[7] = mag(h & 0xF0000u);
+  v[0] = pairf(fld<0xFu>(w), fld<0xF0u>(w));
+  v[1] = pairf(fld<0xF00u>(w), fld<0xF000u>(w));
+  v[2] = pairf(fld<0xF0000u>(w), fld<0xF00u>(h));
+  v[3] = pairf(fld<0xF000u>(h), fld<0xF0000u>(h));
 }
 
-// 16 two-bit fields of a 2-bit slice word: v[i] = field_i * 2^sig2(i)
-__device__ __forceinline__ void dec2(uint32_t w, float (&v)[16]) {
+template <int I>
+__device__ __forceinline__ uint32_t fld2(uint32_t w, uint32_t h) {
+  if constexpr (I <= 10)
+    return fld<(3u << (2 * I))>(w);
+  else
+    return fld<(3u << (2 * I - 12))>(h);
+}
+
+// 16 two-bit fields of a 2-bit slice word as 8 pairs: field_i * 2^sig2(i)
+__device__ __forceinline__ void dec2(uint32_t w, float2 (&v)[8]) {
   const uint32_t h = w >> 12;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = (i <= 10) ? mag(w & (3u << (2 * i))) : mag(h & (3u << (2 * i - 12)));
+  v[0] = pairf(fld2<0>(w, h), fld2<1>(w, h));
+  v[1] = pairf(fld2<2>(w, h), fld2<3>(w, h));
+  v[2] = pairf(fld2<4>(w, h), fld2<5>(w, h));
+  v[3] = pairf(fld2<6>(w, h), fld2<7>(w, h));
+  v[4] = pairf(fld2<8>(w, h), fld2<9>(w, h));
+  v[5] = pairf(fld2<10>(w, h), fld2<11>(w, h));
+  v[6] = pairf(fld2<12>(w, h), fld2<13>(w, h));
+  v[7] = pairf(fld2<14>(w, h), fld2<15>(w, h));
 }
 
 // 3-bit raw unit, 16 tokens: 2-bit slice word w2 plus the 16 slice-1 bits at bits 0..15 of x.
-// v[i] = (field2_i + 4*bit_i) * 2^sig2(i), merged with one exact FFMA.
-__device__ __forceinline__ void dec3(uint32_t w2, uint32_t x, float (&v)[16]) {
+// v[p] = (field2 + 4*bit) * 2^sig2, merged with one exact packed FMA per pair.
+__device__ __forceinline__ void dec3(uint32_t w2, uint32_t x, float2 (&v)[8]) {
   dec2(w2, v);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = fmaf(mag(x & (1u << i)), pow2(sig2(i) - i + 2), v[i]);
+  for (int p = 0; p < 8; ++p) {
+    const int i = 2 * p;
+    const float2 b = pairf(x & (1u << i) | kMagicBits, x & (2u << i) | kMagicBits);
+    v[p] = __ffma2_rn(b, make_float2(pow2(sig2(i) - i + 2), pow2(sig2(i + 1) - i + 1)), v[p]);
+  }
 }
 
 template <int BITS>
@@ -112,19 +145,21 @@ struct Cfg {
   static constexpr int kRecBytes = raw_record_bytes(BITS);
   static constexpr int kStageRec = 528 + kChunks * kPitch;     // >= every record of this width
   static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);
-  static constexpr int kTableBytes = 512 * G;
+  static constexpr int kTableBytes = (PV ? 512 : 1024) * G;
   static constexpr int kStages0 = (kWarpSmemBudget - kTableBytes - 64) / kStageBytes;
-  static constexpr int kStages = kStages0 > 4 ? 4 : (kStages0 < 2 ? 2 : kStages0);
+  static constexpr int kStages = kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0);
   static constexpr int kWarpSmem = ((kStages * kStageBytes + kTableBytes + kStages * 16) + 127) / 128 * 128;
   // q' table: channel c = h*kChanPerChunk + cc stored at ((cc/4)*NH + h)*4 + cc%4
   static constexpr int kNH = 128 / kChanPerChunk;
 };
 
+// q' table of q·Kᵀ: (q'_c, q'_c) pairs; channel c = h*kChanPerChunk + cc sits at float2
+// index ((cc/2)*NH + h)*2 + cc%2, so one 16-byte load gives a lane its next two channels.
 template <int BITS, int G, bool PV>
 __device__ __forceinline__ int table_index(int c) {
   using C = Cfg<BITS, G, PV>;
   const int h = c / C::kChanPerChunk, cc = c % C::kChanPerChunk;
-  return ((cc >> 2) * C::kNH + h) * 4 + (cc & 3);
+  return ((cc >> 1) * C::kNH + h) * 2 + (cc & 1);
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -156,18 +191,36 @@ struct WarpMem {
   }
 };
 
-// Issue the copies of item x into stage s (whole warp participates).
+// Position in the flat item list: (sequence*kv_heads + head, item within it).
+struct Cursor {
+  long bh;
+  int j;
+  __device__ void next(int items_per_bh) {
+    if (++j == items_per_bh) {
+      j = 0;
+      ++bh;
+    }
+  }
+};
+
+// Index entry {offset16, length16} of item c ({0, 0} for a tail item).  Loaded one
+// item ahead of its use so that its latency hides behind a block's arithmetic.
+__device__ __forceinline__ uint2 index_entry(const GemvArgs& a, Cursor c) {
+  if (c.j >= a.n_blocks) return make_uint2(0u, 0u);
+  return *reinterpret_cast<const uint2*>(a.index + ((size_t)c.bh * a.max_blocks + c.j) * 2);
+}
+
+// Issue the copies of item (bh, j) with index entry e into stage s (whole warp participates).
 template <int BITS, int G, bool PV>
-__device__ __forceinline__ void issue_item(const GemvArgs& a, const WarpMem<BITS, G, PV>& m, long x, int s,
-                                           int lane) {
+__device__ __forceinline__ void issue_item(const GemvArgs& a, const WarpMem<BITS, G, PV>& m, Cursor c, uint2 e,
+                                           int s, int lane) {
   using C = Cfg<BITS, G, PV>;
-  const long bh = x / a.items_per_bh;
-  const int j = (int)(x % a.items_per_bh);
+  const long bh = c.bh;
+  const int j = c.j;
   int kind = kKindTail;
   uint64_t off16 = 0;
   uint32_t len16 = 0;
   if (j < a.n_blocks) {
-    const uint2 e = *reinterpret_cast<const uint2*>(a.index + ((size_t)bh * a.max_blocks + j) * 2);
     off16 = e.x;
     len16 = e.y;
     const bool valid = e.x != 0xFFFFFFFFu && len16 >= 1040 / 16 && len16 * 16u <= (uint32_t)C::kRecBytes &&
@@ -209,98 +262,94 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const WarpMem<BITS
 // q·Kᵀ
 // ----------------------------------------------------------------------------
 template <int BITS, int G>
-__device__ __forceinline__ void qk_raw(const unsigned char* st, const float* qp, const float (&cst)[G],
+__device__ __forceinline__ void qk_raw(const unsigned char* st, const float2* qp, const float (&cst)[G],
                                        float* srow0, long ld, float scale, int lane) {
   using C = Cfg<BITS, G, false>;
   if constexpr (BITS == 4) {
+    // lane = (group g, token octet k, channel half h); word k of unit (g, c) holds tokens 32g+8k..+7
     const int h = lane & 1, k = (lane >> 1) & 3, g = lane >> 3;
     const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (2 * g + h) * C::kPitch) + k;
-    float acc[G][8];
+    float2 acc[G][4];
 #pragma unroll
     for (int hd = 0; hd < G; ++hd)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[hd][i] = 0.f;
-#pragma unroll 2
-    for (int c4 = 0; c4 < 16; ++c4) {
-      float4 qv[G];
+      for (int i = 0; i < 4; ++i) acc[hd][i] = make_float2(0.f, 0.f);
+#pragma unroll 4
+    for (int c2 = 0; c2 < 32; ++c2) {
+      float2 v0[4], v1[4];
+      dec4(wp[8 * c2], v0);
+      dec4(wp[8 * c2 + 4], v1);
 #pragma unroll
-      for (int hd = 0; hd < G; ++hd)
-        qv[hd] = *reinterpret_cast<const float4*>(qp + hd * 128 + (c4 * C::kNH + h) * 4);
-      uint32_t w[4];
+      for (int hd = 0; hd < G; ++hd) {
+        const float4 qq = *reinterpret_cast<const float4*>(qp + hd * 128 + (c2 * C::kNH + h) * 2);
+        const float2 q0 = make_float2(qq.x, qq.y), q1 = make_float2(qq.z, qq.w);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) w[t] = wp[4 * (c4 * 4 + t)];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        float v[8];
-        dec4(w[t], v);
-#pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          const float qq = t == 0 ? qv[hd].x : t == 1 ? qv[hd].y : t == 2 ? qv[hd].z : qv[hd].w;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) acc[hd][i] = fmaf(qq, v[i], acc[hd][i]);
+        for (int i = 0; i < 4; ++i) {
+          acc[hd][i] = __ffma2_rn(q0, v0[i], acc[hd][i]);
+          acc[hd][i] = __ffma2_rn(q1, v1[i], acc[hd][i]);
         }
       }
     }
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
+      float t[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[hd][i] += __shfl_xor_sync(0xffffffffu, acc[hd][i], 1);
+      for (int i = 0; i < 4; ++i) {
+        t[2 * i] = acc[hd][i].x + __shfl_xor_sync(0xffffffffu, acc[hd][i].x, 1);
+        t[2 * i + 1] = acc[hd][i].y + __shfl_xor_sync(0xffffffffu, acc[hd][i].y, 1);
+      }
       float o[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float lo = acc[hd][i] * pow2(-sig4(i));
-        const float hi = acc[hd][i + 4] * pow2(-sig4(i + 4));
+        const float lo = t[i] * pow2(-sig4(i));
+        const float hi = t[i + 4] * pow2(-sig4(i + 4));
         o[i] = scale * (cst[hd] + (h ? hi : lo));
       }
       float* dst = srow0 + hd * ld + 32 * g + 8 * k + 4 * h;
       *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
     }
   } else {
+    // lane = (group g, 16-token half k, channel quarter h)
     const int h = lane & 3, k = (lane >> 2) & 1, g = lane >> 3;
     const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + h) * C::kPitch);
-    float acc[G][16];
+    float2 acc[G][8];
 #pragma unroll
     for (int hd = 0; hd < G; ++hd)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc[hd][i] = 0.f;
-#pragma unroll 1
-    for (int c4 = 0; c4 < 8; ++c4) {
-      float4 qv[G];
-#pragma unroll
-      for (int hd = 0; hd < G; ++hd)
-        qv[hd] = *reinterpret_cast<const float4*>(qp + hd * 128 + (c4 * C::kNH + h) * 4);
-      uint32_t w[4], x[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const int cc = c4 * 4 + t;
-        if constexpr (BITS == 2) {
-          w[t] = wp[2 * cc + k];
-        } else {
-          w[t] = wp[3 * cc + k];
-          x[t] = wp[3 * cc + 2] >> (16 * k);
-        }
+      for (int i = 0; i < 8; ++i) acc[hd][i] = make_float2(0.f, 0.f);
+#pragma unroll 2
+    for (int c2 = 0; c2 < 16; ++c2) {
+      float2 v0[8], v1[8];
+      if constexpr (BITS == 2) {
+        dec2(wp[2 * (2 * c2) + k], v0);
+        dec2(wp[2 * (2 * c2 + 1) + k], v1);
+      } else {
+        dec3(wp[3 * (2 * c2) + k], wp[3 * (2 * c2) + 2] >> (16 * k), v0);
+        dec3(wp[3 * (2 * c2 + 1) + k], wp[3 * (2 * c2 + 1) + 2] >> (16 * k), v1);
       }
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        float v[16];
-        if constexpr (BITS == 2)
-          dec2(w[t], v);
-        else
-          dec3(w[t], x[t], v);
+      for (int hd = 0; hd < G; ++hd) {
+        const float4 qq = *reinterpret_cast<const float4*>(qp + hd * 128 + (c2 * C::kNH + h) * 2);
+        const float2 q0 = make_float2(qq.x, qq.y), q1 = make_float2(qq.z, qq.w);
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          const float qq = t == 0 ? qv[hd].x : t == 1 ? qv[hd].y : t == 2 ? qv[hd].z : qv[hd].w;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[hd][i] = fmaf(qq, v[i], acc[hd][i]);
+        for (int i = 0; i < 8; ++i) {
+          acc[hd][i] = __ffma2_rn(q0, v0[i], acc[hd][i]);
+          acc[hd][i] = __ffma2_rn(q1, v1[i], acc[hd][i]);
         }
       }
     }
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
+      float t[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        acc[hd][i] += __shfl_xor_sync(0xffffffffu, acc[hd][i], 1);
-        acc[hd][i] += __shfl_xor_sync(0xffffffffu, acc[hd][i], 2);
+      for (int i = 0; i < 8; ++i) {
+        float x = acc[hd][i].x, y = acc[hd][i].y;
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        y += __shfl_xor_sync(0xffffffffu, y, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        y += __shfl_xor_sync(0xffffffffu, y, 2);
+        t[2 * i] = x;
+        t[2 * i + 1] = y;
       }
       float o[4];
 #pragma unroll
@@ -308,7 +357,7 @@ __device__ __forceinline__ void qk_raw(const unsigned char* st, const float* qp,
         float v = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 4; ++hh)
-          if (h == hh) v = acc[hd][4 * hh + i] * pow2(-sig2(4 * hh + i));
+          if (h == hh) v = t[4 * hh + i] * pow2(-sig2(4 * hh + i));
         o[i] = scale * (cst[hd] + v);
       }
       float* dst = srow0 + hd * ld + 32 * g + 16 * k + 4 * h;
@@ -332,7 +381,7 @@ __device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, 
 }
 
 template <int BITS, int G>
-__device__ __forceinline__ void qk_packed(const unsigned char* st, const float* qp, const float (&cst)[G],
+__device__ __forceinline__ void qk_packed(const unsigned char* st, const float2* qp, const float (&cst)[G],
                                           float* srow0, long ld, float scale, int lane) {
   const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
   const uint8_t* meta = st + kMetaOffset;
@@ -347,7 +396,7 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float* 
       float part = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        part = fmaf(qp[hd * 128 + table_index<BITS, G, false>(4 * lane + i)], (float)((m4 >> (8 * i)) & 15u), part);
+        part = fmaf(qp[hd * 128 + table_index<BITS, G, false>(4 * lane + i)].x, (float)((m4 >> (8 * i)) & 15u), part);
       bsum[hd] = warp_sum(part);
     }
     float acc[G];
@@ -364,7 +413,7 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float* 
         s += w;
 #pragma unroll
         for (int hd = 0; hd < G; ++hd)
-          acc[hd] = fmaf(qp[hd * 128 + table_index<BITS, G, false>(4 * c4 + i)], u, acc[hd]);
+          acc[hd] = fmaf(qp[hd * 128 + table_index<BITS, G, false>(4 * c4 + i)].x, u, acc[hd]);
       }
     }
 #pragma unroll
@@ -418,16 +467,20 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
   }
   __syncwarp();
   long prod = lo;
-  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod) issue_item<BITS, G, false>(a, m, prod, s, lane);
+  Cursor pc{lo / a.items_per_bh, (int)(lo % a.items_per_bh)};
+  Cursor cc = pc;
+  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(a.items_per_bh))
+    issue_item<BITS, G, false>(a, m, pc, index_entry(a, pc), s, lane);
+  uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
 
   const int q_heads = a.kv_heads * G;
   long cur_bh = -1;
   float qr[G][4];
   uint32_t phases = 0;
   int s = 0;
-  for (long x = lo; x < hi; ++x) {
-    const long bh = x / a.items_per_bh;
-    const int j = (int)(x % a.items_per_bh);
+  for (long x = lo; x < hi; ++x, cc.next(a.items_per_bh)) {
+    const long bh = cc.bh;
+    const int j = cc.j;
     const long b = bh / a.kv_heads, h = bh % a.kv_heads;
     float* srow0 = a.scores + ((size_t)b * q_heads + h * G) * a.ld;
     if (bh != cur_bh) {
@@ -457,7 +510,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
         for (int i = lane; i < 128; i += 32) srow0[hd * a.ld + (long)j * 128 + i] = __int_as_float(0x7fc00000);
     } else {
       // per-block q' = q * scale_c (table) and the min term sum_c q_c * mn_c
-      float* qp = m.table();
+      float2* qp = reinterpret_cast<float2*>(m.table());
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -472,8 +525,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
         part = fmaf(qr[hd][2], mn1.x, part);
         part = fmaf(qr[hd][3], mn1.y, part);
         cst[hd] = warp_sum(part);
-        *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane)) =
-            make_float4(qr[hd][0] * sc0.x, qr[hd][1] * sc0.y, qr[hd][2] * sc1.x, qr[hd][3] * sc1.y);
+        const float q0 = qr[hd][0] * sc0.x, q1 = qr[hd][1] * sc0.y, q2 = qr[hd][2] * sc1.x, q3 = qr[hd][3] * sc1.y;
+        *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane)) = make_float4(q0, q0, q1, q1);
+        *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane + 2)) = make_float4(q2, q2, q3, q3);
       }
       __syncwarp();
       float* sblk = srow0 + (long)j * 128;
@@ -484,8 +538,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
     }
     __syncwarp();
     if (prod < hi) {
-      issue_item<BITS, G, false>(a, m, prod, s, lane);
+      issue_item<BITS, G, false>(a, m, pc, next_e, s, lane);
       ++prod;
+      pc.next(a.items_per_bh);
+      if (prod < hi) next_e = index_entry(a, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
@@ -494,59 +550,86 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
 // ----------------------------------------------------------------------------
 // p·V
 // ----------------------------------------------------------------------------
-// Accumulates one raw block into acc[slab][hd] (lane = channel slab*32 + lane).
+// Accumulates one raw block into acc[slab][hd] (lane = channel slab*32 + lane).  The
+// field exponents are folded into p'' = p * scale * 2^-sig, so decoded pairs multiply
+// consecutive p'' pairs directly.
 template <int BITS, int G>
-__device__ __forceinline__ void pv_raw(const unsigned char* st, const float* pp, float (&acc)[4][G], int lane) {
+__device__ __forceinline__ void pv_raw(const unsigned char* st, const float* pp, float2 (&acc)[4][G], int lane) {
   using C = Cfg<BITS, G, true>;
+  constexpr bool kRegP = G <= 2;  // keep the group's p'' in registers across the 4 slabs
 #pragma unroll 1
   for (int g = 0; g < 4; ++g) {
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl) {
-      float v[32];
-      if constexpr (BITS == 4) {
-        const uint4 u = *reinterpret_cast<const uint4*>(st + 528 + (2 * g + (sl >> 1)) * C::kPitch +
-                                                        ((sl & 1) * 32 + lane) * 16);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float t[8];
-          dec4(w[q], t);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[8 * q + i] = t[i];
-        }
-      } else if constexpr (BITS == 2) {
-        const uint2 u = *reinterpret_cast<const uint2*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 8);
-        float t[16];
-        dec2(u.x, t);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = t[i];
-        dec2(u.y, t);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 + i] = t[i];
-      } else {
-        const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 12);
-        const uint32_t w0 = wp[0], w1 = wp[1], w2 = wp[2];
-        float t[16];
-        dec3(w0, w2, t);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = t[i];
-        dec3(w1, w2 >> 16, t);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 + i] = t[i];
-      }
+    float2 pr[kRegP ? G : 1][16];
+    if constexpr (kRegP) {
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
         const float4* p4 = reinterpret_cast<const float4*>(pp + hd * 128 + 32 * g);
-        float a0 = 0.f, a1 = 0.f;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 pv = p4[q];
-          a0 = fmaf(pv.x, v[4 * q + 0], a0);
-          a1 = fmaf(pv.y, v[4 * q + 1], a1);
-          a0 = fmaf(pv.z, v[4 * q + 2], a0);
-          a1 = fmaf(pv.w, v[4 * q + 3], a1);
+          const float4 x = p4[q];
+          pr[hd][2 * q] = make_float2(x.x, x.y);
+          pr[hd][2 * q + 1] = make_float2(x.z, x.w);
         }
-        acc[sl][hd] += a0 + a1;
+      }
+    }
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      float2 v[16];
+      if constexpr (BITS == 4) {
+        const uint4 u = *reinterpret_cast<const uint4*>(st + 528 + (2 * g + (sl >> 1)) * C::kPitch +
+                                                        ((sl & 1) * 32 + lane) * 16);
+        float2 t[4];
+        dec4(u.x, t);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = t[i];
+        dec4(u.y, t);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[4 + i] = t[i];
+        dec4(u.z, t);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[8 + i] = t[i];
+        dec4(u.w, t);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[12 + i] = t[i];
+      } else if constexpr (BITS == 2) {
+        const uint2 u = *reinterpret_cast<const uint2*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 8);
+        float2 t[8];
+        dec2(u.x, t);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = t[i];
+        dec2(u.y, t);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[8 + i] = t[i];
+      } else {
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 12);
+        const uint32_t w0 = wp[0], w1 = wp[1], w2 = wp[2];
+        float2 t[8];
+        dec3(w0, w2, t);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = t[i];
+        dec3(w1, w2 >> 16, t);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[8 + i] = t[i];
+      }
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        float2 a0 = acc[sl][hd], a1 = make_float2(0.f, 0.f);
+        if constexpr (kRegP) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) {
+            a0 = __ffma2_rn(pr[hd][i], v[i], a0);
+            a1 = __ffma2_rn(pr[hd][i + 1], v[i + 1], a1);
+          }
+        } else {
+          const float4* p4 = reinterpret_cast<const float4*>(pp + hd * 128 + 32 * g);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 x = p4[q];
+            a0 = __ffma2_rn(make_float2(x.x, x.y), v[2 * q], a0);
+            a1 = __ffma2_rn(make_float2(x.z, x.w), v[2 * q + 1], a1);
+          }
+        }
+        acc[sl][hd] = __fadd2_rn(a0, a1);
       }
     }
   }
@@ -554,7 +637,7 @@ __device__ __forceinline__ void pv_raw(const unsigned char* st, const float* pp,
 
 template <int BITS, int G>
 __device__ __forceinline__ void pv_packed(const unsigned char* st, const float* pp, const float (&pg)[G][4],
-                                          float (&acc)[4][G], int lane) {
+                                          float2 (&acc)[4][G], int lane) {
   const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
   const uint8_t* meta = st + kMetaOffset;
   const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
@@ -606,53 +689,55 @@ __device__ __forceinline__ void pv_packed(const unsigned char* st, const float* 
             sum = fmaf(lo_mul, s1, sum);
           }
         }
-        acc[sl][hd] += sum;
+        acc[sl][hd].x += sum;
       }
     }
   }
 }
 
-// Writes this warp's partial sums for (b, h) and, if it is the last warp of
-// that (b, h) to do so, reduces all partials in warp order into `out`.
+// Writes this warp's partial sums for (b, h) to its slot (warp + bh) and clears them.
 template <int G>
-__device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float (&acc)[4][G], float (&mp)[G],
+__device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float2 (&acc)[4][G], float (&mp)[G],
                                          int lane) {
-  const long slot = warp + bh;
-  float* part = a.partials + (size_t)slot * G * 128;
+  float* part = a.partials + (size_t)(warp + bh) * G * 128;
 #pragma unroll
   for (int hd = 0; hd < G; ++hd) {
     const float mn = warp_sum(mp[hd]);
 #pragma unroll
-    for (int sl = 0; sl < 4; ++sl) __stcg(part + hd * 128 + sl * 32 + lane, acc[sl][hd] + mn);
-  }
-  __threadfence();
-  // warps that touch this (b, h): items [bh*I, (bh+1)*I) over ranges floor(w*N/W)
-  const long N = a.n_items, Wn = a.n_warps, I = a.items_per_bh;
-  auto warp_of = [&](long item) -> long { return (long)(((long long)(item + 1) * Wn + N - 1) / N) - 1; };
-  const long w0 = warp_of(bh * I), w1 = warp_of((bh + 1) * I - 1);
-  unsigned int prev = 0;
-  if (lane == 0) prev = atomicAdd(a.counters + bh, 1u);
-  prev = __shfl_sync(0xffffffffu, prev, 0);
-  if (prev == (unsigned int)(w1 - w0)) {
-    __threadfence();
-    const long b = bh / a.kv_heads, h = bh % a.kv_heads;
-#pragma unroll 1
-    for (int hd = 0; hd < G; ++hd) {
-#pragma unroll
-      for (int sl = 0; sl < 4; ++sl) {
-        float sum = 0.f;
-        for (long w = w0; w <= w1; ++w) sum += __ldcg(a.partials + (size_t)(w + bh) * G * 128 + hd * 128 + sl * 32 + lane);
-        a.out[((size_t)b * a.kv_heads * G + h * G + hd) * 128 + sl * 32 + lane] = sum;
-      }
+    for (int sl = 0; sl < 4; ++sl) {
+      __stcg(part + hd * 128 + sl * 32 + lane, acc[sl][hd].x + acc[sl][hd].y + mn);
+      acc[sl][hd] = make_float2(0.f, 0.f);
     }
-    if (lane == 0) a.counters[bh] = 0u;
-  }
-#pragma unroll
-  for (int hd = 0; hd < G; ++hd) {
     mp[hd] = 0.f;
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = 0.f;
   }
+}
+
+// Warp whose item range holds `item` (ranges are [floor(w*N/W), floor((w+1)*N/W)), W <= N).
+__device__ __forceinline__ long warp_of_item(long item, long n_items, long n_warps) {
+  return (long)(((long long)(item + 1) * n_warps + n_items - 1) / n_items) - 1;
+}
+
+// Second pass of p·V: out = sum of the partials of every warp that touched
+// (b, h), in warp order (deterministic).  One thread per output element; it is
+// launched as a programmatic dependent of pv_kernel and waits for its results.
+template <int G>
+__global__ void __launch_bounds__(256) pv_reduce_kernel(const GemvArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;  // ((b*kv_heads + h)*G + hd)*128 + c
+  if (t >= (long)a.batch * a.kv_heads * G * 128) return;
+  const long bh = t / (G * 128);
+  const long I = a.items_per_bh;
+  const long w0 = warp_of_item(bh * I, a.n_items, a.n_warps);
+  const long w1 = warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps);
+  const float* base = a.partials + (size_t)bh * G * 128 + (t - bh * G * 128);
+  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  long w = w0;
+  for (; w + 8 <= w1 + 1; w += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s[u] += __ldcg(base + (size_t)(w + u) * G * 128);
+  }
+  for (int u = 0; w <= w1; ++w, ++u) s[u] += __ldcg(base + (size_t)w * G * 128);
+  a.out[t] = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
 }
 
 template <int BITS, int G>
@@ -663,6 +748,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (warp >= a.n_warps) return;
   WarpMem<BITS, G, true> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const long lo = (long)((long long)a.n_items * warp / a.n_warps);
   const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
   if (lane == 0) {
@@ -671,21 +757,26 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
   }
   __syncwarp();
   long prod = lo;
-  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod) issue_item<BITS, G, true>(a, m, prod, s, lane);
+  Cursor pc{lo / a.items_per_bh, (int)(lo % a.items_per_bh)};
+  Cursor cc = pc;
+  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(a.items_per_bh))
+    issue_item<BITS, G, true>(a, m, pc, index_entry(a, pc), s, lane);
+  uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
 
-  float acc[4][G], mp[G];
+  float2 acc[4][G];
+  float mp[G];
 #pragma unroll
   for (int hd = 0; hd < G; ++hd) {
     mp[hd] = 0.f;
 #pragma unroll
-    for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = 0.f;
+    for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = make_float2(0.f, 0.f);
   }
-  long cur_bh = lo / a.items_per_bh;
+  long cur_bh = cc.bh;
   uint32_t phases = 0;
   int s = 0;
-  for (long x = lo; x < hi; ++x) {
-    const long bh = x / a.items_per_bh;
-    const int j = (int)(x % a.items_per_bh);
+  for (long x = lo; x < hi; ++x, cc.next(a.items_per_bh)) {
+    const long bh = cc.bh;
+    const int j = cc.j;
     if (bh != cur_bh) {
       pv_flush<G>(a, cur_bh, warp, acc, mp, lane);
       cur_bh = bh;
@@ -706,7 +797,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
         for (int hd = 0; hd < G; ++hd) {
           const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)a.n_blocks * 128 + t];
 #pragma unroll
-          for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = fmaf(pt, vv[sl], acc[sl][hd]);
+          for (int sl = 0; sl < 4; ++sl) acc[sl][hd].x = fmaf(pt, vv[sl], acc[sl][hd].x);
         }
       }
     } else if (kind == kKindInvalid) {
@@ -735,13 +826,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
           const float pprime = pr[i] * scr[i];
           ps += pprime;
           const int r = 4 * lane + i;  // storage slot
-          float e;
+          int sg;
           if constexpr (BITS == 4)
-            e = pow2(-sig4(r & 7));
+            sg = (r & 7) <= 4 ? 4 * (r & 7) : 4 * (r & 7) - 12;
           else
-            e = pow2(-sig2(r & 15));
-          // (r & 7) / (r & 15) depend only on lane parity classes; the exponent is exact
-          o[i] = kind == kKindRaw ? pprime * e : pprime;
+            sg = (r & 15) <= 10 ? 2 * (r & 15) : 2 * (r & 15) - 12;
+          o[i] = kind == kKindRaw ? pprime * exp2i(-sg) : pprime;  // exact power-of-two scaling
         }
         *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
         if (kind != kKindRaw) {
@@ -761,8 +851,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     }
     __syncwarp();
     if (prod < hi) {
-      issue_item<BITS, G, true>(a, m, prod, s, lane);
+      issue_item<BITS, G, true>(a, m, pc, next_e, s, lane);
       ++prod;
+      pc.next(a.items_per_bh);
+      if (prod < hi) next_e = index_entry(a, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
@@ -847,7 +939,28 @@ cudaError_t launch(GemvArgs a, cudaStream_t stream) {
   a.n_warps = (int)(a.n_items < w ? a.n_items : w);
   const unsigned grid = (unsigned)((a.n_warps + kWarpsPerCta - 1) / kWarpsPerCta);
   void* args[] = {&a};
-  return cudaLaunchKernel(info.fn, dim3(grid), dim3(kWarpsPerCta * 32), args, info.smem, stream);
+  e = cudaLaunchKernel(info.fn, dim3(grid), dim3(kWarpsPerCta * 32), args, info.smem, stream);
+  if (e != cudaSuccess || !PV) return e;
+  // second pass of p·V, launched early (programmatic dependent launch); it waits for pv_kernel
+  const long outputs = (long)a.batch * a.kv_heads * a.group * 128;
+  const void* red = nullptr;
+  switch (a.group) {
+    case 1: red = reinterpret_cast<const void*>(&pv_reduce_kernel<1>); break;
+    case 2: red = reinterpret_cast<const void*>(&pv_reduce_kernel<2>); break;
+    case 4: red = reinterpret_cast<const void*>(&pv_reduce_kernel<4>); break;
+    default: red = reinterpret_cast<const void*>(&pv_reduce_kernel<8>); break;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)((outputs + 255) / 256));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, red, args);
 }
 
 }  // namespace
@@ -860,8 +973,7 @@ int gemv_max_warps() {
 
 size_t pv_workspace_bytes(int batch, int kv_heads, int group) {
   const size_t bh = (size_t)batch * kv_heads;
-  const size_t counters = (bh * 4 + 255) / 256 * 256;
-  return counters + ((size_t)gemv_max_warps() + bh) * group * 128 * sizeof(float);
+  return ((size_t)gemv_max_warps() + bh) * group * 128 * sizeof(float);
 }
 
 cudaError_t launch_qk(GemvArgs a, cudaStream_t stream) { return launch<false>(a, stream); }

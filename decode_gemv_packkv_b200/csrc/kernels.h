@@ -45,7 +45,6 @@ struct GemvArgs {
   const float* p;         // row (b, hq) at (b*q_heads + hq) * ld
   float* out;             // [batch][q_heads][128]
   float* partials;        // [n_warps + batch*kv_heads][group][128]
-  uint32_t* counters;     // [batch*kv_heads], zero between calls
 };
 
 cudaError_t launch_qk(GemvArgs a, cudaStream_t stream);

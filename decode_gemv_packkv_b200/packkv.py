@@ -16,7 +16,7 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpackkv.so")
+LIB_PATH = os.environ.get("PACKKV_LIB") or os.path.join(_HERE, "libpackkv.so")
 
 BLOCK_TOKENS = 128
 HEAD_DIM = 128
@@ -165,7 +165,7 @@ class PackKVCache:
         return self.s.kv_heads
 
     def workspace(self, q_heads: int) -> torch.Tensor:
-        """Zero-initialised p·V workspace for q_heads (kept for reuse; calls leave it zeroed)."""
+        """p·V workspace for q_heads (allocated once, reused by every call)."""
         if q_heads not in self._ws:
             n = packkv_workspace_bytes(self, q_heads)
             self._ws[q_heads] = torch.zeros(max(n, 16), dtype=torch.uint8, device=self.k_arena.device)

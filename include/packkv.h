@@ -162,11 +162,9 @@ packkv_status packkv_qk_gemv(const packkv_cache* cache, const uint16_t* q, int32
  *   p:   device fp32, row (b, hq) at (b*q_heads + hq) * ld_p, ld_p >= T, multiple of 4.
  *   out: device fp32 [batch][q_heads][128].
  *   ws:  device, ws_bytes >= packkv_workspace_bytes(cache, q_heads): split-K
- *        partial sums over the sequence plus one counter per (sequence, kv
- *        head).  The caller zero-fills ws once before its first use; every
- *        completed call leaves the counters at zero again.  Partials are
- *        reduced in a fixed order, so results are deterministic on a given GPU.
- *        Two calls sharing one ws must not overlap in time.
+ *        partial sums over the sequence (no initialisation needed).  A second
+ *        kernel adds them in a fixed order, so results are deterministic on a
+ *        given GPU.  Two calls sharing one ws must not overlap in time.
  * With T == 0, out is set to zero.
  */
 packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t ld_p,

@@ -128,15 +128,14 @@ def test_pv_parity(pk, bits, group, structured):
     assert_within_terms(got2, ref2, terms2, "p·V (signed p)")
 
 
-def test_pv_is_deterministic_and_leaves_workspace_zeroed(pk):
+def test_pv_is_deterministic_with_a_dirty_workspace(pk):
     k, v, q = synth.small_case(12, 2, 4, 2, 20 * 128 + 3)
     cache, _ = _build(pk, k, v, 4, keep_perm=False)
     p = np.random.default_rng(0).random((2, 8, cache.tokens)).astype(np.float32)
     a = _pv(pk, cache, p)
+    cache.workspace(8).fill_(0xAB)     # garbage left by someone else: no initialisation needed
     b = _pv(pk, cache, p)
     assert np.array_equal(a, b)
-    ws = cache.workspace(8).cpu().numpy()
-    assert not ws[:2 * 4 * 4].any(), "counters not reset"
 
 
 def test_empty_cache(pk):
