@@ -266,9 +266,37 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       }
     }
   }
+  // raw records of b = 2 / 4: words in tensor-core fragment order (FORMAT.md section 4).
+  // A[m][k] = code of slot m, channel k (K) or of slot k, channel m (V).
+  if (a.bits != 3) {
+#pragma unroll
+    for (int tensor = 0; tensor < 2; ++tensor) {
+      if (!raw[tensor]) continue;
+      uint32_t* words = rec32[tensor] + kRawWordOffset / 4;
+      for (int wi = tid; wi < 512 * a.bits; wi += blockDim.x) {
+        const int q = wi & 3, lane = (wi >> 2) & 31, jj = (wi >> 7) & 1, tp = wi >> 8;
+        const int kappa = 4 * jj + q, g = lane >> 2, t = lane & 3;
+        uint32_t word = 0;
+        const int nfields = 32 / a.bits;
+        for (int f = 0; f < nfields; ++f) {
+          int e, kh, rh, tile;
+          if (a.bits == 4) {
+            e = f >> 2, kh = (f >> 1) & 1, rh = f & 1, tile = tp;
+          } else {
+            e = f >> 3, kh = (f >> 2) & 1, rh = f & 1, tile = 2 * tp + ((f >> 1) & 1);
+          }
+          const int m = 16 * tile + 8 * rh + g, k = 16 * kappa + 8 * kh + 2 * t + e;
+          const uint32_t code = tensor ? s.cv[s.perm[k]][m] : s.ck[s.perm[m]][k];
+          word |= code << (a.bits * f);
+        }
+        words[wi] = word;
+      }
+    }
+  }
   // pack the units: every word is owned by exactly one thread
   for (int u = tid; u < 2 * kGroups * kHeadDim; u += blockDim.x) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
+    if (raw[tensor] && a.bits != 3) continue;  // written above
     const uint8_t(*cx)[kHeadDim] = tensor ? s.cv : s.ck;
     const int w = raw[tensor] ? a.bits : s.width[tensor][g][c];
     const int base = raw[tensor] ? 0 : s.base[tensor][g][c];

@@ -42,7 +42,10 @@ namespace packkv {
 
 namespace {
 
-constexpr int kWarpsPerCta = 4;
+#ifndef PACKKV_WARPS_PER_CTA
+#define PACKKV_WARPS_PER_CTA 4
+#endif
+constexpr int kWarpsPerCta = PACKKV_WARPS_PER_CTA;
 #ifndef PACKKV_WARP_SMEM_KB
 #define PACKKV_WARP_SMEM_KB 10  // shared memory per warp: one stage, five CTAs of 4 warps per SM
 #endif
@@ -143,9 +146,15 @@ struct Cfg {
   static constexpr int kChunksPerGroup = kChunks / 4;
   static constexpr int kChanPerChunk = 128 / kChunksPerGroup;  // 64 (b=4) or 32
   static constexpr int kRecBytes = raw_record_bytes(BITS);
-  static constexpr int kStageRec = 528 + kChunks * kPitch;     // >= every record of this width
+  // b = 3 raw records are staged in padded chunks (bank-conflict-free CUDA-core decode);
+  // b = 2 / 4 raw records are already in fragment order and are staged in one piece
+  static constexpr bool kChunked = BITS == 3;
+  static constexpr int kStageRec = kChunked ? 528 + kChunks * kPitch : kRecBytes;  // >= every record
   static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);
-  static constexpr int kTableBytes = (PV ? 512 : 1024) * G;
+  static constexpr int kNT = (2 * G + 7) / 8;                  // MMA n-tiles: columns (head, hi/lo)
+  static constexpr int kBTabBytes = 8 * (64 * kNT + 4) * 4;    // [k-tile (padded)][t][column] uint2
+  static constexpr int kCoreTab = (PV ? 512 : 1024) * G;       // CUDA-core q'/p' table
+  static constexpr int kTableBytes = kCoreTab > kBTabBytes ? kCoreTab : kBTabBytes;
   static constexpr int kStages0 = (kWarpSmemBudget - kTableBytes - 64) / kStageBytes;
   static constexpr int kStages = kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0);
   static constexpr int kWarpSmem = ((kStages * kStageBytes + kTableBytes + kStages * 16) + 127) / 128 * 128;
@@ -242,10 +251,12 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const WarpMem<BITS
       mbar_arrive(m.bar(s));
   }
   __syncwarp();
-  if (kind == kKindRaw) {
+  if (kind == kKindRaw && C::kChunked) {
     if (lane < C::kChunks)
       bulk_g2s(st + 528 + lane * C::kPitch, src + 528 + lane * C::kChunkBytes, C::kChunkBytes, m.bar(s));
     if (lane == 16) bulk_g2s(st, src, 528, m.bar(s));
+  } else if (kind == kKindRaw) {
+    if (lane == 16) bulk_g2s(st, src, C::kRecBytes, m.bar(s));
   } else if (kind == kKindPacked) {
     if (lane == 16) bulk_g2s(st, src, len16 * 16u, m.bar(s));
   }
@@ -255,6 +266,278 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const WarpMem<BITS
     const long hq = h * G + hd;
     const float* prow = a.p + ((size_t)b * a.kv_heads * G + hq) * a.ld + (size_t)j * 128;
     bulk_g2s(st + C::kStageRec + hd * 512, prow, 512, m.bar(s));
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Tensor-core decode of raw b = 2 / 4 records (fragment order, FORMAT.md section 4)
+// ----------------------------------------------------------------------------
+// (w & MASK) | 0x64006400: two fields become fp16 1024 + field*2^shift, exactly.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t hfld(uint32_t w) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(0x64006400u));
+  return d;
+}
+
+// Exact field values from hfld: (1024 + field*2^k) * 2^-k - 1024 * 2^-k = field
+// (one fused fp16x2 FMA; every intermediate is an fp16 integer below 2048).
+template <uint32_t MASK, int K>
+__device__ __forceinline__ uint32_t hval(uint32_t w) {
+  const uint32_t bits = hfld<MASK>(w);
+  const __half2 x = *reinterpret_cast<const __half2*>(&bits);
+  const __half2 mul = __float2half2_rn(1.0f / float(1 << K));
+  const __half2 add = __float2half2_rn(-1024.0f / float(1 << K));
+  const __half2 r = __hfma2(x, mul, add);
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+// D += A(16x16, fp16) * B(16x8, fp16), fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Word offset of half kh of the B-table entry (k-tile kt, thread t, column n); the
+// k-tile stride is padded by 4 words so that the table's stores spread over banks.
+template <int NT>
+__device__ __forceinline__ int btab_word(int kt, int t, int n, int kh) {
+  return kt * (64 * NT + 4) + (t * 8 * NT + n) * 2 + kh;
+}
+
+// Per-block B operand of the MMA: column n = 2*head + part holds, for every k
+// (channel for q·Kᵀ, storage slot for p·V), the fp16 high (part 0) or low
+// (part 1) half of v[head][k] * f[head]; f is a power of two putting the head's
+// largest |v| in [2^14, 2^15).  Summing the two columns of a head restores v to
+// about 22 bits.  Table entry [k-tile][t][column] = {b0, b1} of the m16n8k16
+// fragment.  Lane holds v for k = 4*lane .. 4*lane+3.  Returns 1/f per head.
+template <int G, int NT>
+__device__ __forceinline__ void build_btab(uint32_t* btab, const float (&v)[G][4], float (&invf)[G], int lane) {
+  uint32_t pr[G][2][2];  // [head][part][pair]
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd) {
+    const float mx = warp_max(fmaxf(fmaxf(fabsf(v[hd][0]), fabsf(v[hd][1])), fmaxf(fabsf(v[hd][2]), fabsf(v[hd][3]))));
+    const int e = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 : 0;
+    const float f = mx > 0.f ? exp2i(14 - e) : 1.f;
+    invf[hd] = mx > 0.f ? exp2i(e - 14) : 1.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float x0 = v[hd][2 * q] * f, x1 = v[hd][2 * q + 1] * f;
+      const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+      const __half l0 = __float2half_rn(x0 - __half2float(h0)), l1 = __float2half_rn(x1 - __half2float(h1));
+      pr[hd][0][q] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+      pr[hd][1][q] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+    }
+  }
+  // live columns 0 .. 2G-1 only; columns 2G .. 8NT-1 stay zero (zero_btab).  The
+  // lane's column order is rotated by its k-tile so that one store instruction
+  // spreads over the banks instead of hitting the same bank eight times.
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int k = 4 * lane + 2 * q;  // even: the pair (k, k+1)
+    const int kt = k >> 4, kk = k & 15, kh = kk >> 3, t = (kk & 7) >> 1;
+    uint32_t* row = btab + btab_word<NT>(kt, t, 0, kh);
+#pragma unroll
+    for (int i = 0; i < 2 * G; ++i) {
+      const int n = (i + kt) % (2 * G);
+      uint32_t val = 0u;
+#pragma unroll
+      for (int c = 0; c < 2 * G; ++c)
+        if (n == c) val = pr[c >> 1][c & 1][q];
+      row[2 * n] = val;
+    }
+  }
+}
+
+// Zeroes the whole B table (the columns of absent heads must read as zero).
+template <int NT>
+__device__ __forceinline__ void zero_btab(uint32_t* btab, int lane) {
+  uint4* p = reinterpret_cast<uint4*>(btab);
+#pragma unroll
+  for (int i = lane; i < 8 * (64 * NT + 4) / 4; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
+}
+
+// Selects per-thread values of head 4*j + t (the head of MMA columns 2t, 2t+1 in n-tile j).
+template <int G>
+__device__ __forceinline__ float head_sel(const float (&x)[G], int head) {
+  float r = 0.f;
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd)
+    if (head == hd) r = x[hd];
+  return r;
+}
+
+// One raw b = 2 / 4 K block: scores of all 128 slots for the G heads.
+template <int BITS, int G>
+__device__ __forceinline__ void qk_tc(const unsigned char* st, const uint32_t* btab, const float (&cst)[G],
+                                      const float (&invf)[G], float* srow0, long ld,
+                                      float scale, int lane) {
+  constexpr int NT = (2 * G + 7) / 8;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t bf[NT][8][2];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+      const uint2 e = *reinterpret_cast<const uint2*>(btab + btab_word<NT>(kt, t, 8 * j + g, 0));
+      bf[j][kt][0] = e.x;
+      bf[j][kt][1] = e.y;
+    }
+  float c_t[NT], f_t[NT];
+  bool live[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int head = 4 * j + t;
+    live[j] = head < G;
+    c_t[j] = head_sel<G>(cst, head);
+    f_t[j] = head_sel<G>(invf, head);
+  }
+  // words (tile pair tp, k-tile kt) of this lane: uint4 index (tp*2 + kt/4)*32 + lane, component kt%4.
+  // Each k step issues the MMAs of 4 row tiles: 4 independent accumulator chains.
+  const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
+  constexpr int kWordTiles = BITS == 4 ? 4 : 2;  // word rows per half (b = 2: a word feeds two row tiles)
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    uint32_t w[kWordTiles][8];
+#pragma unroll
+    for (int u = 0; u < kWordTiles; ++u) {
+      const int tp = half * kWordTiles + u;
+      const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
+      w[u][0] = wa.x; w[u][1] = wa.y; w[u][2] = wa.z; w[u][3] = wa.w;
+      w[u][4] = wb.x; w[u][5] = wb.y; w[u][6] = wb.z; w[u][7] = wb.w;
+    }
+    float d[4][NT][4];  // 4 row tiles
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[u][j][i] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+#pragma unroll
+      for (int u = 0; u < kWordTiles; ++u) {
+        const uint32_t x = w[u][kt], h = x >> 8;
+        if constexpr (BITS == 4) {
+          const uint32_t r0 = hval<0x000F000Fu, 0>(x), r1 = hval<0x00F000F0u, 4>(x);
+          const uint32_t r2 = hval<0x000F000Fu, 0>(h), r3 = hval<0x00F000F0u, 4>(h);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) mma16816(d[u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
+        } else {
+          const uint32_t r0 = hval<0x00030003u, 0>(x), r1 = hval<0x000C000Cu, 2>(x);
+          const uint32_t r2 = hval<0x00030003u, 0>(h), r3 = hval<0x000C000Cu, 2>(h);
+          const uint32_t s0 = hval<0x00300030u, 4>(x), s1 = hval<0x00C000C0u, 6>(x);
+          const uint32_t s2 = hval<0x00300030u, 4>(h), s3 = hval<0x00C000C0u, 6>(h);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            mma16816(d[2 * u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
+            mma16816(d[2 * u + 1][j], s0, s1, s2, s3, bf[j][kt][0], bf[j][kt][1]);
+          }
+        }
+      }
+    }
+    // row tile u of this half covers slots 16*(4*half + u) + g and + 8
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (!live[j]) continue;
+      float* dst = srow0 + (4 * j + t) * ld;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = 16 * (4 * half + u) + g;
+        dst[r] = scale * fmaf(d[u][j][0] + d[u][j][1], f_t[j], c_t[j]);
+        dst[r + 8] = scale * fmaf(d[u][j][2] + d[u][j][3], f_t[j], c_t[j]);
+      }
+    }
+  }
+}
+
+// One raw b = 2 / 4 V block: adds sum_slots p'*v_hat into the per-thread fp32
+// accumulators of channels 16*T + g (acc_lo) and 16*T + g + 8 (acc_hi), head 4j + t.
+template <int BITS, int G>
+__device__ __forceinline__ void pv_tc(const unsigned char* st, const uint32_t* btab,
+                                      const float (&invf)[G], float (&acc_lo)[(2 * G + 7) / 8][8],
+                                      float (&acc_hi)[(2 * G + 7) / 8][8], int lane) {
+  constexpr int NT = (2 * G + 7) / 8;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t bf[NT][8][2];
+#pragma unroll
+  for (int j = 0; j < NT; ++j)
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+      const uint2 e = *reinterpret_cast<const uint2*>(btab + btab_word<NT>(kt, t, 8 * j + g, 0));
+      bf[j][kt][0] = e.x;
+      bf[j][kt][1] = e.y;
+    }
+  float f_t[NT];
+  bool live[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    live[j] = 4 * j + t < G;
+    f_t[j] = head_sel<G>(invf, 4 * j + t);
+  }
+  const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
+  constexpr int kWordTiles = BITS == 4 ? 4 : 2;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t w[kWordTiles][8];
+#pragma unroll
+    for (int u = 0; u < kWordTiles; ++u) {
+      const int tp = half * kWordTiles + u;
+      const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
+      w[u][0] = wa.x; w[u][1] = wa.y; w[u][2] = wa.z; w[u][3] = wa.w;
+      w[u][4] = wb.x; w[u][5] = wb.y; w[u][6] = wb.z; w[u][7] = wb.w;
+    }
+    float d[4][NT][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[u][j][i] = 0.f;
+#pragma unroll
+    for (int kt = 0; kt < 8; ++kt) {
+#pragma unroll
+      for (int u = 0; u < kWordTiles; ++u) {
+        const uint32_t x = w[u][kt], h = x >> 8;
+        if constexpr (BITS == 4) {
+          const uint32_t r0 = hval<0x000F000Fu, 0>(x), r1 = hval<0x00F000F0u, 4>(x);
+          const uint32_t r2 = hval<0x000F000Fu, 0>(h), r3 = hval<0x00F000F0u, 4>(h);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) mma16816(d[u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
+        } else {
+          const uint32_t r0 = hval<0x00030003u, 0>(x), r1 = hval<0x000C000Cu, 2>(x);
+          const uint32_t r2 = hval<0x00030003u, 0>(h), r3 = hval<0x000C000Cu, 2>(h);
+          const uint32_t s0 = hval<0x00300030u, 4>(x), s1 = hval<0x00C000C0u, 6>(x);
+          const uint32_t s2 = hval<0x00300030u, 4>(h), s3 = hval<0x00C000C0u, 6>(h);
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            mma16816(d[2 * u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
+            mma16816(d[2 * u + 1][j], s0, s1, s2, s3, bf[j][kt][0], bf[j][kt][1]);
+          }
+        }
+      }
+    }
+    // row tile u of this half covers channels 16*(4*half + u) + g and + 8
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      if (!live[j]) continue;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc_lo[j][4 * half + u] = fmaf(d[u][j][0] + d[u][j][1], f_t[j], acc_lo[j][4 * half + u]);
+        acc_hi[j][4 * half + u] = fmaf(d[u][j][2] + d[u][j][3], f_t[j], acc_hi[j][4 * half + u]);
+      }
+    }
   }
 }
 
@@ -475,6 +758,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
 
   const int q_heads = a.kv_heads * G;
   long cur_bh = -1;
+  bool btab_clean = false;  // the table region holds a B table whose absent-head columns are zero
   float qr[G][4];
   uint32_t phases = 0;
   int s = 0;
@@ -509,8 +793,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
       for (int hd = 0; hd < G; ++hd)
         for (int i = lane; i < 128; i += 32) srow0[hd * a.ld + (long)j * 128 + i] = __int_as_float(0x7fc00000);
     } else {
-      // per-block q' = q * scale_c (table) and the min term sum_c q_c * mn_c
-      float2* qp = reinterpret_cast<float2*>(m.table());
+      // per block: the min term sum_c q_c * mn_c, then q' = q * scale_c as the
+      // tensor-core B table (raw b = 2 / 4) or the CUDA-core q' table
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -518,6 +802,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
       const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&scv.x));
       const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&scv.y));
       float cst[G];
+      float qv[G][4];
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
         float part = qr[hd][0] * mn0.x;
@@ -525,16 +810,36 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
         part = fmaf(qr[hd][2], mn1.x, part);
         part = fmaf(qr[hd][3], mn1.y, part);
         cst[hd] = warp_sum(part);
-        const float q0 = qr[hd][0] * sc0.x, q1 = qr[hd][1] * sc0.y, q2 = qr[hd][2] * sc1.x, q3 = qr[hd][3] * sc1.y;
-        *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane)) = make_float4(q0, q0, q1, q1);
-        *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane + 2)) = make_float4(q2, q2, q3, q3);
+        qv[hd][0] = qr[hd][0] * sc0.x;
+        qv[hd][1] = qr[hd][1] * sc0.y;
+        qv[hd][2] = qr[hd][2] * sc1.x;
+        qv[hd][3] = qr[hd][3] * sc1.y;
       }
-      __syncwarp();
       float* sblk = srow0 + (long)j * 128;
-      if (kind == kKindRaw)
-        qk_raw<BITS, G>(st, qp, cst, sblk, a.ld, a.scale, lane);
-      else
-        qk_packed<BITS, G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+      if (kind == kKindRaw && !C::kChunked) {
+        uint32_t* btab = reinterpret_cast<uint32_t*>(m.table());
+        if (!btab_clean) zero_btab<C::kNT>(btab, lane);
+        btab_clean = true;
+        float invf[G];
+        build_btab<G, C::kNT>(btab, qv, invf, lane);
+        __syncwarp();
+        qk_tc<BITS, G>(st, btab, cst, invf, sblk, a.ld, a.scale, lane);
+      } else {
+        btab_clean = false;
+        float2* qp = reinterpret_cast<float2*>(m.table());
+#pragma unroll
+        for (int hd = 0; hd < G; ++hd) {
+          *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane)) =
+              make_float4(qv[hd][0], qv[hd][0], qv[hd][1], qv[hd][1]);
+          *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane + 2)) =
+              make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
+        }
+        __syncwarp();
+        if (kind == kKindRaw)
+          qk_raw<BITS, G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+        else
+          qk_packed<BITS, G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+      }
     }
     __syncwarp();
     if (prod < hi) {
@@ -695,21 +1000,44 @@ __device__ __forceinline__ void pv_packed(const unsigned char* st, const float* 
   }
 }
 
-// Writes this warp's partial sums for (b, h) to its slot (warp + bh) and clears them.
+// Writes this warp's partial sums for (b, h) to its slot (warp + bh) and clears
+// them.  The tensor-core accumulators (thread (g, t) holds channels 16T+g and
+// 16T+g+8 of head 4j+t) go through `buf` (G x 128 floats of warp shared memory)
+// to the lane = channel layout of the CUDA-core accumulators.
 template <int G>
-__device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float2 (&acc)[4][G], float (&mp)[G],
-                                         int lane) {
+__device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float2 (&acc)[4][G],
+                                         float (&acc_lo)[(2 * G + 7) / 8][8], float (&acc_hi)[(2 * G + 7) / 8][8],
+                                         float (&mp)[G], float* buf, int lane) {
+  constexpr int NT = (2 * G + 7) / 8;
+  const int g = lane >> 2, t = lane & 3;
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int head = 4 * j + t;
+#pragma unroll
+    for (int T = 0; T < 8; ++T) {
+      if (head < G) {
+        buf[head * 128 + 16 * T + g] = acc_lo[j][T];
+        buf[head * 128 + 16 * T + g + 8] = acc_hi[j][T];
+      }
+      acc_lo[j][T] = 0.f;
+      acc_hi[j][T] = 0.f;
+    }
+  }
+  __syncwarp();
   float* part = a.partials + (size_t)(warp + bh) * G * 128;
 #pragma unroll
   for (int hd = 0; hd < G; ++hd) {
     const float mn = warp_sum(mp[hd]);
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) {
-      __stcg(part + hd * 128 + sl * 32 + lane, acc[sl][hd].x + acc[sl][hd].y + mn);
+      const int c = sl * 32 + lane;
+      __stcg(part + hd * 128 + c, buf[hd * 128 + c] + acc[sl][hd].x + acc[sl][hd].y + mn);
       acc[sl][hd] = make_float2(0.f, 0.f);
     }
     mp[hd] = 0.f;
   }
+  __syncwarp();
 }
 
 // Warp whose item range holds `item` (ranges are [floor(w*N/W), floor((w+1)*N/W)), W <= N).
@@ -763,14 +1091,21 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     issue_item<BITS, G, true>(a, m, pc, index_entry(a, pc), s, lane);
   uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
 
-  float2 acc[4][G];
+  float2 acc[4][G];  // CUDA-core paths: lane = channel sl*32 + lane
   float mp[G];
+  float acc_lo[C::kNT][8], acc_hi[C::kNT][8];  // tensor-core path
 #pragma unroll
   for (int hd = 0; hd < G; ++hd) {
     mp[hd] = 0.f;
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = make_float2(0.f, 0.f);
   }
+#pragma unroll
+  for (int jn = 0; jn < C::kNT; ++jn)
+#pragma unroll
+    for (int T = 0; T < 8; ++T) acc_lo[jn][T] = acc_hi[jn][T] = 0.f;
+  float* buf = m.table();
+  bool btab_clean = false;  // the table region holds a B table whose absent-head columns are zero
   long cur_bh = cc.bh;
   uint32_t phases = 0;
   int s = 0;
@@ -778,7 +1113,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     const long bh = cc.bh;
     const int j = cc.j;
     if (bh != cur_bh) {
-      pv_flush<G>(a, cur_bh, warp, acc, mp, lane);
+      pv_flush<G>(a, cur_bh, warp, acc, acc_lo, acc_hi, mp, buf, lane);
+      btab_clean = false;  // the flush used the table region as its buffer
       cur_bh = bh;
     }
     const bool ok = mbar_wait_bounded(m.bar(s), (phases >> s) & 1u, a.ctrl);
@@ -803,8 +1139,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     } else if (kind == kKindInvalid) {
       if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
     } else {
-      // p' = p * scale_r (with the field exponent folded in for raw blocks) and the min term
-      float* pp = m.table();
+      // p' = p * scale_r per storage slot and the min term sum_r p_r * mn_r
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -813,41 +1148,56 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
       const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&scv.y));
       const float mnr[4] = {mn0.x, mn0.y, mn1.x, mn1.y};
       const float scr[4] = {sc0.x, sc0.y, sc1.x, sc1.y};
-      float pg[G][4];
+      float pv4[G][4];
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
         const float4 p4 = *reinterpret_cast<const float4*>(st + C::kStageRec + hd * 512 + 16 * lane);
         const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
-        float o[4];
-        float ps = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           mp[hd] = fmaf(pr[i], mnr[i], mp[hd]);
-          const float pprime = pr[i] * scr[i];
-          ps += pprime;
-          const int r = 4 * lane + i;  // storage slot
-          int sg;
-          if constexpr (BITS == 4)
-            sg = (r & 7) <= 4 ? 4 * (r & 7) : 4 * (r & 7) - 12;
-          else
-            sg = (r & 15) <= 10 ? 2 * (r & 15) : 2 * (r & 15) - 12;
-          o[i] = kind == kKindRaw ? pprime * exp2i(-sg) : pprime;  // exact power-of-two scaling
-        }
-        *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-        if (kind != kKindRaw) {
-          // per-group sum of p' (lanes 8g..8g+7 hold group g)
-          ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-          ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-          ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-#pragma unroll
-          for (int g = 0; g < 4; ++g) pg[hd][g] = __shfl_sync(0xffffffffu, ps, 8 * g);
+          pv4[hd][i] = pr[i] * scr[i];
         }
       }
-      __syncwarp();
-      if (kind == kKindRaw)
-        pv_raw<BITS, G>(st, pp, acc, lane);
-      else
-        pv_packed<BITS, G>(st, pp, pg, acc, lane);
+      if (kind == kKindRaw && !C::kChunked) {
+        uint32_t* btab = reinterpret_cast<uint32_t*>(m.table());
+        if (!btab_clean) zero_btab<C::kNT>(btab, lane);
+        btab_clean = true;
+        float invf[G];
+        build_btab<G, C::kNT>(btab, pv4, invf, lane);
+        __syncwarp();
+        pv_tc<BITS, G>(st, btab, invf, acc_lo, acc_hi, lane);
+      } else {
+        btab_clean = false;
+        float* pp = m.table();
+        float pg[G][4];
+#pragma unroll
+        for (int hd = 0; hd < G; ++hd) {
+          float o[4];
+          float ps = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            ps += pv4[hd][i];
+            const int r15 = (4 * lane + i) & 15;  // field position of slot r in a 2-bit slice word
+            const int sg = r15 <= 10 ? 2 * r15 : 2 * r15 - 12;
+            o[i] = kind == kKindRaw ? pv4[hd][i] * exp2i(-sg) : pv4[hd][i];  // exact power-of-two scaling
+          }
+          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+          if (kind != kKindRaw) {
+            // per-group sum of p' (lanes 8g..8g+7 hold group g)
+            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) pg[hd][g] = __shfl_sync(0xffffffffu, ps, 8 * g);
+          }
+        }
+        __syncwarp();
+        if (kind == kKindRaw)
+          pv_raw<BITS, G>(st, pp, acc, lane);
+        else
+          pv_packed<BITS, G>(st, pp, pg, acc, lane);
+      }
     }
     __syncwarp();
     if (prod < hi) {
@@ -858,7 +1208,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
-  pv_flush<G>(a, cur_bh, warp, acc, mp, lane);
+  pv_flush<G>(a, cur_bh, warp, acc, acc_lo, acc_hi, mp, buf, lane);
 }
 
 // ----------------------------------------------------------------------------

@@ -223,6 +223,44 @@ def record_bytes_max(bits: int) -> int:
     return raw_record_bytes(bits)
 
 
+def frag_word_bit(bits: int, m: int, k: int):
+    """(word index, bit offset) of A[m][k] in the raw fragment order (b = 2, 4).
+
+    Restates FORMAT.md section 4: m = 16T + 8rh + g, k = 16kappa + 8kh + 2t + e,
+    lane = 4g + t; the word is picked by (tile row T, kappa, lane) and the field
+    inside it by (e, kh, rh) (and the tile row parity for b = 2).
+    """
+    T, rh, g = m // 16, (m // 8) % 2, m % 8
+    kappa, kh, t, e = k // 16, (k // 8) % 2, (k % 8) // 2, k % 2
+    lane = 4 * g + t
+    J, Q = kappa // 4, kappa % 4
+    if bits == 4:
+        return ((T * 2 + J) * 32 + lane) * 4 + Q, 4 * (4 * e + 2 * kh + rh)
+    if bits == 2:
+        return (((T // 2) * 2 + J) * 32 + lane) * 4 + Q, 2 * (8 * e + 4 * kh + 2 * (T % 2) + rh)
+    raise ValueError("fragment order is defined for b = 2 and b = 4")
+
+
+def pack_raw_fragment(a: np.ndarray, bits: int) -> np.ndarray:
+    """Raw word area of a b = 2 / 4 record: every code of the 128x128 matrix A at its place."""
+    words = [0] * (512 * bits)
+    for m in range(128):
+        for k in range(128):
+            w, bit = frag_word_bit(bits, m, k)
+            words[w] |= int(a[m, k]) << bit
+    return np.array(words, dtype=np.uint64).astype(np.uint32)
+
+
+def unpack_raw_fragment(words: np.ndarray, bits: int) -> np.ndarray:
+    a = np.zeros((128, 128), np.int64)
+    mask = (1 << bits) - 1
+    for m in range(128):
+        for k in range(128):
+            w, bit = frag_word_bit(bits, m, k)
+            a[m, k] = (int(words[w]) >> bit) & mask
+    return a
+
+
 def _ceil16(n: int) -> int:
     return (n + 15) // 16 * 16
 
@@ -250,6 +288,9 @@ def build_record(codes_slot: np.ndarray, mn16: np.ndarray, sc16: np.ndarray,
             offs = codes_slot[32 * g:32 * g + 32, c] - base[g, c]
             words.append(pack_unit(offs, int(width[g, c])))
     all_words = np.concatenate(words).astype(np.uint32) if words else np.zeros(0, np.uint32)
+    if raw and bits in (2, 4):
+        # same header values, word area in tensor-core fragment order (K: rows = slots, V: rows = channels)
+        all_words = pack_raw_fragment(codes_slot.T if is_v else codes_slot, bits)
     flags = (RAW_FLAG if raw else 0) | (V_FLAG if is_v else 0) | (FORMAT_VERSION << 8) | (bits << 16)
     out = bytearray()
     out += struct.pack("<4H", *group_start)
@@ -300,6 +341,10 @@ def parse_record(rec: bytes) -> ParsedRecord:
         width = meta >> 4
         word_at = 1040
     words = np.frombuffer(rec, dtype="<u4", count=total_words, offset=word_at).astype(np.uint64)
+    if raw and bits in (2, 4):
+        a = unpack_raw_fragment(words, bits)
+        codes = a.T.copy() if is_v else a
+        return ParsedRecord(raw, is_v, bits, mn, sc, base, width, codes, gws)
     codes = np.zeros((128, 128), np.int64)
     at = 0
     for g in range(4):

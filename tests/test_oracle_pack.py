@@ -172,3 +172,36 @@ def test_cache_append_equals_block_encode():
     assert np.array_equal(a.k_index[:, :, :2, 0].transpose(0, 1, 2).reshape(-1),
                           np.concatenate([[0], np.cumsum(lens)[:-1]]))
     assert offs[-1] + lens[-1] == len(a.k_arena) // 16
+
+
+def test_raw_fragment_order_hand_words(golden_dir):
+    for line in _lines(os.path.join(golden_dir, "raw_fragment_words.txt")):
+        bits, idx, want = (t.strip() for t in line.split("|"))
+        bits, idx = int(bits), int(idx)
+        a = np.fromfunction(lambda m, k: (m + 2 * k) % (1 << bits), (128, 128), dtype=np.int64)
+        assert int(O.pack_raw_fragment(a, bits)[idx]) == int(want, 16), line
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_raw_fragment_order_is_a_bijection(bits):
+    seen = set()
+    for m in range(128):
+        for k in range(128):
+            w, bit = O.frag_word_bit(bits, m, k)
+            assert 0 <= w < 512 * bits and bit % bits == 0 and bit + bits <= 32
+            seen.add((w, bit))
+    assert len(seen) == 128 * 128
+    rng = np.random.default_rng(bits)
+    a = rng.integers(0, 1 << bits, (128, 128))
+    assert np.array_equal(O.unpack_raw_fragment(O.pack_raw_fragment(a, bits), bits), a)
+
+
+def test_raw_v_record_stores_the_transpose():
+    """In a V record the fragment rows are channels: word 0's first field is code[slot 0][channel 0],
+    its rh field (row 8) is code[slot 0][channel 8]."""
+    k, v, _ = synth.small_case(31, 1, 1, 1, 128)
+    _, v_rec, perm = O.encode_block(k[0, 0], v[0, 0], 4)
+    assert len(v_rec) == O.raw_record_bytes(4)
+    codes = O.quantize_block_v(v[0, 0], 4)[0][perm]      # [slot, channel]
+    w0 = int(np.frombuffer(v_rec, "<u4", 1, 528)[0])
+    assert w0 & 0xF == codes[0, 0] and (w0 >> 4) & 0xF == codes[0, 8] and (w0 >> 16) & 0xF == codes[1, 0]
