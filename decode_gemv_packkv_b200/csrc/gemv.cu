@@ -1326,6 +1326,18 @@ size_t pv_workspace_bytes(int batch, int kv_heads, int group) {
   return ((size_t)gemv_max_warps() + bh) * group * 128 * sizeof(float);
 }
 
+cudaError_t pv_launch_workspace_bytes(const GemvArgs& a, size_t* bytes) {
+  KernelInfo info{};
+  if (!select<true>(a.bits, a.group, &info)) return cudaErrorInvalidValue;
+  int w = 0;
+  const cudaError_t e = resident_warps(info, &w);
+  if (e != cudaSuccess) return e;
+  if (w > gemv_max_warps()) w = gemv_max_warps();
+  const long n_warps = a.n_items < w ? a.n_items : w;
+  *bytes = ((size_t)n_warps + (size_t)a.batch * a.kv_heads) * a.group * 128 * sizeof(float);
+  return cudaSuccess;
+}
+
 cudaError_t launch_qk(GemvArgs a, cudaStream_t stream) { return launch<false>(a, stream); }
 cudaError_t launch_pv(GemvArgs a, cudaStream_t stream) { return launch<true>(a, stream); }
 

@@ -54,5 +54,7 @@ cudaError_t launch_pv(GemvArgs a, cudaStream_t stream);
 // for workspace sizing), and the workspace layout of p·V.
 int gemv_max_warps();
 size_t pv_workspace_bytes(int batch, int kv_heads, int group);
+// Workspace bytes the launch of `a` by launch_pv would use (n_warps chosen as launch_pv does).
+cudaError_t pv_launch_workspace_bytes(const GemvArgs& a, size_t* bytes);
 
 }  // namespace packkv

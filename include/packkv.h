@@ -170,6 +170,29 @@ packkv_status packkv_qk_gemv(const packkv_cache* cache, const uint16_t* q, int32
 packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t ld_p,
                              int32_t q_heads, float* out, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * p·V without a caller-provided workspace.  (The PackKV pages have no
+ * counterpart: this is a calling convention, not part of the method.)
+ * For callers that cannot allocate device memory: runtimes that reserve all
+ * device memory at start-up and forbid later allocations, hosts without a
+ * device allocator to pass in, or decode loops that must not call cudaMalloc
+ * because it synchronises the device.
+ * Same arguments and result as packkv_pv_gemv minus ws/ws_bytes.  The split-K
+ * partials live in a static device array of PACKKV_PV_NOALLOC_SCRATCH_BYTES
+ * that every GPU loading the library holds until the process exits; the call
+ * allocates nothing.  Returns PACKKV_ERR_CAPACITY, without launching, if the
+ * call would need more scratch than that (the need is packkv_workspace_bytes-
+ * like: (resident warps + batch*kv_heads) * G * 512 bytes; e.g. G <= 4 fits
+ * for up to about 1000 (sequence, kv head) pairs on a B200).  The first call
+ * on a device looks up the array's device address (a one-time set-up); make
+ * that first call before any stream capture.  All calls share the one array:
+ * calls that overlap in time on the GPU race.  Nothing in it needs clearing.
+ */
+#define PACKKV_PV_NOALLOC_SCRATCH_BYTES (8u << 20)
+size_t packkv_pv_noalloc_scratch_bytes(void);
+packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, int64_t ld_p,
+                                     int32_t q_heads, float* out, void* stream);
+
 /* Synchronises `stream`, returns PACKKV_OK if no device status bit is set,
  * else PACKKV_ERR_CAPACITY (capacity bit set) or PACKKV_ERR_DEVICE; stores
  * the bits in *bits_out (if not NULL) and clears them. */
