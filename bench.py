@@ -58,6 +58,18 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
+def job_value(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: the tokens every rank decoded in one step over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step * 1e-3)
+
+
+# kernels of this library launched by one step: q·Kᵀ (1), p·V (2: the split pass and its reduce)
+KERNELS_PER_STEP = 3
+
+# wall-clock budget of the reference arm (warm-up + timed steps), seconds
+REFERENCE_SECONDS = 150.0
+
+
 def barrier(device=None):
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
@@ -317,7 +329,7 @@ def run_ours(args):
     cr_v = fp16_bytes / (v_used + index_bytes)
     plain = 128 * 128 * 2 / (128 * 128 * bits / 8 + 512)
     result = {
-        "metric": METRIC, "value": world * B * T / (ms_per_step * 1e-3), "unit": UNIT, "n_gpus": world,
+        "metric": METRIC, "value": job_value(world, B * T, ms_per_step), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": warm * R, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; K per-channel N(mu,sigma) with outlier "
                                                        "channels, V N(0,1)); no weights needed",
@@ -343,10 +355,10 @@ def run_ours(args):
                      "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s", "frac": dom_gbs / hbm_peak,
                      "traffic": None, "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": dom_ms,
                      "peak_source": peak_note},
-        "e2e": {"value": world * B * T / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": job_value(world, B * T, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": int(q_host.numel() * 2), "d2h_bytes_per_step": int(out_host.numel() * 4),
                 "note": "pinned q H2D, q·Kᵀ, softmax (torch, the caller's step), p·V, out D2H, stream sync"},
-        "gpu_launches": 2 * K,
+        "gpu_launches": KERNELS_PER_STEP * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -407,7 +419,7 @@ def run_reference(args):
     # size each step's sample so that warmup + steps take a few minutes at most
     cache, q = oracle_step_sample(w, bits, 1)
     one = oracle_gemv_seconds(cache, q)
-    n_blocks = int(max(1, min(64, 150.0 / max(1, args.steps + args.warmup) / max(one, 1e-4))))
+    n_blocks = int(max(1, min(64, REFERENCE_SECONDS / max(1, args.steps + args.warmup) / max(one, 1e-4))))
     cache, q = oracle_step_sample(w, bits, n_blocks)
     for _ in range(args.warmup):
         oracle_gemv_seconds(cache, q)
