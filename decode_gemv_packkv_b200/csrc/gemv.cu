@@ -1046,26 +1046,46 @@ __device__ __forceinline__ long warp_of_item(long item, long n_items, long n_war
 }
 
 // Second pass of p·V: out = sum of the partials of every warp that touched
-// (b, h), in warp order (deterministic).  One thread per output element; it is
-// launched as a programmatic dependent of pv_kernel and waits for its results.
+// (b, h), in a fixed order (deterministic).  One CTA per output row (b, h, head):
+// warp i of 8 adds partial slots w0+i, w0+i+8, ... with coalesced 16-byte loads,
+// then warp 0 adds the 8 warp sums in order.  It is launched as a programmatic
+// dependent of pv_kernel and waits for its results.
 template <int G>
 __global__ void __launch_bounds__(256) pv_reduce_kernel(const GemvArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;  // ((b*kv_heads + h)*G + hd)*128 + c
-  if (t >= (long)a.batch * a.kv_heads * G * 128) return;
-  const long bh = t / (G * 128);
+  __shared__ float4 warp_sum4[8][32];
+  const long row = blockIdx.x;  // (b*kv_heads + h)*G + head
+  const long bh = row / G;
+  const int hd = (int)(row % G);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long I = a.items_per_bh;
   const long w0 = warp_of_item(bh * I, a.n_items, a.n_warps);
   const long w1 = warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps);
-  const float* base = a.partials + (size_t)bh * G * 128 + (t - bh * G * 128);
-  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  long w = w0;
-  for (; w + 8 <= w1 + 1; w += 8) {
-#pragma unroll
-    for (int u = 0; u < 8; ++u) s[u] += __ldcg(base + (size_t)(w + u) * G * 128);
+  const float4* base = reinterpret_cast<const float4*>(a.partials + ((size_t)bh * G + hd) * 128) + lane;
+  const size_t slot_stride = (size_t)G * 128 / 4;  // float4 per partial slot
+  float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+  long w = w0 + warp;
+  for (; w + 8 <= w1; w += 16) {
+    const float4 x = __ldcg(base + (size_t)w * slot_stride);
+    const float4 y = __ldcg(base + (size_t)(w + 8) * slot_stride);
+    s0.x += x.x; s0.y += x.y; s0.z += x.z; s0.w += x.w;
+    s1.x += y.x; s1.y += y.y; s1.z += y.z; s1.w += y.w;
   }
-  for (int u = 0; w <= w1; ++w, ++u) s[u] += __ldcg(base + (size_t)w * G * 128);
-  a.out[t] = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+  if (w <= w1) {
+    const float4 x = __ldcg(base + (size_t)w * slot_stride);
+    s0.x += x.x; s0.y += x.y; s0.z += x.z; s0.w += x.w;
+  }
+  warp_sum4[warp][lane] = make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+  __syncthreads();
+  if (warp == 0) {
+    float4 r = warp_sum4[0][lane];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+      const float4 x = warp_sum4[i][lane];
+      r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
+    }
+    reinterpret_cast<float4*>(a.out + row * 128)[lane] = r;
+  }
 }
 
 template <int BITS, int G>
@@ -1292,7 +1312,7 @@ cudaError_t launch(GemvArgs a, cudaStream_t stream) {
   e = cudaLaunchKernel(info.fn, dim3(grid), dim3(kWarpsPerCta * 32), args, info.smem, stream);
   if (e != cudaSuccess || !PV) return e;
   // second pass of p·V, launched early (programmatic dependent launch); it waits for pv_kernel
-  const long outputs = (long)a.batch * a.kv_heads * a.group * 128;
+  const long rows = (long)a.batch * a.kv_heads * a.group;
   const void* red = nullptr;
   switch (a.group) {
     case 1: red = reinterpret_cast<const void*>(&pv_reduce_kernel<1>); break;
@@ -1301,7 +1321,7 @@ cudaError_t launch(GemvArgs a, cudaStream_t stream) {
     default: red = reinterpret_cast<const void*>(&pv_reduce_kernel<8>); break;
   }
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)((outputs + 255) / 256));
+  cfg.gridDim = dim3((unsigned)rows);
   cfg.blockDim = dim3(256);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
