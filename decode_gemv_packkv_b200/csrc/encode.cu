@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       }
     }
   }
-  // raw records of b = 2 / 4: words in tensor-core fragment order (FORMAT.md section 4).
+  // raw records of b = 2 / 4: words in 8-bit tensor-core fragment order (FORMAT.md section 4).
   // A[m][k] = code of slot m, channel k (K) or of slot k, channel m (V).
   if (a.bits != 3) {
 #pragma unroll
@@ -274,18 +274,19 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       if (!raw[tensor]) continue;
       uint32_t* words = rec32[tensor] + kRawWordOffset / 4;
       for (int wi = tid; wi < 512 * a.bits; wi += blockDim.x) {
-        const int q = wi & 3, lane = (wi >> 2) & 31, jj = (wi >> 7) & 1, tp = wi >> 8;
-        const int kappa = 4 * jj + q, g = lane >> 2, t = lane & 3;
+        // wi = ((tile row or tile pair)*2 + J)*32 + lane)*4 + 2*Q2 + kh, kappa = 2J + Q2
+        const int kh = wi & 1, q2 = (wi >> 1) & 1, lane = (wi >> 2) & 31, jj = (wi >> 7) & 1, tp = wi >> 8;
+        const int kappa = 2 * jj + q2, g = lane >> 2, t = lane & 3;
         uint32_t word = 0;
         const int nfields = 32 / a.bits;
         for (int f = 0; f < nfields; ++f) {
-          int e, kh, rh, tile;
+          int e, rh, tile;
           if (a.bits == 4) {
-            e = f >> 2, kh = (f >> 1) & 1, rh = f & 1, tile = tp;
+            e = f >> 1, rh = f & 1, tile = tp;
           } else {
-            e = f >> 3, kh = (f >> 2) & 1, rh = f & 1, tile = 2 * tp + ((f >> 1) & 1);
+            e = f >> 2, rh = f & 1, tile = 2 * tp + ((f >> 1) & 1);
           }
-          const int m = 16 * tile + 8 * rh + g, k = 16 * kappa + 8 * kh + 2 * t + e;
+          const int m = 16 * tile + 8 * rh + g, k = 32 * kappa + 16 * kh + 4 * t + e;
           const uint32_t code = tensor ? s.cv[s.perm[k]][m] : s.ck[s.perm[m]][k];
           word |= code << (a.bits * f);
         }
@@ -398,9 +399,6 @@ __global__ void __launch_bounds__(1024) arena_scan_kernel(EncodeArgs a) {
       // neither arena advances; the write pass skips the whole call
       a.ctrl[kCtrlScratch] = 1ull;
       set_status(a.ctrl, PACKKV_DEV_CAPACITY);
-      for (int tensor = 0; tensor < 2; ++tensor) {
-        (void)tensor;
-      }
     } else {
       a.ctrl[kCtrlScratch] = 0ull;
       a.ctrl[kCtrlKEnd] += totals[0];

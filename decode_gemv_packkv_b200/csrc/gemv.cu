@@ -1,7 +1,7 @@
 // Fused decompression + matrix-vector products over the packed cache
-// (PackKV paper page, Figure 2 "computation-aware decompression + matrix-vector
-// multiplication", TL;DR: decompression integrated into the GEMV with no
-// write-back of decompressed data; Figure 1: the two decode products).
+// (PackKV paper page, Figure 2: the decompression is folded into the
+// matrix-vector multiplication; TL;DR: no decompressed data is written back;
+// Figure 1: the two products of decode attention).
 //
 //   q·Kᵀ : scores[b,hq,i] = scale * sum_c q[b,hq,c] * k_hat[b,h,i,c]
 //   p·V  : out[b,hq,c]    = sum_i p[b,hq,i] * v_hat[b,h,i,c]
@@ -13,23 +13,25 @@
 //    heads of the kv head and neighbouring warps stream neighbouring records.
 //  * Each warp runs its own STAGES-deep pipeline of shared-memory stages filled
 //    by the bulk-copy engine (cp.async.bulk + mbarrier complete_tx; never
-//    multicast).  A raw record is copied as a header/params piece plus 8 or 16
-//    chunks at a padded pitch, so that the lanes' 32-bit reads of packed words
-//    fall in distinct banks.  A compressed record is copied in one piece.
-//  * Dequantization is folded out of the inner loop: k_hat = mn_c + s_c*(base+off)
-//    gives score = scale*(sum_c q_c mn_c + sum_c (q_c s_c) base + sum_c (q_c s_c) off);
-//    v_hat = mn_r + s_r*(base+off) gives out_c = sum_r p_r mn_r + sum_r (p_r s_r)(base+off).
-//    The inner loop is one LOP3 (mask | 0x4B000000: the field becomes the low
-//    mantissa bits of 2^23 + field*2^k), one FADD (removes 2^23 exactly) and one
-//    FFMA per element and query head.  The power of two 2^k of each field
-//    position is undone once per token (q·Kᵀ) or folded into p (p·V).
-//  * q·Kᵀ: lanes split (group, token word, channel range); each lane keeps fp32
-//    accumulators for 8 or 16 tokens and a 2- or 4-way shuffle sum finishes.
-//  * p·V: lane = channel; a warp sums its item range into per-channel fp32
-//    partials and writes them to the workspace at every (sequence, head)
-//    boundary (split-K over the sequence); a second-pass kernel, launched as a
-//    programmatic dependent so its launch overlaps the first, adds the partials
-//    of each (sequence, head) in warp order: deterministic.
+//    multicast).
+//  * Dequantization is folded out of the inner loop: k_hat = mn_c + s_c*code
+//    gives score = scale*(sum_c q_c mn_c + sum_c (q_c s_c) code); v_hat =
+//    mn_r + s_r*code gives out_c = sum_r p_r mn_r + sum_r (p_r s_r) code.
+//  * Raw 2/4-bit records (the common case) hold their codes in the fragment
+//    order of an 8-bit integer tensor-core operand: one AND per 32-bit word
+//    yields a whole A register of four codes (times a known power of two), and
+//    mma.sync m16n8k32 (u8 x s8 -> s32, exact) multiplies them by q' or p'
+//    written as three base-128 digits of q'*f (f = 127 / max|q'| per record and
+//    head; about 22 significant bits, the digits in three B columns).
+//  * 3-bit raw records and compressed (frame-of-reference) records are decoded
+//    on the CUDA cores: magic-number decode (LOP3 into the mantissa of 2^23,
+//    packed FP32 add) for raw 3-bit units, per-unit field extraction for
+//    compressed units.
+//  * p·V: a warp sums its item range into per-channel fp32 partials and writes
+//    them to the workspace at every (sequence, head) boundary (split-K over the
+//    sequence); a second-pass kernel, launched as a programmatic dependent so
+//    its launch overlaps the first, adds the partials of each (sequence, head)
+//    in warp order: deterministic.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -47,17 +49,15 @@ namespace {
 #endif
 constexpr int kWarpsPerCta = PACKKV_WARPS_PER_CTA;
 #ifndef PACKKV_WARP_SMEM_KB
-#define PACKKV_WARP_SMEM_KB 10  // shared memory per warp: one stage, five CTAs of 4 warps per SM
+#define PACKKV_WARP_SMEM_KB 10  // shared memory per warp: one 4-bit stage, five CTAs of 4 warps per SM
 #endif
 constexpr int kWarpSmemBudget = PACKKV_WARP_SMEM_KB * 1024;
 constexpr uint32_t kMagicBits = 0x4B000000u;
 constexpr float kMagic = 8388608.0f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer in the low bits
+constexpr int kRoundBits = 0x4B400000;
 
 enum ItemKind : int { kKindRaw = 0, kKindPacked = 1, kKindInvalid = 2, kKindTail = 3 };
-
-__device__ __forceinline__ float mag(uint32_t field_bits) {
-  return __uint_as_float(field_bits | kMagicBits) - kMagic;
-}
 
 // (w & mask) | 0x4B000000 in one LOP3: the field lands in the low mantissa bits of 2^23.
 template <uint32_t MASK>
@@ -72,23 +72,13 @@ __device__ __forceinline__ float2 pairf(uint32_t a, uint32_t b) {
   return __fadd2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), make_float2(-kMagic, -kMagic));
 }
 
-// Field position exponents of the in-register decode (value = field * 2^sig).
-__host__ __device__ constexpr int sig4(int i) { return i <= 4 ? 4 * i : 4 * i - 12; }
+// Field position exponent of token i (0..15) in the 2-bit decode below (value = field * 2^sig2).
 __host__ __device__ constexpr int sig2(int i) { return i <= 10 ? 2 * i : 2 * i - 12; }
 __host__ __device__ constexpr float pow2(int e) {
   return e >= 0 ? float(1u << e) : 1.0f / float(1u << (-e));
 }
 // 2^e for a run-time e in [-126, 127], from the exponent bits (no division)
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
-
-// 8 nibbles of a 4-bit slice word as 4 pairs: v[p] = (field_2p * 2^sig4(2p), field_2p+1 * 2^sig4(2p+1))
-__device__ __forceinline__ void dec4(uint32_t w, float2 (&v)[4]) {
-  const uint32_t h = w >> 12;
-  v[0] = pairf(fld<0xFu>(w), fld<0xF0u>(w));
-  v[1] = pairf(fld<0xF00u>(w), fld<0xF000u>(w));
-  v[2] = pairf(fld<0xF0000u>(w), fld<0xF00u>(h));
-  v[3] = pairf(fld<0xF000u>(h), fld<0xF0000u>(h));
-}
 
 template <int I>
 __device__ __forceinline__ uint32_t fld2(uint32_t w, uint32_t h) {
@@ -123,57 +113,62 @@ __device__ __forceinline__ void dec3(uint32_t w2, uint32_t x, float2 (&v)[8]) {
   }
 }
 
-template <int BITS>
-struct RawLayout;
-template <>
-struct RawLayout<4> {
-  static constexpr int kChunks = 8, kChunkBytes = 1024;
-};
-template <>
-struct RawLayout<3> {
-  static constexpr int kChunks = 16, kChunkBytes = 384;
-};
-template <>
-struct RawLayout<2> {
-  static constexpr int kChunks = 16, kChunkBytes = 256;
-};
-
 template <int BITS, int G, bool PV>
 struct Cfg {
-  static constexpr int kChunks = RawLayout<BITS>::kChunks;
-  static constexpr int kChunkBytes = RawLayout<BITS>::kChunkBytes;
-  static constexpr int kPitch = kChunkBytes + 16;
-  static constexpr int kChunksPerGroup = kChunks / 4;
-  static constexpr int kChanPerChunk = 128 / kChunksPerGroup;  // 64 (b=4) or 32
   static constexpr int kRecBytes = raw_record_bytes(BITS);
-  // b = 3 raw records are staged in padded chunks (bank-conflict-free CUDA-core decode);
-  // b = 2 / 4 raw records are already in fragment order and are staged in one piece
+  // b = 3 raw records are staged as 16 chunks (group g, channel quarter h: 32 units of
+  // 3 words) at a padded pitch (bank-conflict-free decode); b = 2 / 4 raw records are
+  // in fragment order and are staged in one piece, as are compressed records.
   static constexpr bool kChunked = BITS == 3;
+  static constexpr int kChunks = 16, kChunkBytes = 384, kPitch = 400;
   static constexpr int kStageRec = kChunked ? 528 + kChunks * kPitch : kRecBytes;  // >= every record
-  static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);
-  static constexpr int kNT = (2 * G + 7) / 8;                  // MMA n-tiles: columns (head, hi/lo)
-  static constexpr int kBTabBytes = 8 * (64 * kNT + 4) * 4;    // [k-tile (padded)][t][column] uint2
-  static constexpr int kCoreTab = (PV ? 512 : 1024) * G;       // CUDA-core q'/p' table
-  static constexpr int kTableBytes = kCoreTab > kBTabBytes ? kCoreTab : kBTabBytes;
-  static constexpr int kStages0 = (kWarpSmemBudget - kTableBytes - 64) / kStageBytes;
+  static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);              // p·V: + p rows
+  // int8 tensor-core B table: columns n = 4*head + digit (digit 3 = 0), NT n-tiles of 8
+  static constexpr int kNT = (4 * G + 7) / 8;
+  static constexpr int kI8Tab = 4 * (64 * kNT + 8) * 4;
+  // CUDA-core tables: q' pairs [G][128] (q·Kᵀ); p'' [G][128] + group sums of p' [G][4] (p·V)
+  static constexpr int kCoreTab = PV ? 512 * G + 16 * G : 1024 * G;
+  static constexpr int kTableBytes = ((kCoreTab > kI8Tab ? kCoreTab : kI8Tab) + 15) / 16 * 16;
+  static constexpr int kSumBytes = PV ? 512 * G : 0;          // p·V: [G][128] channel sums
+  static constexpr int kFixed = kTableBytes + kSumBytes;
+  static constexpr int kStages0 = (kWarpSmemBudget - kFixed - 64) / kStageBytes;
   static constexpr int kStages = kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0);
-  static constexpr int kWarpSmem = ((kStages * kStageBytes + kTableBytes + kStages * 16) + 127) / 128 * 128;
-  // q' table: channel c = h*kChanPerChunk + cc stored at ((cc/4)*NH + h)*4 + cc%4
-  static constexpr int kNH = 128 / kChanPerChunk;
+  static constexpr int kWarpSmem = ((kStages * kStageBytes + kFixed + kStages * 16) + 127) / 128 * 128;
+  static_assert(kStageBytes % 16 == 0 && kFixed % 16 == 0, "stage alignment");
 };
 
-// q' table of q·Kᵀ: (q'_c, q'_c) pairs; channel c = h*kChanPerChunk + cc sits at float2
-// index ((cc/2)*NH + h)*2 + cc%2, so one 16-byte load gives a lane its next two channels.
+// Warp-private shared memory: [stages][table][channel sums (p·V)][mbarriers][kinds].
 template <int BITS, int G, bool PV>
-__device__ __forceinline__ int table_index(int c) {
+struct WarpMem {
   using C = Cfg<BITS, G, PV>;
-  const int h = c / C::kChanPerChunk, cc = c % C::kChanPerChunk;
-  return ((cc >> 1) * C::kNH + h) * 2 + (cc & 1);
+  unsigned char* base;
+  __device__ unsigned char* stage(int s) const { return base + s * C::kStageBytes; }
+  __device__ unsigned char* fixed() const { return base + C::kStages * C::kStageBytes; }
+  __device__ uint32_t* table() const { return reinterpret_cast<uint32_t*>(fixed()); }
+  __device__ float* sums() const { return reinterpret_cast<float*>(fixed() + C::kTableBytes); }
+  __device__ uint64_t* bar(int s) const { return reinterpret_cast<uint64_t*>(fixed() + C::kFixed) + s; }
+  __device__ int* kind(int s) const {
+    return reinterpret_cast<int*>(fixed() + C::kFixed + C::kStages * 8) + s;
+  }
+};
+
+// CUDA-core q' table of q·Kᵀ: (q'_c, q'_c) pairs; channel c = 32*h + cc sits at float2
+// index ((cc/2)*4 + h)*2 + cc%2, so that a 16-byte load gives a lane of the 3-bit
+// decode (chunk h) its next two channels.
+__device__ __forceinline__ int table_index(int c) {
+  const int h = c >> 5, cc = c & 31;
+  return ((cc >> 1) * 4 + h) * 2 + (cc & 1);
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
   return x;
 }
 
@@ -185,20 +180,15 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Warp-private shared memory region.
-template <int BITS, int G, bool PV>
-struct WarpMem {
-  using C = Cfg<BITS, G, PV>;
-  unsigned char* base;
-  __device__ unsigned char* stage(int s) const { return base + s * C::kStageBytes; }
-  __device__ float* table() const { return reinterpret_cast<float*>(base + C::kStages * C::kStageBytes); }
-  __device__ uint64_t* bar(int s) const {
-    return reinterpret_cast<uint64_t*>(base + C::kStages * C::kStageBytes + C::kTableBytes) + s;
-  }
-  __device__ int* kind(int s) const {
-    return reinterpret_cast<int*>(base + C::kStages * C::kStageBytes + C::kTableBytes + C::kStages * 8) + s;
-  }
-};
+// 16-byte shared-memory load that the compiler issues where it stands (keeps it from
+// hoisting a whole table of loop-invariant loads into registers).
+__device__ __forceinline__ float4 lds_f4(const float* p) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(smem_addr(p)));
+  return r;
+}
 
 // Position in the flat item list: (sequence*kv_heads + head, item within it).
 struct Cursor {
@@ -213,7 +203,7 @@ struct Cursor {
 };
 
 // Index entry {offset16, length16} of item c ({0, 0} for a tail item).  Loaded one
-// item ahead of its use so that its latency hides behind a block's arithmetic.
+// item ahead of its use so that its latency hides behind a record's arithmetic.
 __device__ __forceinline__ uint2 index_entry(const GemvArgs& a, Cursor c) {
   if (c.j >= a.n_blocks) return make_uint2(0u, 0u);
   return *reinterpret_cast<const uint2*>(a.index + ((size_t)c.bh * a.max_blocks + c.j) * 2);
@@ -269,106 +259,129 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const WarpMem<BITS
   }
 }
 
-// ----------------------------------------------------------------------------
-// Tensor-core decode of raw b = 2 / 4 records (fragment order, FORMAT.md section 4)
-// ----------------------------------------------------------------------------
-// (w & MASK) | 0x64006400: two fields become fp16 1024 + field*2^shift, exactly.
-template <uint32_t MASK>
-__device__ __forceinline__ uint32_t hfld(uint32_t w) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(0x64006400u));
-  return d;
+// After a wait gave up: waits, bounded, for the warp's other copies in flight
+// (items x+1 .. prod-1) so that none lands after the warp has exited.
+template <int BITS, int G, bool PV>
+__device__ void drain_stages(const WarpMem<BITS, G, PV>& m, uint32_t phases, int s, long x, long prod,
+                             uint64_t* ctrl) {
+  using C = Cfg<BITS, G, PV>;
+  for (long i = x + 1; i < prod; ++i) {
+    const int si = (int)((s + (i - x)) % C::kStages);
+    mbar_wait_bounded(m.bar(si), (phases >> si) & 1u, ctrl);
+  }
 }
 
-// Exact field values from hfld: (1024 + field*2^k) * 2^-k - 1024 * 2^-k = field
-// (one fused fp16x2 FMA; every intermediate is an fp16 integer below 2048).
-template <uint32_t MASK, int K>
-__device__ __forceinline__ uint32_t hval(uint32_t w) {
-  const uint32_t bits = hfld<MASK>(w);
-  const __half2 x = *reinterpret_cast<const __half2*>(&bits);
-  const __half2 mul = __float2half2_rn(1.0f / float(1 << K));
-  const __half2 add = __float2half2_rn(-1024.0f / float(1 << K));
-  const __half2 r = __hfma2(x, mul, add);
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-
-// D += A(16x16, fp16) * B(16x8, fp16), fp32 accumulate.
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
+// ----------------------------------------------------------------------------
+// 8-bit integer tensor-core decode of raw b = 2 / 4 records (FORMAT.md section 4)
+// ----------------------------------------------------------------------------
+// D(16x8, s32) += A(16x32, u8) * B(32x8, s8): exact integer products and sums.
+__device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
+// Exact float of an integer |d| < 2^22.
+__device__ __forceinline__ float i2f_small(int d) { return __int_as_float(d + kRoundBits) - kRound; }
+
+// The low bytes of four floats of the form r + 1.5*2^23 (r an integer, |r| <= 127):
+// the two's-complement bytes of r, packed in order.
+__device__ __forceinline__ uint32_t pack4(float2 lo, float2 hi) {
+  const uint32_t x0 = __float_as_uint(lo.x), x1 = __float_as_uint(lo.y);
+  const uint32_t x2 = __float_as_uint(hi.x), x3 = __float_as_uint(hi.y);
+  return __byte_perm(__byte_perm(x0, x1, 0x0040), __byte_perm(x2, x3, 0x0040), 0x5410);
 }
 
-// Word offset of half kh of the B-table entry (k-tile kt, thread t, column n); the
-// k-tile stride is padded by 4 words so that the table's stores spread over banks.
+// Word of the int8 B table holding B[k = 32*kap + 16*kh + 4*t .. +3][n], read by lane
+// 4*(n%8) + t as b_kh of n-tile n/8; a lane's words for one k-step are consecutive.
 template <int NT>
-__device__ __forceinline__ int btab_word(int kt, int t, int n, int kh) {
-  return kt * (64 * NT + 4) + (t * 8 * NT + n) * 2 + kh;
+__device__ __forceinline__ int i8tab_word(int kap, int kh, int t, int n) {
+  return kap * (64 * NT + 8) + (4 * (n & 7) + t) * 2 * NT + kh * NT + (n >> 3);
 }
 
-// Per-block B operand of the MMA: column n = 2*head + part holds, for every k
-// (channel for q·Kᵀ, storage slot for p·V), the fp16 high (part 0) or low
-// (part 1) half of v[head][k] * f[head]; f is a power of two putting the head's
-// largest |v| in [2^14, 2^15).  Summing the two columns of a head restores v to
-// about 22 bits.  Table entry [k-tile][t][column] = {b0, b1} of the m16n8k16
-// fragment.  Lane holds v for k = 4*lane .. 4*lane+3.  Returns 1/f per head.
+// B table of the int8 products for one record: lane holds x[head][i] for k = 4*lane + i
+// (channel for q·Kᵀ, storage slot for p·V).  Per head f = 127 / max|x| and
+// y = x*f = d0 + d1/128 + d2/16384 with integer digits |d0| <= 127, |d1|, |d2| <= 64
+// (each the rounding of the remainder so far, so |y - sum| <= 2^-15); column
+// 4*head + i holds digit i (column 4*head + 3 and the columns of absent heads are
+// zero).  Returns 1/f per head.
 template <int G, int NT>
-__device__ __forceinline__ void build_btab(uint32_t* btab, const float (&v)[G][4], float (&invf)[G], int lane) {
-  uint32_t pr[G][2][2];  // [head][part][pair]
+__device__ __forceinline__ void build_i8tab(uint32_t* tab, const float (&x)[G][4], float (&invf)[G], int lane) {
+  const int kap = lane >> 3, kh = (lane >> 2) & 1, t = lane & 3;
+  const float2 R = make_float2(kRound, kRound), nR = make_float2(-kRound, -kRound);
+  const float2 k128 = make_float2(128.f, 128.f);
 #pragma unroll
-  for (int hd = 0; hd < G; ++hd) {
-    const float mx = warp_max(fmaxf(fmaxf(fabsf(v[hd][0]), fabsf(v[hd][1])), fmaxf(fabsf(v[hd][2]), fabsf(v[hd][3]))));
-    const int e = mx > 0.f ? (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127 : 0;
-    const float f = mx > 0.f ? exp2i(14 - e) : 1.f;
-    invf[hd] = mx > 0.f ? exp2i(e - 14) : 1.f;
+  for (int hd = 0; hd < 2 * NT; ++hd) {
+    uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
+    if (hd < G) {
+      const int h = hd < G ? hd : 0;
+      const float mx =
+          warp_max(fmaxf(fmaxf(fabsf(x[h][0]), fabsf(x[h][1])), fmaxf(fabsf(x[h][2]), fabsf(x[h][3]))));
+      const float f = mx > 0.f ? __fdividef(127.f, mx) : 1.f;
+      invf[h] = mx > 0.f ? __fdividef(mx, 127.f) : 1.f;
+      const float2 m128 = make_float2(-128.f, -128.f);
+      float2 t0[2], t1[2], t2[2];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const float x0 = v[hd][2 * q] * f, x1 = v[hd][2 * q + 1] * f;
-      const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-      const __half l0 = __float2half_rn(x0 - __half2float(h0)), l1 = __float2half_rn(x1 - __half2float(h1));
-      pr[hd][0][q] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
-      pr[hd][1][q] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+      for (int q = 0; q < 2; ++q) {
+        float2 y = __fmul2_rn(make_float2(x[h][2 * q], x[h][2 * q + 1]), make_float2(f, f));
+        y = make_float2(fminf(fmaxf(y.x, -127.f), 127.f), fminf(fmaxf(y.y, -127.f), 127.f));
+        t0[q] = __fadd2_rn(y, R);                                          // low byte: d0 = rint(y)
+        const float2 r1 = __ffma2_rn(__fadd2_rn(t0[q], nR), m128, __fmul2_rn(y, k128));  // 128(y - d0), exact
+        t1[q] = __fadd2_rn(r1, R);                                         // low byte: d1 = rint(r1)
+        const float2 r2 = __ffma2_rn(__fadd2_rn(t1[q], nR), m128, __fmul2_rn(r1, k128));  // 128(r1 - d1), exact
+        t2[q] = __fadd2_rn(r2, R);                                         // low byte: d2 = rint(r2)
+      }
+      w0 = pack4(t0[0], t0[1]);
+      w1 = pack4(t1[0], t1[1]);
+      w2 = pack4(t2[0], t2[1]);
     }
-  }
-  // live columns 0 .. 2G-1 only; columns 2G .. 8NT-1 stay zero (zero_btab).  The
-  // lane's column order is rotated by its k-tile so that one store instruction
-  // spreads over the banks instead of hitting the same bank eight times.
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int k = 4 * lane + 2 * q;  // even: the pair (k, k+1)
-    const int kt = k >> 4, kk = k & 15, kh = kk >> 3, t = (kk & 7) >> 1;
-    uint32_t* row = btab + btab_word<NT>(kt, t, 0, kh);
-#pragma unroll
-    for (int i = 0; i < 2 * G; ++i) {
-      const int n = (i + kt) % (2 * G);
-      uint32_t val = 0u;
-#pragma unroll
-      for (int c = 0; c < 2 * G; ++c)
-        if (n == c) val = pr[c >> 1][c & 1][q];
-      row[2 * n] = val;
-    }
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 0)] = w0;
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 1)] = w1;
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 2)] = w2;
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 3)] = 0u;
   }
 }
 
-// Zeroes the whole B table (the columns of absent heads must read as zero).
+// B fragments of this lane: bf[kap][j] = {b0, b1} of n-tile j at k-step kap.
 template <int NT>
-__device__ __forceinline__ void zero_btab(uint32_t* btab, int lane) {
-  uint4* p = reinterpret_cast<uint4*>(btab);
+__device__ __forceinline__ void load_i8frags(const uint32_t* tab, uint32_t (&bf)[4][NT][2], int lane) {
 #pragma unroll
-  for (int i = lane; i < 8 * (64 * NT + 4) / 4; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
-  __syncwarp();
+  for (int kap = 0; kap < 4; ++kap) {
+    const uint32_t* p = tab + kap * (64 * NT + 8) + lane * 2 * NT;  // [kh][j] words
+    if constexpr (NT == 1) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      bf[kap][0][0] = v.x;
+      bf[kap][0][1] = v.y;
+    } else {
+#pragma unroll
+      for (int q = 0; q < NT / 2; ++q) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p + 4 * q);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int idx = 4 * q + r, kh = idx / NT, j = idx % NT;
+          bf[kap][j][kh] = w4[r];
+        }
+      }
+    }
+  }
 }
 
-// Selects per-thread values of head 4*j + t (the head of MMA columns 2t, 2t+1 in n-tile j).
+// Sum of the three digit columns of an accumulator tile (thread (g, t) holds columns
+// 2t, 2t+1 = digits (0, 1) of head 2j + t/2 for even t, digit 2 and the zero column
+// for odd t): returns, in even-t threads, D0 + D1/128 + D2/16384 for rows g (lo) and
+// g + 8 (hi).
+__device__ __forceinline__ void digit_sum(const int (&d)[4], int t, float& lo, float& hi) {
+  const float w0 = (t & 1) ? 1.f / 16384.f : 1.f, w1 = (t & 1) ? 0.f : 1.f / 128.f;
+  lo = fmaf(i2f_small(d[1]), w1, i2f_small(d[0]) * w0);
+  hi = fmaf(i2f_small(d[3]), w1, i2f_small(d[2]) * w0);
+  lo += __shfl_down_sync(0xffffffffu, lo, 1);
+  hi += __shfl_down_sync(0xffffffffu, hi, 1);
+}
+
+// Selects the value of a run-time head index from a register array.
 template <int G>
 __device__ __forceinline__ float head_sel(const float (&x)[G], int head) {
   float r = 0.f;
@@ -378,241 +391,156 @@ __device__ __forceinline__ float head_sel(const float (&x)[G], int head) {
   return r;
 }
 
-// One raw b = 2 / 4 K block: scores of all 128 slots for the G heads.
-template <int BITS, int G>
-__device__ __forceinline__ void qk_tc(const unsigned char* st, const uint32_t* btab, const float (&cst)[G],
-                                      const float (&invf)[G], float* srow0, long ld,
-                                      float scale, int lane) {
-  constexpr int NT = (2 * G + 7) / 8;
-  const int g = lane >> 2, t = lane & 3;
-  uint32_t bf[NT][8][2];
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int kt = 0; kt < 8; ++kt) {
-      const uint2 e = *reinterpret_cast<const uint2*>(btab + btab_word<NT>(kt, t, 8 * j + g, 0));
-      bf[j][kt][0] = e.x;
-      bf[j][kt][1] = e.y;
-    }
-  float c_t[NT], f_t[NT];
-  bool live[NT];
-#pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int head = 4 * j + t;
-    live[j] = head < G;
-    c_t[j] = head_sel<G>(cst, head);
-    f_t[j] = head_sel<G>(invf, head);
-  }
-  // words (tile pair tp, k-tile kt) of this lane: uint4 index (tp*2 + kt/4)*32 + lane, component kt%4.
-  // Each k step issues the MMAs of 4 row tiles: 4 independent accumulator chains.
+// A registers of one row tile from its two fragment words (k halves kh = 0, 1).
+// b = 4: rows g (low nibbles, x1) and g + 8 (high nibbles, x16).
+__device__ __forceinline__ void afrag4(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
+  a[0] = w0 & 0x0F0F0F0Fu;
+  a[1] = w0 & 0xF0F0F0F0u;
+  a[2] = w1 & 0x0F0F0F0Fu;
+  a[3] = w1 & 0xF0F0F0F0u;
+}
+
+// b = 2: even tile rows g (x1), g + 8 (x4); odd tile rows g (x16), g + 8 (x64).
+__device__ __forceinline__ void afrag2(uint32_t w0, uint32_t w1, uint32_t (&ae)[4], uint32_t (&ao)[4]) {
+  ae[0] = w0 & 0x03030303u;
+  ae[1] = w0 & 0x0C0C0C0Cu;
+  ae[2] = w1 & 0x03030303u;
+  ae[3] = w1 & 0x0C0C0C0Cu;
+  ao[0] = w0 & 0x30303030u;
+  ao[1] = w0 & 0xC0C0C0C0u;
+  ao[2] = w1 & 0x30303030u;
+  ao[3] = w1 & 0xC0C0C0C0u;
+}
+
+// 1 / (power of two carried by the A fields) of row g (upper = 0) or g + 8 of a tile.
+template <int BITS>
+__host__ __device__ constexpr float row_unscale(int odd_tile, int upper) {
+  return BITS == 4 ? (upper ? 1.f / 16.f : 1.f)
+                   : (odd_tile ? (upper ? 1.f / 64.f : 1.f / 16.f) : (upper ? 0.25f : 1.f));
+}
+
+// Runs the tensor-core product of one raw b = 2 / 4 record: for every row tile T
+// (16 rows) calls emit(T, n-tile j, d) with the exact integer tile d.  Rows are
+// slots (q·Kᵀ, K record) or channels (p·V, V record).
+template <int BITS, int NT, class Emit>
+__device__ __forceinline__ void i8_product(const unsigned char* st, const uint32_t (&bf)[4][NT][2], int lane,
+                                           Emit&& emit) {
   const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
-  constexpr int kWordTiles = BITS == 4 ? 4 : 2;  // word rows per half (b = 2: a word feeds two row tiles)
-#pragma unroll 1
-  for (int half = 0; half < 2; ++half) {
-    uint32_t w[kWordTiles][8];
+  constexpr int kRows = BITS == 4 ? 8 : 4;  // word rows: tiles (b = 4) or tile pairs (b = 2)
 #pragma unroll
-    for (int u = 0; u < kWordTiles; ++u) {
-      const int tp = half * kWordTiles + u;
-      const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
-      w[u][0] = wa.x; w[u][1] = wa.y; w[u][2] = wa.z; w[u][3] = wa.w;
-      w[u][4] = wb.x; w[u][5] = wb.y; w[u][6] = wb.z; w[u][7] = wb.w;
-    }
-    float d[4][NT][4];  // 4 row tiles
+  for (int tp = 0; tp < kRows; ++tp) {
+    const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
+    // k-step kap: words (kh 0, kh 1) = (wa.x, wa.y), (wa.z, wa.w), (wb.x, wb.y), (wb.z, wb.w)
+    const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
+    if constexpr (BITS == 4) {
+      int d[NT][4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+      for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0;
 #pragma unroll
-      for (int j = 0; j < NT; ++j)
+      for (int kap = 0; kap < 4; ++kap) {
+        uint32_t a[4];
+        afrag4(w[kap][0], w[kap][1], a);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) d[u][j][i] = 0.f;
+        for (int j = 0; j < NT; ++j) imma16832(d[j], a, bf[kap][j][0], bf[kap][j][1]);
+      }
 #pragma unroll
-    for (int kt = 0; kt < 8; ++kt) {
+      for (int j = 0; j < NT; ++j) emit(tp, j, d[j]);
+    } else {
+      int de[NT][4], dd[NT][4];
 #pragma unroll
-      for (int u = 0; u < kWordTiles; ++u) {
-        const uint32_t x = w[u][kt], h = x >> 8;
-        if constexpr (BITS == 4) {
-          const uint32_t r0 = hval<0x000F000Fu, 0>(x), r1 = hval<0x00F000F0u, 4>(x);
-          const uint32_t r2 = hval<0x000F000Fu, 0>(h), r3 = hval<0x00F000F0u, 4>(h);
+      for (int j = 0; j < NT; ++j) {
+        de[j][0] = de[j][1] = de[j][2] = de[j][3] = 0;
+        dd[j][0] = dd[j][1] = dd[j][2] = dd[j][3] = 0;
+      }
 #pragma unroll
-          for (int j = 0; j < NT; ++j) mma16816(d[u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
-        } else {
-          const uint32_t r0 = hval<0x00030003u, 0>(x), r1 = hval<0x000C000Cu, 2>(x);
-          const uint32_t r2 = hval<0x00030003u, 0>(h), r3 = hval<0x000C000Cu, 2>(h);
-          const uint32_t s0 = hval<0x00300030u, 4>(x), s1 = hval<0x00C000C0u, 6>(x);
-          const uint32_t s2 = hval<0x00300030u, 4>(h), s3 = hval<0x00C000C0u, 6>(h);
+      for (int kap = 0; kap < 4; ++kap) {
+        uint32_t ae[4], ao[4];
+        afrag2(w[kap][0], w[kap][1], ae, ao);
 #pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            mma16816(d[2 * u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
-            mma16816(d[2 * u + 1][j], s0, s1, s2, s3, bf[j][kt][0], bf[j][kt][1]);
-          }
+        for (int j = 0; j < NT; ++j) {
+          imma16832(de[j], ae, bf[kap][j][0], bf[kap][j][1]);
+          imma16832(dd[j], ao, bf[kap][j][0], bf[kap][j][1]);
         }
       }
-    }
-    // row tile u of this half covers slots 16*(4*half + u) + g and + 8
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      if (!live[j]) continue;
-      float* dst = srow0 + (4 * j + t) * ld;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = 16 * (4 * half + u) + g;
-        dst[r] = scale * fmaf(d[u][j][0] + d[u][j][1], f_t[j], c_t[j]);
-        dst[r + 8] = scale * fmaf(d[u][j][2] + d[u][j][3], f_t[j], c_t[j]);
+      for (int j = 0; j < NT; ++j) {
+        emit(2 * tp, j, de[j]);
+        emit(2 * tp + 1, j, dd[j]);
       }
     }
   }
 }
 
-// One raw b = 2 / 4 V block: adds sum_slots p'*v_hat into the per-thread fp32
-// accumulators of channels 16*T + g (acc_lo) and 16*T + g + 8 (acc_hi), head 4j + t.
+// q·Kᵀ of one raw b = 2 / 4 K record: scores of all 128 slots for the G heads.
 template <int BITS, int G>
-__device__ __forceinline__ void pv_tc(const unsigned char* st, const uint32_t* btab,
-                                      const float (&invf)[G], float (&acc_lo)[(2 * G + 7) / 8][8],
-                                      float (&acc_hi)[(2 * G + 7) / 8][8], int lane) {
-  constexpr int NT = (2 * G + 7) / 8;
+__device__ __forceinline__ void qk_i8(const unsigned char* st, const uint32_t* tab, const float (&cst)[G],
+                                      const float (&invf)[G], float* sblk, long ld, float scale, int lane) {
+  constexpr int NT = (4 * G + 7) / 8;
   const int g = lane >> 2, t = lane & 3;
-  uint32_t bf[NT][8][2];
-#pragma unroll
-  for (int j = 0; j < NT; ++j)
-#pragma unroll
-    for (int kt = 0; kt < 8; ++kt) {
-      const uint2 e = *reinterpret_cast<const uint2*>(btab + btab_word<NT>(kt, t, 8 * j + g, 0));
-      bf[j][kt][0] = e.x;
-      bf[j][kt][1] = e.y;
+  uint32_t bf[4][NT][2];
+  load_i8frags<NT>(tab, bf, lane);
+  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, const int (&d)[4]) {
+    float lo, hi;
+    digit_sum(d, t, lo, hi);
+    const int head = 2 * j + (t >> 1);
+    if ((t & 1) == 0 && head < G) {
+      const float f = head_sel<G>(invf, head), c = head_sel<G>(cst, head);
+      float* dst = sblk + head * ld + 16 * T + g;
+      dst[0] = scale * fmaf(lo, f * row_unscale<BITS>(T & 1, 0), c);
+      dst[8] = scale * fmaf(hi, f * row_unscale<BITS>(T & 1, 1), c);
     }
+  });
+}
+
+// p·V of one raw b = 2 / 4 V record: adds sum_slots p'*code into the accumulators of
+// channels 16T + g (acc_lo) and 16T + g + 8 (acc_hi) of head 2j + t/2 (even t).
+template <int BITS, int G>
+__device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* tab, const float (&invf)[G],
+                                      float (&acc_lo)[(4 * G + 7) / 8][8], float (&acc_hi)[(4 * G + 7) / 8][8],
+                                      int lane) {
+  constexpr int NT = (4 * G + 7) / 8;
+  const int t = lane & 3;
+  uint32_t bf[4][NT][2];
+  load_i8frags<NT>(tab, bf, lane);
   float f_t[NT];
-  bool live[NT];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    live[j] = 4 * j + t < G;
-    f_t[j] = head_sel<G>(invf, 4 * j + t);
-  }
-  const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
-  constexpr int kWordTiles = BITS == 4 ? 4 : 2;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t w[kWordTiles][8];
-#pragma unroll
-    for (int u = 0; u < kWordTiles; ++u) {
-      const int tp = half * kWordTiles + u;
-      const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
-      w[u][0] = wa.x; w[u][1] = wa.y; w[u][2] = wa.z; w[u][3] = wa.w;
-      w[u][4] = wb.x; w[u][5] = wb.y; w[u][6] = wb.z; w[u][7] = wb.w;
-    }
-    float d[4][NT][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) d[u][j][i] = 0.f;
-#pragma unroll
-    for (int kt = 0; kt < 8; ++kt) {
-#pragma unroll
-      for (int u = 0; u < kWordTiles; ++u) {
-        const uint32_t x = w[u][kt], h = x >> 8;
-        if constexpr (BITS == 4) {
-          const uint32_t r0 = hval<0x000F000Fu, 0>(x), r1 = hval<0x00F000F0u, 4>(x);
-          const uint32_t r2 = hval<0x000F000Fu, 0>(h), r3 = hval<0x00F000F0u, 4>(h);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) mma16816(d[u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
-        } else {
-          const uint32_t r0 = hval<0x00030003u, 0>(x), r1 = hval<0x000C000Cu, 2>(x);
-          const uint32_t r2 = hval<0x00030003u, 0>(h), r3 = hval<0x000C000Cu, 2>(h);
-          const uint32_t s0 = hval<0x00300030u, 4>(x), s1 = hval<0x00C000C0u, 6>(x);
-          const uint32_t s2 = hval<0x00300030u, 4>(h), s3 = hval<0x00C000C0u, 6>(h);
-#pragma unroll
-          for (int j = 0; j < NT; ++j) {
-            mma16816(d[2 * u][j], r0, r1, r2, r3, bf[j][kt][0], bf[j][kt][1]);
-            mma16816(d[2 * u + 1][j], s0, s1, s2, s3, bf[j][kt][0], bf[j][kt][1]);
-          }
-        }
-      }
-    }
-    // row tile u of this half covers channels 16*(4*half + u) + g and + 8
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      if (!live[j]) continue;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc_lo[j][4 * half + u] = fmaf(d[u][j][0] + d[u][j][1], f_t[j], acc_lo[j][4 * half + u]);
-        acc_hi[j][4 * half + u] = fmaf(d[u][j][2] + d[u][j][3], f_t[j], acc_hi[j][4 * half + u]);
-      }
-    }
-  }
+  for (int j = 0; j < NT; ++j) f_t[j] = head_sel<G>(invf, 2 * j + (t >> 1));
+  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, const int (&d)[4]) {
+    float lo, hi;
+    digit_sum(d, t, lo, hi);
+    acc_lo[j][T] = fmaf(lo, f_t[j] * row_unscale<BITS>(T & 1, 0), acc_lo[j][T]);
+    acc_hi[j][T] = fmaf(hi, f_t[j] * row_unscale<BITS>(T & 1, 1), acc_hi[j][T]);
+  });
 }
 
 // ----------------------------------------------------------------------------
-// q·Kᵀ
+// q·Kᵀ on the CUDA cores
 // ----------------------------------------------------------------------------
-template <int BITS, int G>
-__device__ __forceinline__ void qk_raw(const unsigned char* st, const float2* qp, const float (&cst)[G],
-                                       float* srow0, long ld, float scale, int lane) {
-  using C = Cfg<BITS, G, false>;
-  if constexpr (BITS == 4) {
-    // lane = (group g, token octet k, channel half h); word k of unit (g, c) holds tokens 32g+8k..+7
-    const int h = lane & 1, k = (lane >> 1) & 3, g = lane >> 3;
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (2 * g + h) * C::kPitch) + k;
-    float2 acc[G][4];
+// One raw b = 3 K record: lane (g, k, h) decodes tokens 32g + 16k .. +15 over the 32
+// channels of chunk 4g + h (a 4-lane reduction over h finishes), heads in chunks of
+// at most four (the words are decoded once per chunk).
+template <int G>
+__device__ __forceinline__ void qk_raw3(const unsigned char* st, const float2* qp, const float (&cst)[G],
+                                        float* sblk, long ld, float scale, int lane) {
+  using C = Cfg<3, G, false>;
+  constexpr int HC = G > 4 ? 4 : G;
+  const int h = lane & 3, k = (lane >> 2) & 1, g = lane >> 3;
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + h) * C::kPitch);
+#pragma unroll 1
+  for (int h0 = 0; h0 < G; h0 += HC) {
+    float2 acc[HC][8];
 #pragma unroll
-    for (int hd = 0; hd < G; ++hd)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[hd][i] = make_float2(0.f, 0.f);
-#pragma unroll 4
-    for (int c2 = 0; c2 < 32; ++c2) {
-      float2 v0[4], v1[4];
-      dec4(wp[8 * c2], v0);
-      dec4(wp[8 * c2 + 4], v1);
-#pragma unroll
-      for (int hd = 0; hd < G; ++hd) {
-        const float4 qq = *reinterpret_cast<const float4*>(qp + hd * 128 + (c2 * C::kNH + h) * 2);
-        const float2 q0 = make_float2(qq.x, qq.y), q1 = make_float2(qq.z, qq.w);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          acc[hd][i] = __ffma2_rn(q0, v0[i], acc[hd][i]);
-          acc[hd][i] = __ffma2_rn(q1, v1[i], acc[hd][i]);
-        }
-      }
-    }
-#pragma unroll
-    for (int hd = 0; hd < G; ++hd) {
-      float t[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        t[2 * i] = acc[hd][i].x + __shfl_xor_sync(0xffffffffu, acc[hd][i].x, 1);
-        t[2 * i + 1] = acc[hd][i].y + __shfl_xor_sync(0xffffffffu, acc[hd][i].y, 1);
-      }
-      float o[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = t[i] * pow2(-sig4(i));
-        const float hi = t[i + 4] * pow2(-sig4(i + 4));
-        o[i] = scale * (cst[hd] + (h ? hi : lo));
-      }
-      float* dst = srow0 + hd * ld + 32 * g + 8 * k + 4 * h;
-      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
-    }
-  } else {
-    // lane = (group g, 16-token half k, channel quarter h)
-    const int h = lane & 3, k = (lane >> 2) & 1, g = lane >> 3;
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + h) * C::kPitch);
-    float2 acc[G][8];
-#pragma unroll
-    for (int hd = 0; hd < G; ++hd)
+    for (int hd = 0; hd < HC; ++hd)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[hd][i] = make_float2(0.f, 0.f);
 #pragma unroll 2
     for (int c2 = 0; c2 < 16; ++c2) {
       float2 v0[8], v1[8];
-      if constexpr (BITS == 2) {
-        dec2(wp[2 * (2 * c2) + k], v0);
-        dec2(wp[2 * (2 * c2 + 1) + k], v1);
-      } else {
-        dec3(wp[3 * (2 * c2) + k], wp[3 * (2 * c2) + 2] >> (16 * k), v0);
-        dec3(wp[3 * (2 * c2 + 1) + k], wp[3 * (2 * c2 + 1) + 2] >> (16 * k), v1);
-      }
+      dec3(wp[3 * (2 * c2) + k], wp[3 * (2 * c2) + 2] >> (16 * k), v0);
+      dec3(wp[3 * (2 * c2 + 1) + k], wp[3 * (2 * c2 + 1) + 2] >> (16 * k), v1);
 #pragma unroll
-      for (int hd = 0; hd < G; ++hd) {
-        const float4 qq = *reinterpret_cast<const float4*>(qp + hd * 128 + (c2 * C::kNH + h) * 2);
+      for (int hd = 0; hd < HC; ++hd) {
+        const float4 qq = *reinterpret_cast<const float4*>(qp + (h0 + hd) * 128 + (c2 * 4 + h) * 2);
         const float2 q0 = make_float2(qq.x, qq.y), q1 = make_float2(qq.z, qq.w);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -622,8 +550,8 @@ __device__ __forceinline__ void qk_raw(const unsigned char* st, const float2* qp
       }
     }
 #pragma unroll
-    for (int hd = 0; hd < G; ++hd) {
-      float t[16];
+    for (int hd = 0; hd < HC; ++hd) {
+      float tt[16];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float x = acc[hd][i].x, y = acc[hd][i].y;
@@ -631,8 +559,8 @@ __device__ __forceinline__ void qk_raw(const unsigned char* st, const float2* qp
         y += __shfl_xor_sync(0xffffffffu, y, 1);
         x += __shfl_xor_sync(0xffffffffu, x, 2);
         y += __shfl_xor_sync(0xffffffffu, y, 2);
-        t[2 * i] = x;
-        t[2 * i + 1] = y;
+        tt[2 * i] = x;
+        tt[2 * i + 1] = y;
       }
       float o[4];
 #pragma unroll
@@ -640,10 +568,10 @@ __device__ __forceinline__ void qk_raw(const unsigned char* st, const float2* qp
         float v = 0.f;
 #pragma unroll
         for (int hh = 0; hh < 4; ++hh)
-          if (h == hh) v = t[4 * hh + i] * pow2(-sig2(4 * hh + i));
-        o[i] = scale * (cst[hd] + v);
+          if (h == hh) v = tt[4 * hh + i] * pow2(-sig2(4 * hh + i));
+        o[i] = scale * (head_sel<G>(cst, h0 + hd) + v);
       }
-      float* dst = srow0 + hd * ld + 32 * g + 16 * k + 4 * h;
+      float* dst = sblk + (h0 + hd) * ld + 32 * g + 16 * k + 4 * h;
       *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
     }
   }
@@ -663,9 +591,10 @@ __device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, 
   return u;
 }
 
-template <int BITS, int G>
+// One compressed K record, lane = token within each pack group.
+template <int G>
 __device__ __forceinline__ void qk_packed(const unsigned char* st, const float2* qp, const float (&cst)[G],
-                                          float* srow0, long ld, float scale, int lane) {
+                                          float* sblk, long ld, float scale, int lane) {
   const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
   const uint8_t* meta = st + kMetaOffset;
   const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
@@ -679,7 +608,7 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float2*
       float part = 0.f;
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        part = fmaf(qp[hd * 128 + table_index<BITS, G, false>(4 * lane + i)].x, (float)((m4 >> (8 * i)) & 15u), part);
+        part = fmaf(qp[hd * 128 + table_index(4 * lane + i)].x, (float)((m4 >> (8 * i)) & 15u), part);
       bsum[hd] = warp_sum(part);
     }
     float acc[G];
@@ -695,12 +624,11 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float2*
         const float u = (float)unit_field(W, s, w, lane);
         s += w;
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd)
-          acc[hd] = fmaf(qp[hd * 128 + table_index<BITS, G, false>(4 * c4 + i)].x, u, acc[hd]);
+        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(qp[hd * 128 + table_index(4 * c4 + i)].x, u, acc[hd]);
       }
     }
 #pragma unroll
-    for (int hd = 0; hd < G; ++hd) srow0[hd * ld + 32 * g + lane] = scale * (cst[hd] + bsum[hd] + acc[hd]);
+    for (int hd = 0; hd < G; ++hd) sblk[hd * ld + 32 * g + lane] = scale * (cst[hd] + bsum[hd] + acc[hd]);
   }
 }
 
@@ -741,28 +669,28 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
   const int lane = threadIdx.x & 31;
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (warp >= a.n_warps) return;
-  WarpMem<BITS, G, false> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
+  const WarpMem<BITS, G, false> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
   const long lo = (long)((long long)a.n_items * warp / a.n_warps);
   const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
+  const int I = a.items_per_bh;
   if (lane == 0) {
     for (int s = 0; s < C::kStages; ++s) mbar_init(m.bar(s), 1);
     fence_mbar_init();
   }
   __syncwarp();
   long prod = lo;
-  Cursor pc{lo / a.items_per_bh, (int)(lo % a.items_per_bh)};
+  Cursor pc{lo / I, (int)(lo % I)};
   Cursor cc = pc;
-  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(a.items_per_bh))
+  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(I))
     issue_item<BITS, G, false>(a, m, pc, index_entry(a, pc), s, lane);
   uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
 
   const int q_heads = a.kv_heads * G;
   long cur_bh = -1;
-  bool btab_clean = false;  // the table region holds a B table whose absent-head columns are zero
   float qr[G][4];
   uint32_t phases = 0;
   int s = 0;
-  for (long x = lo; x < hi; ++x, cc.next(a.items_per_bh)) {
+  for (long x = lo; x < hi; ++x, cc.next(I)) {
     const long bh = cc.bh;
     const int j = cc.j;
     const long b = bh / a.kv_heads, h = bh % a.kv_heads;
@@ -782,7 +710,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
     }
     const bool ok = mbar_wait_bounded(m.bar(s), (phases >> s) & 1u, a.ctrl);
     phases ^= 1u << s;
-    if (!ok) return;  // the copy never landed: stop this warp (status already set)
+    if (!ok) {  // the copy never landed: stop this warp (status already set)
+      drain_stages<BITS, G, false>(m, phases, s, x, prod, a.ctrl);
+      return;
+    }
     const int kind = *m.kind(s);
     const unsigned char* st = m.stage(s);
     if (kind == kKindTail) {
@@ -793,8 +724,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
       for (int hd = 0; hd < G; ++hd)
         for (int i = lane; i < 128; i += 32) srow0[hd * a.ld + (long)j * 128 + i] = __int_as_float(0x7fc00000);
     } else {
-      // per block: the min term sum_c q_c * mn_c, then q' = q * scale_c as the
-      // tensor-core B table (raw b = 2 / 4) or the CUDA-core q' table
+      // per record: the min term sum_c q_c * mn_c, then q' = q * scale_c as the
+      // int8 tensor-core B table (raw b = 2 / 4) or the CUDA-core q' table
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -817,35 +748,33 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
       }
       float* sblk = srow0 + (long)j * 128;
       if (kind == kKindRaw && !C::kChunked) {
-        uint32_t* btab = reinterpret_cast<uint32_t*>(m.table());
-        if (!btab_clean) zero_btab<C::kNT>(btab, lane);
-        btab_clean = true;
+        uint32_t* tab = m.table();
         float invf[G];
-        build_btab<G, C::kNT>(btab, qv, invf, lane);
+        build_i8tab<G, C::kNT>(tab, qv, invf, lane);
         __syncwarp();
-        qk_tc<BITS, G>(st, btab, cst, invf, sblk, a.ld, a.scale, lane);
+        qk_i8<BITS, G>(st, tab, cst, invf, sblk, a.ld, a.scale, lane);
       } else {
-        btab_clean = false;
         float2* qp = reinterpret_cast<float2*>(m.table());
 #pragma unroll
         for (int hd = 0; hd < G; ++hd) {
-          *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane)) =
+          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane)) =
               make_float4(qv[hd][0], qv[hd][0], qv[hd][1], qv[hd][1]);
-          *reinterpret_cast<float4*>(qp + hd * 128 + table_index<BITS, G, false>(4 * lane + 2)) =
+          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane + 2)) =
               make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
         }
         __syncwarp();
-        if (kind == kKindRaw)
-          qk_raw<BITS, G>(st, qp, cst, sblk, a.ld, a.scale, lane);
-        else
-          qk_packed<BITS, G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+        if (kind == kKindRaw) {
+          if constexpr (BITS == 3) qk_raw3<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+        } else {
+          qk_packed<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+        }
       }
     }
     __syncwarp();
     if (prod < hi) {
       issue_item<BITS, G, false>(a, m, pc, next_e, s, lane);
       ++prod;
-      pc.next(a.items_per_bh);
+      pc.next(I);
       if (prod < hi) next_e = index_entry(a, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
@@ -853,96 +782,43 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
 }
 
 // ----------------------------------------------------------------------------
-// p·V
+// p·V on the CUDA cores
 // ----------------------------------------------------------------------------
-// Accumulates one raw block into acc[slab][hd] (lane = channel slab*32 + lane).  The
-// field exponents are folded into p'' = p * scale * 2^-sig, so decoded pairs multiply
-// consecutive p'' pairs directly.
-template <int BITS, int G>
-__device__ __forceinline__ void pv_raw(const unsigned char* st, const float* pp, float2 (&acc)[4][G], int lane) {
-  using C = Cfg<BITS, G, true>;
-  constexpr bool kRegP = G <= 2;  // keep the group's p'' in registers across the 4 slabs
+// One raw b = 3 V record, lane = channel sl*32 + lane; adds into the warp's shared
+// [G][128] channel sums.  The field exponents are folded into p'' = p * scale *
+// 2^-sig (pp: [G][128] by storage slot).
+template <int G>
+__device__ __forceinline__ void pv_raw3(const unsigned char* st, const float* pp, float* sacc, int lane) {
+  using C = Cfg<3, G, true>;
 #pragma unroll 1
   for (int g = 0; g < 4; ++g) {
-    float2 pr[kRegP ? G : 1][16];
-    if constexpr (kRegP) {
+#pragma unroll 1
+    for (int sl = 0; sl < 4; ++sl) {
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 12);
+      const uint32_t w2 = wp[2];
+      float2 v[2][8];
+      dec3(wp[0], w2, v[0]);        // slots 32g .. 32g+15
+      dec3(wp[1], w2 >> 16, v[1]);  // slots 32g+16 .. 32g+31
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
-        const float4* p4 = reinterpret_cast<const float4*>(pp + hd * 128 + 32 * g);
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const float4 x = p4[q];
-          pr[hd][2 * q] = make_float2(x.x, x.y);
-          pr[hd][2 * q + 1] = make_float2(x.z, x.w);
+          const float4 x = lds_f4(pp + hd * 128 + 32 * g + 4 * q);
+          a0 = __ffma2_rn(make_float2(x.x, x.y), v[q >> 2][2 * (q & 3)], a0);
+          a1 = __ffma2_rn(make_float2(x.z, x.w), v[q >> 2][2 * (q & 3) + 1], a1);
         }
-      }
-    }
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl) {
-      float2 v[16];
-      if constexpr (BITS == 4) {
-        const uint4 u = *reinterpret_cast<const uint4*>(st + 528 + (2 * g + (sl >> 1)) * C::kPitch +
-                                                        ((sl & 1) * 32 + lane) * 16);
-        float2 t[4];
-        dec4(u.x, t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = t[i];
-        dec4(u.y, t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[4 + i] = t[i];
-        dec4(u.z, t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[8 + i] = t[i];
-        dec4(u.w, t);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[12 + i] = t[i];
-      } else if constexpr (BITS == 2) {
-        const uint2 u = *reinterpret_cast<const uint2*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 8);
-        float2 t[8];
-        dec2(u.x, t);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = t[i];
-        dec2(u.y, t);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[8 + i] = t[i];
-      } else {
-        const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 12);
-        const uint32_t w0 = wp[0], w1 = wp[1], w2 = wp[2];
-        float2 t[8];
-        dec3(w0, w2, t);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = t[i];
-        dec3(w1, w2 >> 16, t);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[8 + i] = t[i];
-      }
-#pragma unroll
-      for (int hd = 0; hd < G; ++hd) {
-        float2 a0 = acc[sl][hd], a1 = make_float2(0.f, 0.f);
-        if constexpr (kRegP) {
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) {
-            a0 = __ffma2_rn(pr[hd][i], v[i], a0);
-            a1 = __ffma2_rn(pr[hd][i + 1], v[i + 1], a1);
-          }
-        } else {
-          const float4* p4 = reinterpret_cast<const float4*>(pp + hd * 128 + 32 * g);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 x = p4[q];
-            a0 = __ffma2_rn(make_float2(x.x, x.y), v[2 * q], a0);
-            a1 = __ffma2_rn(make_float2(x.z, x.w), v[2 * q + 1], a1);
-          }
-        }
-        acc[sl][hd] = __fadd2_rn(a0, a1);
+        sacc[hd * 128 + sl * 32 + lane] += (a0.x + a0.y) + (a1.x + a1.y);
       }
     }
   }
 }
 
-template <int BITS, int G>
-__device__ __forceinline__ void pv_packed(const unsigned char* st, const float* pp, const float (&pg)[G][4],
-                                          float2 (&acc)[4][G], int lane) {
+// One compressed V record, lane = channel sl*32 + lane; adds into the warp's shared
+// [G][128] channel sums.  pg[hd*4 + g] = sum of p' over pack group g.
+template <int G>
+__device__ __forceinline__ void pv_packed(const unsigned char* st, const float* pp, const float* pg, float* sacc,
+                                          int lane) {
   const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
   const uint8_t* meta = st + kMetaOffset;
   const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
@@ -965,7 +841,7 @@ __device__ __forceinline__ void pv_packed(const unsigned char* st, const float* 
 #pragma unroll 1
       for (int hd = 0; hd < G; ++hd) {
         const float* pr = pp + hd * 128 + 32 * g;
-        float sum = (float)base * pg[hd][g];
+        float sum = (float)base * pg[hd * 4 + g];
         if (w == 4) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -994,31 +870,67 @@ __device__ __forceinline__ void pv_packed(const unsigned char* st, const float* 
             sum = fmaf(lo_mul, s1, sum);
           }
         }
-        acc[sl][hd].x += sum;
+        sacc[hd * 128 + c] += sum;
       }
     }
   }
 }
 
-// Writes this warp's partial sums for (b, h) to its slot (warp + bh) and clears
-// them.  The tensor-core accumulators (thread (g, t) holds channels 16T+g and
-// 16T+g+8 of head 4j+t) go through `buf` (G x 128 floats of warp shared memory)
-// to the lane = channel layout of the CUDA-core accumulators.
+// The fp16 tail of one (sequence, head), lane = channel sl*32 + lane; adds into the
+// warp's shared [G][128] channel sums.
 template <int G>
-__device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float2 (&acc)[4][G],
-                                         float (&acc_lo)[(2 * G + 7) / 8][8], float (&acc_hi)[(2 * G + 7) / 8][8],
-                                         float (&mp)[G], float* buf, int lane) {
-  constexpr int NT = (2 * G + 7) / 8;
+__device__ __forceinline__ void pv_tail(const GemvArgs& a, long bh, float* sacc, int lane) {
+  const long b = bh / a.kv_heads, h = bh % a.kv_heads;
+  const uint16_t* tail = a.tail + (size_t)bh * 128 * 128;
+  float acc[4][G];
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) acc[sl][hd] = 0.f;
+  for (int t = 0; t < a.tail_len; ++t) {
+    float vv[4];
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)a.n_blocks * 128 + t];
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = fmaf(pt, vv[sl], acc[sl][hd]);
+    }
+  }
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) sacc[hd * 128 + sl * 32 + lane] += acc[sl][hd];
+}
+
+// Zeroes a warp's [G][128] channel sums.
+template <int G>
+__device__ __forceinline__ void zero_sums(float* sacc, int lane) {
+  float4* p = reinterpret_cast<float4*>(sacc);
+#pragma unroll
+  for (int i = lane; i < G * 32; i += 32) p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Writes this warp's partial sums for (b, h) to its slot (warp + bh) and clears them:
+// the tensor-core accumulators (even-t thread (g, t) holds channels 16T+g and 16T+g+8
+// of head 2j + t/2) and the min term are added into the shared channel sums, which
+// then go out with coalesced stores.
+template <int G>
+__device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float* sacc,
+                                         float (&acc_lo)[(4 * G + 7) / 8][8], float (&acc_hi)[(4 * G + 7) / 8][8],
+                                         float (&mp)[G], int lane) {
+  constexpr int NT = (4 * G + 7) / 8;
   const int g = lane >> 2, t = lane & 3;
   __syncwarp();
 #pragma unroll
   for (int j = 0; j < NT; ++j) {
-    const int head = 4 * j + t;
+    const int head = 2 * j + (t >> 1);
 #pragma unroll
     for (int T = 0; T < 8; ++T) {
-      if (head < G) {
-        buf[head * 128 + 16 * T + g] = acc_lo[j][T];
-        buf[head * 128 + 16 * T + g + 8] = acc_hi[j][T];
+      if ((t & 1) == 0 && head < G) {
+        sacc[head * 128 + 16 * T + g] += acc_lo[j][T];
+        sacc[head * 128 + 16 * T + g + 8] += acc_hi[j][T];
       }
       acc_lo[j][T] = 0.f;
       acc_hi[j][T] = 0.f;
@@ -1032,11 +944,12 @@ __device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, f
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) {
       const int c = sl * 32 + lane;
-      __stcg(part + hd * 128 + c, buf[hd * 128 + c] + acc[sl][hd].x + acc[sl][hd].y + mn);
-      acc[sl][hd] = make_float2(0.f, 0.f);
+      __stcg(part + hd * 128 + c, sacc[hd * 128 + c] + mn);
     }
     mp[hd] = 0.f;
   }
+  __syncwarp();
+  zero_sums<G>(sacc, lane);
   __syncwarp();
 }
 
@@ -1059,9 +972,9 @@ __global__ void __launch_bounds__(256) pv_reduce_kernel(const GemvArgs a) {
   const int hd = (int)(row % G);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long I = a.items_per_bh;
-  const long w0 = warp_of_item(bh * I, a.n_items, a.n_warps);
-  const long w1 = warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps);
-  const float4* base = reinterpret_cast<const float4*>(a.partials + ((size_t)bh * G + hd) * 128) + lane;
+  const long w0 = warp_of_item(bh * I, a.n_items, a.n_warps) + bh;
+  const long w1 = warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps) + bh;
+  const float4* base = reinterpret_cast<const float4*>(a.partials + hd * 128) + lane;
   const size_t slot_stride = (size_t)G * 128 / 4;  // float4 per partial slot
   float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
   long w = w0 + warp;
@@ -1092,70 +1005,57 @@ template <int BITS, int G>
 __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a) {
   using C = Cfg<BITS, G, true>;
   extern __shared__ __align__(128) unsigned char smem[];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (warp >= a.n_warps) return;
-  WarpMem<BITS, G, true> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const WarpMem<BITS, G, true> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
   const long lo = (long)((long long)a.n_items * warp / a.n_warps);
   const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
+  const int I = a.items_per_bh;
   if (lane == 0) {
     for (int s = 0; s < C::kStages; ++s) mbar_init(m.bar(s), 1);
     fence_mbar_init();
   }
   __syncwarp();
   long prod = lo;
-  Cursor pc{lo / a.items_per_bh, (int)(lo % a.items_per_bh)};
+  Cursor pc{lo / I, (int)(lo % I)};
   Cursor cc = pc;
-  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(a.items_per_bh))
+  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(I))
     issue_item<BITS, G, true>(a, m, pc, index_entry(a, pc), s, lane);
   uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
 
-  float2 acc[4][G];  // CUDA-core paths: lane = channel sl*32 + lane
-  float mp[G];
+  float mp[G];  // sum over the warp's records of p * mn (lane: slots 4*lane .. +3)
   float acc_lo[C::kNT][8], acc_hi[C::kNT][8];  // tensor-core path
 #pragma unroll
-  for (int hd = 0; hd < G; ++hd) {
-    mp[hd] = 0.f;
-#pragma unroll
-    for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = make_float2(0.f, 0.f);
-  }
+  for (int hd = 0; hd < G; ++hd) mp[hd] = 0.f;
 #pragma unroll
   for (int jn = 0; jn < C::kNT; ++jn)
 #pragma unroll
     for (int T = 0; T < 8; ++T) acc_lo[jn][T] = acc_hi[jn][T] = 0.f;
-  float* buf = m.table();
-  bool btab_clean = false;  // the table region holds a B table whose absent-head columns are zero
+  float* sacc = m.sums();
+  float* pp = reinterpret_cast<float*>(m.table());  // p'' [G][128] then group sums [G][4]
+  zero_sums<G>(sacc, lane);
+  __syncwarp();
   long cur_bh = cc.bh;
   uint32_t phases = 0;
   int s = 0;
-  for (long x = lo; x < hi; ++x, cc.next(a.items_per_bh)) {
+  for (long x = lo; x < hi; ++x, cc.next(I)) {
     const long bh = cc.bh;
-    const int j = cc.j;
     if (bh != cur_bh) {
-      pv_flush<G>(a, cur_bh, warp, acc, acc_lo, acc_hi, mp, buf, lane);
-      btab_clean = false;  // the flush used the table region as its buffer
+      pv_flush<G>(a, cur_bh, warp, sacc, acc_lo, acc_hi, mp, lane);
       cur_bh = bh;
     }
     const bool ok = mbar_wait_bounded(m.bar(s), (phases >> s) & 1u, a.ctrl);
     phases ^= 1u << s;
-    if (!ok) return;
+    if (!ok) {
+      drain_stages<BITS, G, true>(m, phases, s, x, prod, a.ctrl);
+      return;
+    }
     const int kind = *m.kind(s);
     const unsigned char* st = m.stage(s);
-    const long b = bh / a.kv_heads, h = bh % a.kv_heads;
     if (kind == kKindTail) {
-      const uint16_t* tail = a.tail + (size_t)bh * 128 * 128;
-      for (int t = 0; t < a.tail_len; ++t) {
-        float vv[4];
-#pragma unroll
-        for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
-#pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)a.n_blocks * 128 + t];
-#pragma unroll
-          for (int sl = 0; sl < 4; ++sl) acc[sl][hd].x = fmaf(pt, vv[sl], acc[sl][hd].x);
-        }
-      }
+      pv_tail<G>(a, bh, sacc, lane);
     } else if (kind == kKindInvalid) {
       if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
     } else {
@@ -1180,17 +1080,13 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
         }
       }
       if (kind == kKindRaw && !C::kChunked) {
-        uint32_t* btab = reinterpret_cast<uint32_t*>(m.table());
-        if (!btab_clean) zero_btab<C::kNT>(btab, lane);
-        btab_clean = true;
+        uint32_t* tab = m.table();
         float invf[G];
-        build_btab<G, C::kNT>(btab, pv4, invf, lane);
+        build_i8tab<G, C::kNT>(tab, pv4, invf, lane);
         __syncwarp();
-        pv_tc<BITS, G>(st, btab, invf, acc_lo, acc_hi, lane);
+        pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
       } else {
-        btab_clean = false;
-        float* pp = m.table();
-        float pg[G][4];
+        const bool raw = kind == kKindRaw;
 #pragma unroll
         for (int hd = 0; hd < G; ++hd) {
           float o[4];
@@ -1200,35 +1096,35 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
             ps += pv4[hd][i];
             const int r15 = (4 * lane + i) & 15;  // field position of slot r in a 2-bit slice word
             const int sg = r15 <= 10 ? 2 * r15 : 2 * r15 - 12;
-            o[i] = kind == kKindRaw ? pv4[hd][i] * exp2i(-sg) : pv4[hd][i];  // exact power-of-two scaling
+            o[i] = raw ? pv4[hd][i] * exp2i(-sg) : pv4[hd][i];  // exact power-of-two scaling
           }
           *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-          if (kind != kKindRaw) {
+          if (!raw) {
             // per-group sum of p' (lanes 8g..8g+7 hold group g)
             ps += __shfl_xor_sync(0xffffffffu, ps, 1);
             ps += __shfl_xor_sync(0xffffffffu, ps, 2);
             ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-#pragma unroll
-            for (int g = 0; g < 4; ++g) pg[hd][g] = __shfl_sync(0xffffffffu, ps, 8 * g);
+            if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
           }
         }
         __syncwarp();
-        if (kind == kKindRaw)
-          pv_raw<BITS, G>(st, pp, acc, lane);
-        else
-          pv_packed<BITS, G>(st, pp, pg, acc, lane);
+        if (raw) {
+          if constexpr (BITS == 3) pv_raw3<G>(st, pp, sacc, lane);
+        } else {
+          pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
+        }
       }
     }
     __syncwarp();
     if (prod < hi) {
       issue_item<BITS, G, true>(a, m, pc, next_e, s, lane);
       ++prod;
-      pc.next(a.items_per_bh);
+      pc.next(I);
       if (prod < hi) next_e = index_entry(a, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
-  pv_flush<G>(a, cur_bh, warp, acc, acc_lo, acc_hi, mp, buf, lane);
+  pv_flush<G>(a, cur_bh, warp, sacc, acc_lo, acc_hi, mp, lane);
 }
 
 // ----------------------------------------------------------------------------

@@ -182,8 +182,9 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
  * that every GPU loading the library holds until the process exits; the call
  * allocates nothing.  Returns PACKKV_ERR_CAPACITY, without launching, if the
  * call would need more scratch than that (the need is packkv_workspace_bytes-
- * like: (resident warps + batch*kv_heads) * G * 512 bytes; e.g. G <= 4 fits
- * for up to about 1000 (sequence, kv head) pairs on a B200).  The first call
+ * like: (CTAs launched + batch*kv_heads) * G * 512 bytes, with at most four
+ * CTAs per SM; e.g. with G = 4 about 3500 (sequence, kv head) pairs fit on a
+ * B200).  The first call
  * on a device looks up the array's device address (a one-time set-up); make
  * that first call before any stream capture.  All calls share the one array:
  * calls that overlap in time on the GPU race.  Nothing in it needs clearing.

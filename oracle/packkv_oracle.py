@@ -226,18 +226,20 @@ def record_bytes_max(bits: int) -> int:
 def frag_word_bit(bits: int, m: int, k: int):
     """(word index, bit offset) of A[m][k] in the raw fragment order (b = 2, 4).
 
-    Restates FORMAT.md section 4: m = 16T + 8rh + g, k = 16kappa + 8kh + 2t + e,
-    lane = 4g + t; the word is picked by (tile row T, kappa, lane) and the field
-    inside it by (e, kh, rh) (and the tile row parity for b = 2).
+    Restates FORMAT.md section 4: m = 16T + 8rh + g, k = 32kappa + 16kh + 4t + e,
+    lane = 4g + t; the word is picked by (row tile T (b = 4) or tile pair T div 2
+    (b = 2), kappa, kh, lane) and the field inside it by (e, rh) (and the tile
+    row parity for b = 2): byte e of the word holds row g in its low field(s)
+    and row g + 8 above them.
     """
     T, rh, g = m // 16, (m // 8) % 2, m % 8
-    kappa, kh, t, e = k // 16, (k // 8) % 2, (k % 8) // 2, k % 2
+    kappa, kh, t, e = k // 32, (k // 16) % 2, (k % 16) // 4, k % 4
     lane = 4 * g + t
-    J, Q = kappa // 4, kappa % 4
+    J, Q2 = kappa // 2, kappa % 2
     if bits == 4:
-        return ((T * 2 + J) * 32 + lane) * 4 + Q, 4 * (4 * e + 2 * kh + rh)
+        return ((T * 2 + J) * 32 + lane) * 4 + 2 * Q2 + kh, 4 * (2 * e + rh)
     if bits == 2:
-        return (((T // 2) * 2 + J) * 32 + lane) * 4 + Q, 2 * (8 * e + 4 * kh + 2 * (T % 2) + rh)
+        return (((T // 2) * 2 + J) * 32 + lane) * 4 + 2 * Q2 + kh, 2 * (4 * e + 2 * (T % 2) + rh)
     raise ValueError("fragment order is defined for b = 2 and b = 4")
 
 

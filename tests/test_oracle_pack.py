@@ -175,10 +175,11 @@ def test_cache_append_equals_block_encode():
 
 
 def test_raw_fragment_order_hand_words(golden_dir):
+    matrices = {"m+2k": lambda m, k: m + 2 * k, "m/8+k": lambda m, k: m // 8 + k}
     for line in _lines(os.path.join(golden_dir, "raw_fragment_words.txt")):
-        bits, idx, want = (t.strip() for t in line.split("|"))
+        bits, name, idx, want = (t.strip() for t in line.split("|"))
         bits, idx = int(bits), int(idx)
-        a = np.fromfunction(lambda m, k: (m + 2 * k) % (1 << bits), (128, 128), dtype=np.int64)
+        a = np.fromfunction(lambda m, k: matrices[name](m, k) % (1 << bits), (128, 128), dtype=np.int64)
         assert int(O.pack_raw_fragment(a, bits)[idx]) == int(want, 16), line
 
 
@@ -198,10 +199,10 @@ def test_raw_fragment_order_is_a_bijection(bits):
 
 def test_raw_v_record_stores_the_transpose():
     """In a V record the fragment rows are channels: word 0's first field is code[slot 0][channel 0],
-    its rh field (row 8) is code[slot 0][channel 8]."""
+    its rh field (row 8) is code[slot 0][channel 8], and byte 1 starts with code[slot 1][channel 0]."""
     k, v, _ = synth.small_case(31, 1, 1, 1, 128)
     _, v_rec, perm = O.encode_block(k[0, 0], v[0, 0], 4)
     assert len(v_rec) == O.raw_record_bytes(4)
     codes = O.quantize_block_v(v[0, 0], 4)[0][perm]      # [slot, channel]
     w0 = int(np.frombuffer(v_rec, "<u4", 1, 528)[0])
-    assert w0 & 0xF == codes[0, 0] and (w0 >> 4) & 0xF == codes[0, 8] and (w0 >> 16) & 0xF == codes[1, 0]
+    assert w0 & 0xF == codes[0, 0] and (w0 >> 4) & 0xF == codes[0, 8] and (w0 >> 8) & 0xF == codes[1, 0]
