@@ -2,15 +2,25 @@
 // bit-packing (FORMAT.md sections 1-4; PackKV paper page, Figure 2 steps (1)
 // and (2), Figure 5 granularities, TL;DR).
 //
-// One encode call runs three kernels on the caller's stream:
-//   1. encode_kernel<false>: per (sequence, head, block) CTA, quantize + reorder
-//      + unit widths, and store the record length in the index;
-//   2. arena_scan_kernel: one CTA turns the lengths into arena offsets in
-//      ascending (sequence, head, block) order, advances the arena ends and
-//      checks capacity (so the arena layout is deterministic);
-//   3. encode_kernel<true>: recomputes the block (cheaper than staging the codes
-//      in a workspace the ABI does not have), assembles the record in shared
-//      memory and writes it with 16-byte stores at its offset.
+// One encode call is one pass over the input: a CTA per (sequence, head, block)
+// quantizes the K and V blocks, ranks the tokens, sizes the units, assembles both
+// records in shared memory and writes them at their arena offsets.  The offsets
+// follow ascending (sequence, head, block) order, so they are prefix sums of
+// the record lengths; a CTA learns its prefix by decoupled look-back over the
+// index entries of the blocks before it:
+//   * a CTA takes a ticket (the order in which CTAs started) and handles block
+//     `ticket`, so every block before it belongs to a CTA that is running or done;
+//   * once its lengths are known it publishes them in its index entries
+//     ({length, AGGREGATE} in the {offset, length} words), then walks back until
+//     it meets an entry that is final ({offset16, length16}: the prefix through
+//     that block is offset16 - arena end + length16), summing the aggregates on
+//     the way, and writes its own final entry;
+//   * the last CTA to finish advances the arena ends, or, if any record did not
+//     fit, marks every index entry of the call invalid and sets
+//     PACKKV_DEV_CAPACITY (a record that did not fit was not written; records
+//     that fit may have been written past the old arena end).
+// Every wait (input copy, look-back) gives up after about a second, sets
+// PACKKV_DEV_TIMEOUT and fails the call instead of hanging.
 // The encoder runs once per 128 tokens per head; it is not on the per-token path.
 #include <cuda_runtime.h>
 
@@ -19,6 +29,11 @@
 
 namespace packkv {
 
+namespace {
+
+constexpr uint32_t kFlagAggregate = 0x80000000u;  // {x = own length16, y = flag}: prefix not known yet
+constexpr uint32_t kDone2 = 2u;                   // done counter step (bit 0: some record did not fit)
+
 struct EncodeSmem {
   __half kx[kBlockTokens][kHeadDim];   // input K block; later the K record buffer
   __half vx[kBlockTokens][kHeadDim];   // input V block; later the V record buffer
@@ -26,7 +41,9 @@ struct EncodeSmem {
   uint8_t cv[kBlockTokens][kHeadDim];  // V codes [token][channel]
   uint16_t kmin[kHeadDim], kscale[kHeadDim];     // per channel
   uint16_t vmin[kBlockTokens], vscale[kBlockTokens];  // per token (original order)
+  float red[4][256];                   // min / max halves
   int key[kBlockTokens];
+  int rank_part[2][kBlockTokens];
   uint8_t perm[kBlockTokens];          // perm[slot] = token
   uint8_t base[2][kGroups][kHeadDim];
   uint8_t width[2][kGroups][kHeadDim];
@@ -34,41 +51,93 @@ struct EncodeSmem {
   int group_total[2][kGroups];
   int wsum[2];
   int nonfinite;
+  int failed;                          // this CTA's inputs or prefix could not be obtained
+  int last;                            // this CTA finished last
+  long ticket;
+  unsigned long long prefix[2];        // exclusive prefix (16-byte units) of the K / V record
+  uint64_t bar;
 };
 
 __device__ __forceinline__ int bitlen(uint32_t x) { return x == 0 ? 0 : 32 - __clz(x); }
 
-template <bool kWrite>
+__device__ __forceinline__ unsigned long long* entry64(uint32_t* index, const EncodeArgs& a, long blk_in_call) {
+  const long bh = blk_in_call / a.nb, i = blk_in_call % a.nb;
+  return reinterpret_cast<unsigned long long*>(index + ((size_t)bh * a.max_blocks + a.n_old + i) * 2);
+}
+
+// Exclusive prefix, in 16-byte units, of block `t` of the call for one tensor, by
+// look-back over the entries of blocks t-1, t-2, ...  Returns false (and sets
+// PACKKV_DEV_TIMEOUT) if a predecessor did not publish within about a second.
+__device__ bool look_back(uint32_t* index, const EncodeArgs& a, long t, unsigned long long end0,
+                          unsigned long long* excl) {
+  unsigned long long sum = 0;
+  long p = t - 1;
+  uint64_t start = 0;
+  uint32_t it = 0;
+  while (p >= 0) {
+    const unsigned long long e = atomicAdd(entry64(index, a, p), 0ull);
+    const uint32_t x = (uint32_t)e, y = (uint32_t)(e >> 32);
+    if (y == 0u) {  // not published yet
+      if (start == 0) start = global_ns();
+      if ((++it & 255u) == 0u && global_ns() - start > 1000000000ull) {
+        set_status(a.ctrl, PACKKV_DEV_TIMEOUT);
+        *excl = sum;
+        return false;
+      }
+      continue;
+    }
+    if (y & kFlagAggregate) {
+      sum += x;
+      --p;
+    } else {
+      sum += (unsigned long long)x - end0 + y;  // final entry: prefix through block p
+      break;
+    }
+  }
+  *excl = sum;
+  return true;
+}
+
 __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   EncodeSmem& s = *reinterpret_cast<EncodeSmem*>(smem_raw);
   const int tid = threadIdx.x;
-  const int blk = blockIdx.x % a.nb;
-  const int bh = blockIdx.x / a.nb;  // b * heads + h
   const int qmax = (1 << a.bits) - 1;
+  const long n_call = (long)a.batch * a.heads * a.nb;
+  unsigned int* counters = reinterpret_cast<unsigned int*>(a.ctrl + kCtrlScratch);  // [ticket, done]
+
+  // ---- ticket, then both input blocks by bulk copy ---------------------------
+  if (tid == 0) {
+    s.ticket = (long)atomicAdd(&counters[0], 1u);
+    s.nonfinite = 0;
+    s.failed = 0;
+    s.wsum[0] = s.wsum[1] = 0;
+    mbar_init(&s.bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const long t_call = s.ticket;                 // block index within the call
+  const int blk = (int)(t_call % a.nb);
+  const long bh = t_call / a.nb;                // b * heads + h
   const size_t in_base = ((size_t)bh * a.nb + blk) * kBlockTokens * kHeadDim;
   const size_t slot = (size_t)bh * a.max_blocks + a.n_old + blk;
-
-  if (kWrite) {
-    // the scan kernel marks a whole call as failed when an arena would overflow
-    const uint64_t fail = a.ctrl[kCtrlScratch];
-    if (fail) return;
+  if (tid == 0) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive_expect_tx(&s.bar, 2u * kBlockTokens * kHeadDim * 2u);
+    bulk_g2s(&s.kx[0][0], a.k + in_base, kBlockTokens * kHeadDim * 2u, &s.bar);
+    bulk_g2s(&s.vx[0][0], a.v + in_base, kBlockTokens * kHeadDim * 2u, &s.bar);
   }
-
-  // ---- load both blocks (16-byte vectors), flag non-finite values ----------
-  if (tid == 0) s.nonfinite = 0;
-  if (tid < 2) s.wsum[tid] = 0;
+  const bool input_ok = mbar_wait_bounded(&s.bar, 0u, a.ctrl);
+  if (!input_ok) s.failed = 1;  // every writer writes 1
   __syncthreads();
+
+  // ---- non-finite values ------------------------------------------------------
   {
-    const uint4* ksrc = reinterpret_cast<const uint4*>(a.k + in_base);
-    const uint4* vsrc = reinterpret_cast<const uint4*>(a.v + in_base);
-    uint4* kdst = reinterpret_cast<uint4*>(&s.kx[0][0]);
-    uint4* vdst = reinterpret_cast<uint4*>(&s.vx[0][0]);
+    const uint4* kin = reinterpret_cast<const uint4*>(&s.kx[0][0]);
+    const uint4* vin = reinterpret_cast<const uint4*>(&s.vx[0][0]);
     int bad = 0;
     for (int i = tid; i < kBlockTokens * kHeadDim / 8; i += blockDim.x) {
-      uint4 kk = ksrc[i], vv = vsrc[i];
-      kdst[i] = kk;
-      vdst[i] = vv;
+      const uint4 kk = kin[i], vv = vin[i];
       const uint32_t w[8] = {kk.x, kk.y, kk.z, kk.w, vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -77,38 +146,44 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     }
     if (bad) s.nonfinite = 1;
   }
-  __syncthreads();
-  if (!kWrite && tid == 0 && s.nonfinite) set_status(a.ctrl, PACKKV_DEV_NONFINITE);
 
-  // ---- quantization parameters: K per channel, V per token -----------------
+  // ---- quantization parameters: K per channel, V per token -------------------
   {
-    float mn = 3.4e38f, mx = -3.4e38f;
-    if (tid < kHeadDim) {
-      const int c = tid;
-      for (int t = 0; t < kBlockTokens; ++t) {
-        const float x = __half2float(s.kx[t][c]);
-        mn = fminf(mn, x);
-        mx = fmaxf(mx, x);
-      }
-    } else {
-      const int t = tid - kHeadDim;
-      for (int i = 0; i < kHeadDim; ++i) {
-        const float x = __half2float(s.vx[t][(i + t) & (kHeadDim - 1)]);
-        mn = fminf(mn, x);
-        mx = fmaxf(mx, x);
-      }
+    // two threads per channel (K) and per token (V), each over half of the block
+    const int half = tid >> 7, idx = tid & 127;
+    float mn = 3.4e38f, mx = -3.4e38f, vmn = 3.4e38f, vmx = -3.4e38f;
+#pragma unroll 8
+    for (int i = 0; i < 64; ++i) {
+      const float xk = __half2float(s.kx[64 * half + i][idx]);
+      mn = fminf(mn, xk);
+      mx = fmaxf(mx, xk);
+      const float xv = __half2float(s.vx[idx][(64 * half + i + idx) & (kHeadDim - 1)]);  // rotated: banks
+      vmn = fminf(vmn, xv);
+      vmx = fmaxf(vmx, xv);
     }
-    if (mn == 0.0f) mn = 0.0f;  // -0 is stored as +0
-    const float range = __fsub_rn(mx, mn);
+    s.red[0][tid] = mn;
+    s.red[1][tid] = mx;
+    s.red[2][tid] = vmn;
+    s.red[3][tid] = vmx;
+  }
+  __syncthreads();
+  if (tid == 0 && s.nonfinite) set_status(a.ctrl, PACKKV_DEV_NONFINITE);
+  {
+    const bool is_k = tid < 128;
+    const int i = tid & 127, r0 = is_k ? 0 : 2;
+    float lo = fminf(s.red[r0][i], s.red[r0][128 + i]);
+    const float hi = fmaxf(s.red[r0 + 1][i], s.red[r0 + 1][128 + i]);
+    if (lo == 0.0f) lo = 0.0f;  // -0 is stored as +0
+    const float range = __fsub_rn(hi, lo);
     uint16_t sc = 0;
     if (range > 0.0f) sc = __half_as_ushort(__float2half_ru(__fdiv_rn(range, (float)qmax)));
-    const uint16_t mnb = __half_as_ushort(__float2half_rn(mn));  // exact: mn is an fp16 value
-    if (tid < kHeadDim) {
-      s.kmin[tid] = mnb;
-      s.kscale[tid] = sc;
+    const uint16_t mnb = __half_as_ushort(__float2half_rn(lo));  // exact: lo is an fp16 value
+    if (is_k) {
+      s.kmin[i] = mnb;
+      s.kscale[i] = sc;
     } else {
-      s.vmin[tid - kHeadDim] = mnb;
-      s.vscale[tid - kHeadDim] = sc;
+      s.vmin[i] = mnb;
+      s.vscale[i] = sc;
     }
   }
   __syncthreads();
@@ -153,15 +228,22 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     }
   }
   __syncthreads();
-  if (tid < kBlockTokens) {
-    const int kt = s.key[tid];
+  {
+    // rank of token t = #{u : key[u] < key[t] or (key[u] == key[t] and u < t)}; two
+    // threads per token, each counting over half of the tokens
+    const int t = tid & 127, half = tid >> 7;
+    const int kt = s.key[t];
     int r = 0;
-    for (int u = 0; u < kBlockTokens; ++u) {
+#pragma unroll 8
+    for (int i = 0; i < 64; ++i) {
+      const int u = 64 * half + i;
       const int ku = s.key[u];
-      r += (ku < kt) | ((ku == kt) & (u < tid));
+      r += (ku < kt) | ((ku == kt) & (u < t));
     }
-    s.perm[r] = (uint8_t)tid;
+    s.rank_part[half][t] = r;
   }
+  __syncthreads();
+  if (tid < kBlockTokens) s.perm[s.rank_part[0][tid] + s.rank_part[1][tid]] = (uint8_t)tid;
   __syncthreads();
 
   // ---- frame of reference and width of every (group, channel) unit ----------
@@ -169,6 +251,7 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
     const uint8_t(*cx)[kHeadDim] = tensor ? s.cv : s.ck;
     int lo = 255, hi = 0;
+#pragma unroll 8
     for (int j = 0; j < kGroupTokens; ++j) {
       const int code = cx[s.perm[g * kGroupTokens + j]][c];
       lo = min(lo, code);
@@ -191,15 +274,16 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     rec_bytes[tensor] = raw[tensor] ? raw_bytes : packed;
   }
 
-  if (!kWrite) {
-    if (tid == 0) {
-      a.k_index[slot * 2 + 1] = (uint32_t)(rec_bytes[0] >> 4);
-      a.v_index[slot * 2 + 1] = (uint32_t)(rec_bytes[1] >> 4);
-    }
-    return;
+  // ---- publish the lengths (look-back aggregates) ---------------------------
+  if (tid == 0 || tid == 32) {
+    const int tensor = tid >> 5;
+    uint32_t* index = tensor ? a.v_index : a.k_index;
+    const unsigned long long agg =
+        (unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) | ((unsigned long long)kFlagAggregate << 32);
+    atomicExch(entry64(index, a, t_call), agg);
   }
 
-  // ---- write pass: unit word offsets ----------------------------------------
+  // ---- unit word offsets ------------------------------------------------------
   {
     const int warp = tid >> 5, lane = tid & 31;  // 8 warps = (tensor, group)
     const int tensor = warp >> 2, g = warp & 3;
@@ -228,9 +312,9 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 
   // ---- assemble both records in shared memory (reusing the input buffers) ---
   uint32_t* rec32[2] = {reinterpret_cast<uint32_t*>(&s.kx[0][0]), reinterpret_cast<uint32_t*>(&s.vx[0][0])};
-  for (int i = tid; i < raw_bytes / 4; i += blockDim.x) {
-    rec32[0][i] = 0u;
-    rec32[1][i] = 0u;
+  for (int i = tid; i < raw_bytes / 16; i += blockDim.x) {
+    reinterpret_cast<uint4*>(rec32[0])[i] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(rec32[1])[i] = make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();
 #pragma unroll
@@ -327,96 +411,71 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
       rem -= p;
     }
   }
+
+  // ---- look-back: arena offsets (thread 0: K, thread 32: V) -------------------
+  if (tid == 0 || tid == 32) {
+    const int tensor = tid >> 5;
+    uint32_t* index = tensor ? a.v_index : a.k_index;
+    const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
+    unsigned long long excl = 0;
+    if (!look_back(index, a, t_call, end0, &excl)) s.failed = 1;
+    s.prefix[tensor] = excl;
+    // final entry {offset16, length16}; a failed call is invalidated by the last CTA
+    const unsigned long long fin = (unsigned long long)(uint32_t)(end0 + excl) |
+                                   ((unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) << 32);
+    atomicExch(entry64(index, a, t_call), fin);
+  }
   __syncthreads();
 
-  // ---- write the records and the permutation --------------------------------
+  // ---- write the records that fit and the permutation ------------------------
+  bool fits_all = !s.failed;
 #pragma unroll
   for (int tensor = 0; tensor < 2; ++tensor) {
-    const uint32_t* index = tensor ? a.v_index : a.k_index;
     uint8_t* arena = tensor ? a.v_arena : a.k_arena;
-    const uint64_t off16 = index[slot * 2];
+    const unsigned long long off16 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd] + s.prefix[tensor];
+    const bool fits =
+        !s.failed && (off16 + (unsigned long long)(rec_bytes[tensor] >> 4)) * 16ull <= a.arena_bytes;
+    fits_all = fits_all && fits;
+    if (!fits) continue;
     uint4* dst = reinterpret_cast<uint4*>(arena + off16 * 16);
     const uint4* src = reinterpret_cast<const uint4*>(rec32[tensor]);
     for (int i = tid; i < rec_bytes[tensor] / 16; i += blockDim.x) dst[i] = src[i];
   }
   if (a.perm != nullptr && tid < kBlockTokens) a.perm[slot * kBlockTokens + tid] = s.perm[tid];
-}
+  __syncthreads();
 
-// One CTA: arena offsets from record lengths, in (sequence, head, block) order.
-__global__ void __launch_bounds__(1024) arena_scan_kernel(EncodeArgs a) {
-  __shared__ unsigned long long warp_sums[32];
-  __shared__ unsigned long long totals[2];
-  __shared__ int failed;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const long n = (long)a.batch * a.heads * a.nb;
-  const long per = (n + blockDim.x - 1) / blockDim.x;
-  const long first = min(n, per * tid), last = min(n, first + per);
-  if (tid == 0) failed = 0;
-  for (int tensor = 0; tensor < 2; ++tensor) {
-    uint32_t* index = tensor ? a.v_index : a.k_index;
-    auto entry = [&](long e) -> uint32_t* {
-      const long bh = e / a.nb, i = e % a.nb;
-      return index + ((size_t)bh * a.max_blocks + a.n_old + i) * 2;
-    };
-    unsigned long long local = 0;
-    for (long e = first; e < last; ++e) local += entry(e)[1];
-    unsigned long long incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) warp_sums[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      unsigned long long ws = warp_sums[lane];
-      unsigned long long wi = ws;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long y = __shfl_up_sync(0xffffffffu, wi, o);
-        if (lane >= o) wi += y;
-      }
-      warp_sums[lane] = wi - ws;
-      if (lane == 31) totals[tensor] = wi;
-    }
-    __syncthreads();
-    const unsigned long long end = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
-    const unsigned long long total = totals[tensor];
-    const bool fits = (end + total) * 16ull <= a.arena_bytes;
-    if (!fits && tid == 0) failed = 1;
-    unsigned long long at = end + warp_sums[warp] + (incl - local);
-    for (long e = first; e < last; ++e) {
-      uint32_t* ent = entry(e);
-      const uint32_t len = ent[1];
-      ent[0] = fits ? (uint32_t)at : 0xFFFFFFFFu;
-      if (!fits) ent[1] = 0u;
-      at += len;
-    }
-    __syncthreads();
-  }
+  // ---- completion: the last CTA advances the arena ends or fails the call ----
   if (tid == 0) {
-    if (failed) {
-      // neither arena advances; the write pass skips the whole call
-      a.ctrl[kCtrlScratch] = 1ull;
-      set_status(a.ctrl, PACKKV_DEV_CAPACITY);
-    } else {
-      a.ctrl[kCtrlScratch] = 0ull;
-      a.ctrl[kCtrlKEnd] += totals[0];
-      a.ctrl[kCtrlVEnd] += totals[1];
+    __threadfence();
+    const unsigned int mine = kDone2 | (fits_all ? 0u : 1u);
+    const unsigned int prev = atomicAdd(&counters[1], mine);
+    s.last = (long)(prev >> 1) == n_call - 1;
+    if (s.last) {
+      __threadfence();
+      s.failed = (int)((prev | mine) & 1u);
     }
   }
-  if (failed) {
-    // mark every new entry of both tensors invalid (the K pass above may have fit)
-    for (int tensor = 0; tensor < 2; ++tensor) {
-      uint32_t* index = tensor ? a.v_index : a.k_index;
-      for (long e = first; e < last; ++e) {
-        const long bh = e / a.nb, i = e % a.nb;
-        uint32_t* ent = index + ((size_t)bh * a.max_blocks + a.n_old + i) * 2;
-        ent[0] = 0xFFFFFFFFu;
-        ent[1] = 0u;
-      }
+  __syncthreads();
+  // a copy that did not land in time: give it one more bounded wait before exiting
+  if (!input_ok && tid == 0) mbar_wait_bounded(&s.bar, 0u, a.ctrl);
+  if (!s.last) return;
+  if (s.failed) {
+    for (long e = tid; e < n_call; e += blockDim.x) {
+      *entry64(a.k_index, a, e) = 0xFFFFFFFFull;  // {offset 0xFFFFFFFF, length 0}
+      *entry64(a.v_index, a, e) = 0xFFFFFFFFull;
     }
+    if (tid == 0) set_status(a.ctrl, PACKKV_DEV_CAPACITY);
+  } else if (tid == 0 || tid == 32) {
+    // prefix through the last block of the call = its final entry's offset - end + length
+    const int tensor = tid >> 5;
+    uint32_t* index = tensor ? a.v_index : a.k_index;
+    const unsigned long long e = atomicAdd(entry64(index, a, n_call - 1), 0ull);
+    const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
+    const unsigned long long total = (unsigned long long)(uint32_t)e - end0 + (uint32_t)(e >> 32);
+    a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd] = end0 + total;
   }
+  __syncthreads();
+  if (tid == 0) a.ctrl[kCtrlScratch] = 0ull;  // ticket and done counters for the next call
 }
 
 // Copies one token per (sequence, head) into the tail at position `pos`.
@@ -434,22 +493,29 @@ __global__ void append_tail_kernel(const uint16_t* __restrict__ k, const uint16_
   dst[ch] = src[ch];
 }
 
+}  // namespace
+
 size_t encode_smem_bytes() { return sizeof(EncodeSmem); }
 
 cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t stream) {
   const size_t smem = sizeof(EncodeSmem);
   static bool configured = false;  // per process; the attribute is per function, not per device
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(encode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(encode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e = cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = true;
   }
+  // the look-back reads the new index entries as "not yet published" (0), and the
+  // ticket and done counters start from zero
+  const size_t pitch = (size_t)a.max_blocks * 8;
+  const size_t width = (size_t)a.nb * 8;
+  const size_t height = (size_t)a.batch * a.heads;
+  cudaError_t e = cudaMemset2DAsync(a.k_index + (size_t)a.n_old * 2, pitch, 0, width, height, stream);
+  if (e == cudaSuccess) e = cudaMemset2DAsync(a.v_index + (size_t)a.n_old * 2, pitch, 0, width, height, stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.ctrl + kCtrlScratch, 0, sizeof(uint64_t), stream);
+  if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long)a.batch * a.heads * a.nb);
-  encode_kernel<false><<<grid, 256, smem, stream>>>(a);
-  arena_scan_kernel<<<1, 1024, 0, stream>>>(a);
-  encode_kernel<true><<<grid, 256, smem, stream>>>(a);
+  encode_kernel<<<grid, 256, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -126,8 +126,12 @@ packkv_status packkv_cache_reset(packkv_cache* cache, void* stream);
  * Requires tail_len == 0 and n_blocks + cache->n_blocks <= max_blocks
  * (else PACKKV_ERR_INVALID_ARG / PACKKV_ERR_CAPACITY, nothing launched).
  * On success cache->n_blocks += n_blocks.  If an arena overflows on the device,
- * PACKKV_DEV_CAPACITY is set, nothing is written to the arenas and the new
- * index entries are marked invalid.  n_blocks == 0 is a no-op.
+ * PACKKV_DEV_CAPACITY is set, the arena ends do not move and every new index
+ * entry is marked invalid; records that fitted may have been written into the
+ * free space past the old arena end.  One pass over the input: the records'
+ * arena offsets come from a decoupled look-back over the new index entries
+ * (which the call clears first) and ctrl[3] counts the call's blocks.
+ * n_blocks == 0 is a no-op.
  */
 packkv_status packkv_encode_block(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
                                   int32_t n_blocks, void* stream);
