@@ -202,12 +202,28 @@ struct Cursor {
   }
 };
 
-// Index entry {offset16, length16} of item c ({0, 0} for a tail item).  Loaded one
-// item ahead of its use so that its latency hides behind a record's arithmetic.
-__device__ __forceinline__ uint2 index_entry(const GemvArgs& a, Cursor c) {
-  if (c.j >= a.n_blocks) return make_uint2(0u, 0u);
-  return *reinterpret_cast<const uint2*>(a.index + ((size_t)c.bh * a.max_blocks + c.j) * 2);
-}
+// Index entries {offset16, length16} of 32 consecutive items of a warp's range, one
+// per lane ({0, 0} for a tail item or past the range), loaded with one coalesced
+// load; any lane reads the entry of any item of the window by shuffle.
+struct EntryWindow {
+  long base;  // first item of the window
+  uint2 ent;  // entry of item base + lane
+  __device__ void load(const GemvArgs& a, long first, long hi, int lane) {
+    base = first;
+    ent = make_uint2(0u, 0u);
+    const long item = first + lane;
+    if (item < hi) {
+      const long bh = item / a.items_per_bh;
+      const int j = (int)(item % a.items_per_bh);
+      if (j < a.n_blocks) ent = *reinterpret_cast<const uint2*>(a.index + ((size_t)bh * a.max_blocks + j) * 2);
+    }
+  }
+  // Whole warp; base <= item < base + 32.
+  __device__ uint2 get(long item) const {
+    const int src = (int)(item - base);
+    return make_uint2(__shfl_sync(0xffffffffu, ent.x, src), __shfl_sync(0xffffffffu, ent.y, src));
+  }
+};
 
 // Issue the copies of item (bh, j) with index entry e into stage s (whole warp participates).
 template <int BITS, int G, bool PV>
@@ -681,9 +697,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
   long prod = lo;
   Cursor pc{lo / I, (int)(lo % I)};
   Cursor cc = pc;
+  EntryWindow win;
+  win.load(a, lo, hi, lane);
   for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(I))
-    issue_item<BITS, G, false>(a, m, pc, index_entry(a, pc), s, lane);
-  uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
+    issue_item<BITS, G, false>(a, m, pc, win.get(prod), s, lane);
 
   const int q_heads = a.kv_heads * G;
   long cur_bh = -1;
@@ -772,10 +789,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
     }
     __syncwarp();
     if (prod < hi) {
-      issue_item<BITS, G, false>(a, m, pc, next_e, s, lane);
+      if (prod - win.base >= 32) win.load(a, prod, hi, lane);
+      issue_item<BITS, G, false>(a, m, pc, win.get(prod), s, lane);
       ++prod;
       pc.next(I);
-      if (prod < hi) next_e = index_entry(a, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
@@ -960,13 +977,23 @@ __device__ __forceinline__ long warp_of_item(long item, long n_items, long n_war
 
 // Second pass of p·V: out = sum of the partials of every warp that touched
 // (b, h), in a fixed order (deterministic).  One CTA per output row (b, h, head):
-// warp i of 8 adds partial slots w0+i, w0+i+8, ... with coalesced 16-byte loads,
-// then warp 0 adds the 8 warp sums in order.  It is launched as a programmatic
+// warp i of 16 adds partial slots w0+i, w0+i+16, ... four independent 16-byte loads
+// at a time (the partials sit in L2, so the time is latency, not bandwidth), then
+// warp 0 adds the 16 warp sums in order.  It is launched as a programmatic
 // dependent of pv_kernel and waits for its results.
+constexpr int kReduceWarps = 16;
+
+__device__ __forceinline__ void add4(float4& s, const float4 x) {
+  s.x += x.x;
+  s.y += x.y;
+  s.z += x.z;
+  s.w += x.w;
+}
+
 template <int G>
-__global__ void __launch_bounds__(256) pv_reduce_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kReduceWarps * 32) pv_reduce_kernel(const GemvArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  __shared__ float4 warp_sum4[8][32];
+  __shared__ float4 warp_sum4[kReduceWarps][32];
   const long row = blockIdx.x;  // (b*kv_heads + h)*G + head
   const long bh = row / G;
   const int hd = (int)(row % G);
@@ -976,27 +1003,29 @@ __global__ void __launch_bounds__(256) pv_reduce_kernel(const GemvArgs a) {
   const long w1 = warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps) + bh;
   const float4* base = reinterpret_cast<const float4*>(a.partials + hd * 128) + lane;
   const size_t slot_stride = (size_t)G * 128 / 4;  // float4 per partial slot
-  float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+  constexpr long W = kReduceWarps;
+  float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0, s2 = s0, s3 = s0;
   long w = w0 + warp;
-  for (; w + 8 <= w1; w += 16) {
-    const float4 x = __ldcg(base + (size_t)w * slot_stride);
-    const float4 y = __ldcg(base + (size_t)(w + 8) * slot_stride);
-    s0.x += x.x; s0.y += x.y; s0.z += x.z; s0.w += x.w;
-    s1.x += y.x; s1.y += y.y; s1.z += y.z; s1.w += y.w;
+  for (; w + 3 * W <= w1; w += 4 * W) {
+    const float4 x0 = __ldcg(base + (size_t)w * slot_stride);
+    const float4 x1 = __ldcg(base + (size_t)(w + W) * slot_stride);
+    const float4 x2 = __ldcg(base + (size_t)(w + 2 * W) * slot_stride);
+    const float4 x3 = __ldcg(base + (size_t)(w + 3 * W) * slot_stride);
+    add4(s0, x0);
+    add4(s1, x1);
+    add4(s2, x2);
+    add4(s3, x3);
   }
-  if (w <= w1) {
-    const float4 x = __ldcg(base + (size_t)w * slot_stride);
-    s0.x += x.x; s0.y += x.y; s0.z += x.z; s0.w += x.w;
-  }
-  warp_sum4[warp][lane] = make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+  for (; w <= w1; w += W) add4(s0, __ldcg(base + (size_t)w * slot_stride));
+  add4(s0, s1);
+  add4(s2, s3);
+  add4(s0, s2);
+  warp_sum4[warp][lane] = s0;
   __syncthreads();
   if (warp == 0) {
     float4 r = warp_sum4[0][lane];
 #pragma unroll
-    for (int i = 1; i < 8; ++i) {
-      const float4 x = warp_sum4[i][lane];
-      r.x += x.x; r.y += x.y; r.z += x.z; r.w += x.w;
-    }
+    for (int i = 1; i < kReduceWarps; ++i) add4(r, warp_sum4[i][lane]);
     reinterpret_cast<float4*>(a.out + row * 128)[lane] = r;
   }
 }
@@ -1021,9 +1050,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
   long prod = lo;
   Cursor pc{lo / I, (int)(lo % I)};
   Cursor cc = pc;
+  EntryWindow win;
+  win.load(a, lo, hi, lane);
   for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(I))
-    issue_item<BITS, G, true>(a, m, pc, index_entry(a, pc), s, lane);
-  uint2 next_e = prod < hi ? index_entry(a, pc) : make_uint2(0u, 0u);
+    issue_item<BITS, G, true>(a, m, pc, win.get(prod), s, lane);
 
   float mp[G];  // sum over the warp's records of p * mn (lane: slots 4*lane .. +3)
   float acc_lo[C::kNT][8], acc_hi[C::kNT][8];  // tensor-core path
@@ -1117,10 +1147,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     }
     __syncwarp();
     if (prod < hi) {
-      issue_item<BITS, G, true>(a, m, pc, next_e, s, lane);
+      if (prod - win.base >= 32) win.load(a, prod, hi, lane);
+      issue_item<BITS, G, true>(a, m, pc, win.get(prod), s, lane);
       ++prod;
       pc.next(I);
-      if (prod < hi) next_e = index_entry(a, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
@@ -1218,7 +1248,7 @@ cudaError_t launch(GemvArgs a, cudaStream_t stream) {
   }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)rows);
-  cfg.blockDim = dim3(256);
+  cfg.blockDim = dim3(kReduceWarps * 32);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
