@@ -33,17 +33,19 @@ namespace {
 
 constexpr uint32_t kFlagAggregate = 0x80000000u;  // {x = own length16, y = flag}: prefix not known yet
 constexpr uint32_t kDone2 = 2u;                   // done counter step (bit 0: some record did not fit)
+constexpr int kEncodeThreads = 512;
+constexpr int kParts = kEncodeThreads / kBlockTokens;  // threads per channel / token in the reductions
 
-struct EncodeSmem {
+struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
   __half kx[kBlockTokens][kHeadDim];   // input K block; later the K record buffer
   __half vx[kBlockTokens][kHeadDim];   // input V block; later the V record buffer
   uint8_t ck[kBlockTokens][kHeadDim];  // K codes [token][channel]
   uint8_t cv[kBlockTokens][kHeadDim];  // V codes [token][channel]
   uint16_t kmin[kHeadDim], kscale[kHeadDim];     // per channel
   uint16_t vmin[kBlockTokens], vscale[kBlockTokens];  // per token (original order)
-  float red[4][256];                   // min / max halves
+  float red[4][kEncodeThreads];        // min / max partials
   int key[kBlockTokens];
-  int rank_part[2][kBlockTokens];
+  int rank_part[kParts][kBlockTokens];
   uint8_t perm[kBlockTokens];          // perm[slot] = token
   uint8_t base[2][kGroups][kHeadDim];
   uint8_t width[2][kGroups][kHeadDim];
@@ -58,6 +60,8 @@ struct EncodeSmem {
   uint64_t bar;
 };
 
+static_assert(sizeof(EncodeSmem) <= 113 * 1024, "two encoder CTAs per SM");
+
 __device__ __forceinline__ int bitlen(uint32_t x) { return x == 0 ? 0 : 32 - __clz(x); }
 
 __device__ __forceinline__ unsigned long long* entry64(uint32_t* index, const EncodeArgs& a, long blk_in_call) {
@@ -65,40 +69,60 @@ __device__ __forceinline__ unsigned long long* entry64(uint32_t* index, const En
   return reinterpret_cast<unsigned long long*>(index + ((size_t)bh * a.max_blocks + a.n_old + i) * 2);
 }
 
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Exclusive prefix, in 16-byte units, of block `t` of the call for one tensor, by
-// look-back over the entries of blocks t-1, t-2, ...  Returns false (and sets
-// PACKKV_DEV_TIMEOUT) if a predecessor did not publish within about a second.
+// look-back over the entries of blocks t-1, t-2, ..., 32 at a time (one warp, lane
+// l reading block p - l).  Within a window, the nearest final entry ends the walk
+// (its prefix plus the aggregates above it); a window without one adds its 32
+// aggregates and moves down.  A window waits while any entry above its nearest
+// final entry is unpublished.  Returns false (and sets PACKKV_DEV_TIMEOUT) if a
+// predecessor did not publish within about a second.
 __device__ bool look_back(uint32_t* index, const EncodeArgs& a, long t, unsigned long long end0,
-                          unsigned long long* excl) {
+                          unsigned long long* excl, int lane) {
   unsigned long long sum = 0;
-  long p = t - 1;
+  long p = t - 1;  // top of the current window
   uint64_t start = 0;
   uint32_t it = 0;
   while (p >= 0) {
-    const unsigned long long e = atomicAdd(entry64(index, a, p), 0ull);
-    const uint32_t x = (uint32_t)e, y = (uint32_t)(e >> 32);
-    if (y == 0u) {  // not published yet
+    const long mine = p - lane;
+    unsigned long long e = 0;
+    if (mine >= 0) e = ld_relaxed(entry64(index, a, mine));
+    const uint32_t y = (uint32_t)(e >> 32);
+    const bool unpublished = mine >= 0 && y == 0u;
+    const bool fin = mine >= 0 && y != 0u && !(y & kFlagAggregate);
+    const uint32_t fin_mask = __ballot_sync(0xffffffffu, fin);
+    const uint32_t unp_mask = __ballot_sync(0xffffffffu, unpublished);
+    // lanes above (nearer to t than) the nearest final entry must all be published
+    const int stop = fin_mask ? __ffs(fin_mask) - 1 : 32;  // lowest lane = nearest block
+    const uint32_t need = stop >= 32 ? 0xffffffffu : ((1u << stop) - 1u);
+    if (unp_mask & need) {
       if (start == 0) start = global_ns();
-      if ((++it & 255u) == 0u && global_ns() - start > 1000000000ull) {
-        set_status(a.ctrl, PACKKV_DEV_TIMEOUT);
+      if ((++it & 63u) == 0u && global_ns() - start > 1000000000ull) {
+        if (lane == 0) set_status(a.ctrl, PACKKV_DEV_TIMEOUT);
         *excl = sum;
         return false;
       }
       continue;
     }
-    if (y & kFlagAggregate) {
-      sum += x;
-      --p;
-    } else {
-      sum += (unsigned long long)x - end0 + y;  // final entry: prefix through block p
-      break;
-    }
+    unsigned long long v = 0;
+    if (mine >= 0 && lane < stop) v = (uint32_t)e;                                  // aggregates
+    if (lane == stop) v = (unsigned long long)(uint32_t)e - end0 + y;               // final: prefix
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    sum += v;
+    if (stop < 32) break;
+    p -= 32;
   }
   *excl = sum;
   return true;
 }
 
-__global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
+__global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   EncodeSmem& s = *reinterpret_cast<EncodeSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -149,15 +173,16 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
 
   // ---- quantization parameters: K per channel, V per token -------------------
   {
-    // two threads per channel (K) and per token (V), each over half of the block
-    const int half = tid >> 7, idx = tid & 127;
+    // kParts threads per channel (K) and per token (V), each over a slice of the block
+    constexpr int kSlice = kBlockTokens / kParts;
+    const int part = tid / kBlockTokens, idx = tid % kBlockTokens;
     float mn = 3.4e38f, mx = -3.4e38f, vmn = 3.4e38f, vmx = -3.4e38f;
 #pragma unroll 8
-    for (int i = 0; i < 64; ++i) {
-      const float xk = __half2float(s.kx[64 * half + i][idx]);
+    for (int i = 0; i < kSlice; ++i) {
+      const float xk = __half2float(s.kx[kSlice * part + i][idx]);
       mn = fminf(mn, xk);
       mx = fmaxf(mx, xk);
-      const float xv = __half2float(s.vx[idx][(64 * half + i + idx) & (kHeadDim - 1)]);  // rotated: banks
+      const float xv = __half2float(s.vx[idx][(kSlice * part + i + idx) & (kHeadDim - 1)]);  // rotated: banks
       vmn = fminf(vmn, xv);
       vmx = fmaxf(vmx, xv);
     }
@@ -168,11 +193,15 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   }
   __syncthreads();
   if (tid == 0 && s.nonfinite) set_status(a.ctrl, PACKKV_DEV_NONFINITE);
-  {
-    const bool is_k = tid < 128;
-    const int i = tid & 127, r0 = is_k ? 0 : 2;
-    float lo = fminf(s.red[r0][i], s.red[r0][128 + i]);
-    const float hi = fmaxf(s.red[r0 + 1][i], s.red[r0 + 1][128 + i]);
+  if (tid < 2 * kBlockTokens) {
+    const bool is_k = tid < kBlockTokens;
+    const int i = tid % kBlockTokens, r0 = is_k ? 0 : 2;
+    float lo = s.red[r0][i], hi = s.red[r0 + 1][i];
+#pragma unroll
+    for (int q = 1; q < kParts; ++q) {
+      lo = fminf(lo, s.red[r0][q * kBlockTokens + i]);
+      hi = fmaxf(hi, s.red[r0 + 1][q * kBlockTokens + i]);
+    }
     if (lo == 0.0f) lo = 0.0f;  // -0 is stored as +0
     const float range = __fsub_rn(hi, lo);
     uint16_t sc = 0;
@@ -229,21 +258,27 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   }
   __syncthreads();
   {
-    // rank of token t = #{u : key[u] < key[t] or (key[u] == key[t] and u < t)}; two
-    // threads per token, each counting over half of the tokens
-    const int t = tid & 127, half = tid >> 7;
+    // rank of token t = #{u : key[u] < key[t] or (key[u] == key[t] and u < t)};
+    // kParts threads per token, each counting over a slice of the tokens
+    constexpr int kSlice = kBlockTokens / kParts;
+    const int t = tid % kBlockTokens, part = tid / kBlockTokens;
     const int kt = s.key[t];
     int r = 0;
 #pragma unroll 8
-    for (int i = 0; i < 64; ++i) {
-      const int u = 64 * half + i;
+    for (int i = 0; i < kSlice; ++i) {
+      const int u = kSlice * part + i;
       const int ku = s.key[u];
       r += (ku < kt) | ((ku == kt) & (u < t));
     }
-    s.rank_part[half][t] = r;
+    s.rank_part[part][t] = r;
   }
   __syncthreads();
-  if (tid < kBlockTokens) s.perm[s.rank_part[0][tid] + s.rank_part[1][tid]] = (uint8_t)tid;
+  if (tid < kBlockTokens) {
+    int r = 0;
+#pragma unroll
+    for (int q = 0; q < kParts; ++q) r += s.rank_part[q][tid];
+    s.perm[r] = (uint8_t)tid;
+  }
   __syncthreads();
 
   // ---- frame of reference and width of every (group, channel) unit ----------
@@ -284,8 +319,8 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
   }
 
   // ---- unit word offsets ------------------------------------------------------
-  {
-    const int warp = tid >> 5, lane = tid & 31;  // 8 warps = (tensor, group)
+  if (tid < 256) {
+    const int warp = tid >> 5, lane = tid & 31;  // warps 0..7 = (tensor, group)
     const int tensor = warp >> 2, g = warp & 3;
     int w4[4];
     int local = 0;
@@ -412,18 +447,21 @@ __global__ void __launch_bounds__(256) encode_kernel(EncodeArgs a) {
     }
   }
 
-  // ---- look-back: arena offsets (thread 0: K, thread 32: V) -------------------
-  if (tid == 0 || tid == 32) {
-    const int tensor = tid >> 5;
+  // ---- look-back: arena offsets (warp 0: K, warp 1: V) -------------------------
+  if (tid < 64) {
+    const int tensor = tid >> 5, lane = tid & 31;
     uint32_t* index = tensor ? a.v_index : a.k_index;
     const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
     unsigned long long excl = 0;
-    if (!look_back(index, a, t_call, end0, &excl)) s.failed = 1;
-    s.prefix[tensor] = excl;
-    // final entry {offset16, length16}; a failed call is invalidated by the last CTA
-    const unsigned long long fin = (unsigned long long)(uint32_t)(end0 + excl) |
-                                   ((unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) << 32);
-    atomicExch(entry64(index, a, t_call), fin);
+    const bool ok = look_back(index, a, t_call, end0, &excl, lane);
+    if (lane == 0) {
+      if (!ok) s.failed = 1;
+      s.prefix[tensor] = excl;
+      // final entry {offset16, length16}; a failed call is invalidated by the last CTA
+      const unsigned long long fin = (unsigned long long)(uint32_t)(end0 + excl) |
+                                     ((unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) << 32);
+      atomicExch(entry64(index, a, t_call), fin);
+    }
   }
   __syncthreads();
 
@@ -515,7 +553,7 @@ cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t stream) {
   if (e == cudaSuccess) e = cudaMemsetAsync(a.ctrl + kCtrlScratch, 0, sizeof(uint64_t), stream);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((long)a.batch * a.heads * a.nb);
-  encode_kernel<<<grid, 256, smem, stream>>>(a);
+  encode_kernel<<<grid, kEncodeThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
