@@ -526,6 +526,17 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.n
     return softmax(s) @ np.asarray(v, np.float64)
 
 
+def cache_attention(cache: OracleCache, q: np.ndarray, scale: float):
+    """Decode attention over the packed cache for every (b, hq): the scores, the
+    softmax over all tokens of the sequence (packed blocks in storage order, then
+    the tail) and the probability-weighted sum of the decoded values ([Fig. 1];
+    [Fig. 2]: both products read the packed cache).  Returns out [B, Hq, D] and,
+    per element, the sum of |p_i * v_hat_ic| (the scale of the parity tolerance).
+    """
+    scores, _ = cache_qk(cache, q, scale)
+    return cache_pv(cache, softmax(scores))
+
+
 def compression_ratio(n_tokens_total: int, arena_bytes: int, index_bytes: int) -> float:
     """fp16 bytes of one tensor / (record bytes + index bytes)."""
     return n_tokens_total * HEAD_DIM * 2 / float(arena_bytes + index_bytes)

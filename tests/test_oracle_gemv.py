@@ -144,3 +144,47 @@ def test_quantization_error_propagates_within_bound():
         exact = (k[0, 0].astype(np.float64) @ q[0, 0].astype(np.float64))[cache.perm[0, 0, 0]]
         bound = np.abs(q[0, 0].astype(np.float64)) @ O.quant_error_bound(rec.scale, bits)
         assert np.all(np.abs(s[0, 0] - exact) <= bound)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_fused_attention_on_grid_inputs_is_plain_softmax_attention(bits):
+    """Lossless inputs: the oracle's decode attention over the packed, permuted cache
+    equals textbook softmax attention (numpy, fp64) over the original tokens in
+    arrival order: the storage permutation and the packing drop out."""
+    rng = np.random.default_rng(200 + bits)
+    B, H, G, T = 1, 2, 2, 256 + 17
+    k, v = _grid_kv(rng, B, H, 384, bits)
+    k, v = k[:, :, :T], v[:, :, :T]
+    q = rng.standard_normal((B, H * G, 128)).astype(np.float16)
+    cache = O.OracleCache(B, H, 4, bits)
+    cache.encode_blocks(k[:, :, :256], v[:, :, :256], 2)
+    for t in range(256, T):
+        cache.append_token(k[:, :, t], v[:, :, t])
+    scale = 1 / np.sqrt(128)
+    out, terms = O.cache_attention(cache, q, scale)
+    for b in range(B):
+        for h in range(H):
+            kk = k[b, h].astype(np.float64)
+            vv = v[b, h].astype(np.float64)
+            for g in range(G):
+                hq = h * G + g
+                s = scale * (kk @ q[b, hq].astype(np.float64))
+                e = np.exp(s - s.max())
+                want = (e / e.sum()) @ vv
+                np.testing.assert_allclose(out[b, hq], want, rtol=1e-10, atol=1e-10)
+                # the tolerance scale bounds the result (triangle inequality) and is the
+                # probability-weighted sum of |v|
+                assert np.all(terms[b, hq] >= np.abs(out[b, hq]) - 1e-12)
+                np.testing.assert_allclose(terms[b, hq], (e / e.sum()) @ np.abs(vv), rtol=1e-10)
+
+
+def test_fused_attention_probabilities_sum_to_one():
+    """With V constant 1 in every channel the output is the sum of the probabilities: 1."""
+    k, _, q = synth.small_case(7, 1, 1, 2, 128 * 2 + 5)
+    v = np.ones_like(k)
+    cache = O.OracleCache(1, 1, 3, 4)
+    cache.encode_blocks(k[:, :, :256], v[:, :, :256], 2)
+    for t in range(256, k.shape[2]):
+        cache.append_token(k[:, :, t], v[:, :, t])
+    out, _ = O.cache_attention(cache, q, 0.3)
+    np.testing.assert_allclose(out, 1.0, rtol=1e-12)
