@@ -13,6 +13,7 @@ namespace {
 
 using packkv::EncodeArgs;
 using packkv::GemvArgs;
+using packkv::AttnArgs;
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -211,6 +212,49 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
   a.out = out;
   a.partials = reinterpret_cast<float*>(ws);
   return cuda_status(packkv::launch_pv(a, as_stream(stream)));
+}
+
+size_t packkv_attention_workspace_bytes(const packkv_cache* cache, int32_t q_heads) {
+  if (check_cache(cache) != PACKKV_OK) return 0;
+  int g = 0;
+  if (!group_ok(cache, q_heads, &g)) return 0;
+  return packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, g);
+}
+
+packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t* q, int32_t q_heads, float scale,
+                                      float* out, void* ws, size_t ws_bytes, void* stream) {
+  const packkv_status st = check_cache(cache);
+  if (st != PACKKV_OK) return st;
+  int g = 0;
+  if (q_heads < 1 || q_heads % cache->kv_heads != 0) return PACKKV_ERR_INVALID_ARG;
+  if (!group_ok(cache, q_heads, &g)) return PACKKV_ERR_UNSUPPORTED;
+  const int64_t T = (int64_t)cache->n_blocks * PACKKV_BLOCK_TOKENS + cache->tail_len;
+  if (T == 0 || !aligned16(q) || !aligned16(out)) return PACKKV_ERR_INVALID_ARG;
+  const size_t need = packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, g);
+  if (!aligned16(ws) || ws_bytes < need) return PACKKV_ERR_INVALID_ARG;
+  AttnArgs a{};
+  a.k_arena = cache->k_arena;
+  a.v_arena = cache->v_arena;
+  a.k_index = cache->k_index;
+  a.v_index = cache->v_index;
+  a.k_tail = cache->k_tail;
+  a.v_tail = cache->v_tail;
+  a.batch = cache->batch;
+  a.kv_heads = cache->kv_heads;
+  a.group = g;
+  a.max_blocks = cache->max_blocks;
+  a.n_blocks = cache->n_blocks;
+  a.tail_len = cache->tail_len;
+  a.bits = (int)cache->fmt.bits;
+  a.arena16 = cache->arena_bytes / 16;
+  a.ctrl = cache->ctrl;
+  a.items_per_bh = cache->n_blocks + (cache->tail_len > 0 ? 1 : 0);
+  a.n_items = (long)cache->batch * cache->kv_heads * a.items_per_bh;
+  a.q = q;
+  a.scale = scale;
+  a.out = out;
+  a.partials = reinterpret_cast<float*>(ws);
+  return cuda_status(packkv::launch_attention(a, as_stream(stream)));
 }
 
 packkv_status packkv_get_status(const packkv_cache* cache, void* stream, uint32_t* bits_out) {

@@ -1,0 +1,619 @@
+// Fused decode attention over the packed cache (PackKV paper page, Figure 1: the
+// scores, the softmax between them and the weighted sum of values that make up
+// decode attention; Figure 2: the decompression folded into both products).
+//
+//   out[b,hq,c] = sum_i softmax_i(scale * q[b,hq]·k_hat[b,h,i]) * v_hat[b,h,i,c]
+//
+// over the packed blocks (storage order) and the fp16 tail.  One pass over both
+// arenas: a warp owns a contiguous range of items (blocks, then the tail) of the
+// flat (sequence, kv-head) list, as the q·Kᵀ / p·V kernels do.  Per item it
+// stages the K record and the V record (one single-stage ring each, so that the
+// next K record loads during this item's p·V and the next V record during the
+// next item's q·Kᵀ), computes the item's scores into shared memory with the
+// q·Kᵀ decode paths, updates a running maximum and sum of exponentials per head
+// (online softmax), and adds the probability-weighted values with the p·V decode
+// paths.  At every (sequence, head) boundary it writes its sums, maximum and sum
+// of exponentials per query head to its workspace slot; a second kernel,
+// launched as a programmatic dependent, merges the slots of each (sequence,
+// head) in warp order with the log-sum-exp rule: deterministic.  Neither the
+// scores nor the probabilities ever reach global memory.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <unordered_map>
+
+#include "decode.cuh"
+
+namespace packkv {
+
+namespace {
+
+#ifndef PACKKV_ATTN_WARPS_PER_CTA
+#define PACKKV_ATTN_WARPS_PER_CTA 2
+#endif
+constexpr int kAttnWarps = PACKKV_ATTN_WARPS_PER_CTA;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kSlotFloats = 132;  // per (workspace slot, head): 128 sums, running max, sum of exp, pad
+constexpr float kNegInf = -__builtin_huge_valf();
+
+template <int BITS, int G>
+struct AttnCfg {
+  using C = Cfg<BITS, G, false>;
+  static constexpr int kStageRec = C::kStageRec;  // one K or one V record
+  static constexpr int kNT = (4 * G + 7) / 8;
+  static constexpr int kI8Tab = 4 * (64 * kNT + 8) * 4;
+  static constexpr int kCoreTab = 1024 * G;  // q' pairs [G][128]; p'' [G][128] + group sums [G][4] fit too
+  static constexpr int kTableBytes = ((kI8Tab > kCoreTab ? kI8Tab : kCoreTab) + 15) / 16 * 16;
+  static constexpr int kScoreBytes = 512 * G;  // [G][128] scores, then probabilities
+  static constexpr int kSumBytes = 512 * G;    // [G][128] channel sums (CUDA-core and tail paths)
+  static constexpr int kFixed = 2 * kStageRec + kTableBytes + kScoreBytes + kSumBytes;
+  static constexpr int kWarpSmem = (kFixed + 32 + 127) / 128 * 128;
+  static_assert(kStageRec % 16 == 0 && kFixed % 16 == 0, "stage alignment");
+};
+
+// Warp-private shared memory: [K stage][V stage][table][scores][sums][2 mbarriers][2 kinds].
+template <int BITS, int G>
+struct AttnMem {
+  using A = AttnCfg<BITS, G>;
+  unsigned char* base;
+  __device__ unsigned char* stage(int s) const { return base + s * A::kStageRec; }
+  __device__ uint32_t* table() const { return reinterpret_cast<uint32_t*>(base + 2 * A::kStageRec); }
+  __device__ float* scores() const {
+    return reinterpret_cast<float*>(base + 2 * A::kStageRec + A::kTableBytes);
+  }
+  __device__ float* sums() const { return scores() + 128 * G; }
+  __device__ uint64_t* bar(int s) const { return reinterpret_cast<uint64_t*>(base + A::kFixed) + s; }
+  __device__ int* kind(int s) const { return reinterpret_cast<int*>(base + A::kFixed + 16) + s; }
+};
+
+// The K (v = false) or V (v = true) half of the arguments, in the form the shared
+// staging and decode helpers take.
+__device__ __forceinline__ GemvArgs tensor_view(const AttnArgs& a, bool v) {
+  GemvArgs g{};
+  g.arena = v ? a.v_arena : a.k_arena;
+  g.index = v ? a.v_index : a.k_index;
+  g.tail = v ? a.v_tail : a.k_tail;
+  g.batch = a.batch;
+  g.kv_heads = a.kv_heads;
+  g.group = a.group;
+  g.max_blocks = a.max_blocks;
+  g.n_blocks = a.n_blocks;
+  g.tail_len = a.tail_len;
+  g.bits = a.bits;
+  g.arena16 = a.arena16;
+  g.ctrl = a.ctrl;
+  g.n_items = a.n_items;
+  g.items_per_bh = a.items_per_bh;
+  g.n_warps = a.n_warps;
+  return g;
+}
+
+// Scaled scores of the fp16 tail tokens of (sequence, head) bh into sc[head*128 + t].
+template <int G>
+__device__ __forceinline__ void tail_scores(const AttnArgs& a, long bh, const float (&qr)[G][4], float* sc,
+                                            int lane) {
+  const uint16_t* tail = a.k_tail + (size_t)bh * 128 * 128;
+  for (int t0 = 0; t0 < a.tail_len; t0 += 32) {
+    float mine[G];
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) mine[hd] = 0.f;
+    const int tn = min(32, a.tail_len - t0);
+    for (int t = 0; t < tn; ++t) {
+      const uint2 hv = *reinterpret_cast<const uint2*>(tail + (size_t)(t0 + t) * 128 + 4 * lane);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        float part = qr[hd][0] * f0.x;
+        part = fmaf(qr[hd][1], f0.y, part);
+        part = fmaf(qr[hd][2], f1.x, part);
+        part = fmaf(qr[hd][3], f1.y, part);
+        part = warp_sum(part);
+        if (lane == t) mine[hd] = part;
+      }
+    }
+    if (lane < tn) {
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) sc[hd * 128 + t0 + lane] = a.scale * mine[hd];
+    }
+  }
+}
+
+// Adds sum_t p[head][t] * v_tail[t][c] into the channel sums (lane = channel sl*32 + lane).
+template <int G>
+__device__ __forceinline__ void tail_values(const AttnArgs& a, long bh, const float* p, float* sacc, int lane) {
+  const uint16_t* tail = a.v_tail + (size_t)bh * 128 * 128;
+  float acc[4][G];
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) acc[sl][hd] = 0.f;
+  for (int t = 0; t < a.tail_len; ++t) {
+    float vv[4];
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      const float pt = p[hd * 128 + t];
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = fmaf(pt, vv[sl], acc[sl][hd]);
+    }
+  }
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) sacc[hd * 128 + sl * 32 + lane] += acc[sl][hd];
+}
+
+// Writes this warp's state for (b, h) to its slot (warp + bh) and clears it: per query
+// head the 128 value sums (tensor-core accumulators, channel sums and the min term
+// together), the running maximum and the running sum of exponentials.
+template <int G>
+__device__ __forceinline__ void attn_flush(const AttnArgs& a, long bh, int warp, float* sacc,
+                                           float (&acc_lo)[(4 * G + 7) / 8][8],
+                                           float (&acc_hi)[(4 * G + 7) / 8][8], float (&mp)[G], float (&mrun)[G],
+                                           float (&lrun)[G], int lane) {
+  constexpr int NT = (4 * G + 7) / 8;
+  const int g = lane >> 2, t = lane & 3;
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int head = 2 * j + (t >> 1);
+#pragma unroll
+    for (int T = 0; T < 8; ++T) {
+      if ((t & 1) == 0 && head < G) {
+        sacc[head * 128 + 16 * T + g] += acc_lo[j][T];
+        sacc[head * 128 + 16 * T + g + 8] += acc_hi[j][T];
+      }
+      acc_lo[j][T] = 0.f;
+      acc_hi[j][T] = 0.f;
+    }
+  }
+  __syncwarp();
+  float* part = a.partials + (size_t)(warp + bh) * G * kSlotFloats;
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd) {
+    const float mn = warp_sum(mp[hd]);
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      const int c = sl * 32 + lane;
+      __stcg(part + hd * kSlotFloats + c, sacc[hd * 128 + c] + mn);
+    }
+    if (lane == 0) {
+      __stcg(part + hd * kSlotFloats + 128, mrun[hd]);
+      __stcg(part + hd * kSlotFloats + 129, lrun[hd]);
+    }
+    mp[hd] = 0.f;
+    mrun[hd] = kNegInf;
+    lrun[hd] = 0.f;
+  }
+  __syncwarp();
+  zero_sums<G>(sacc, lane);
+  __syncwarp();
+}
+
+template <int BITS, int G>
+__global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a) {
+  using A = AttnCfg<BITS, G>;
+  using C = Cfg<BITS, G, false>;
+  constexpr int NT = A::kNT;
+  extern __shared__ __align__(128) unsigned char smem[];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int warp = blockIdx.x * kAttnWarps + (threadIdx.x >> 5);
+  if (warp >= a.n_warps) return;
+  const AttnMem<BITS, G> m{smem + (threadIdx.x >> 5) * A::kWarpSmem};
+  const GemvArgs ka = tensor_view(a, false), va = tensor_view(a, true);
+  const long lo = (long)((long long)a.n_items * warp / a.n_warps);
+  const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
+  const int I = a.items_per_bh;
+  if (lane == 0) {
+    mbar_init(m.bar(0), 1);
+    mbar_init(m.bar(1), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  Cursor cc{lo / I, (int)(lo % I)};
+  EntryWindow wk, wv;
+  wk.load(ka, lo, hi, lane);
+  wv.load(va, lo, hi, lane);
+  issue_item<BITS, G, false>(ka, m, cc, wk.get(lo), 0, lane);
+  issue_item<BITS, G, false>(va, m, cc, wv.get(lo), 1, lane);
+
+  const int q_heads = a.kv_heads * G;
+  float qr[G][4];
+  float mrun[G], lrun[G], mp[G];
+  float acc_lo[NT][8], acc_hi[NT][8];
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd) {
+    mrun[hd] = kNegInf;
+    lrun[hd] = 0.f;
+    mp[hd] = 0.f;
+  }
+#pragma unroll
+  for (int jn = 0; jn < NT; ++jn)
+#pragma unroll
+    for (int T = 0; T < 8; ++T) acc_lo[jn][T] = acc_hi[jn][T] = 0.f;
+  float* sacc = m.sums();
+  float* sc = m.scores();
+  zero_sums<G>(sacc, lane);
+  __syncwarp();
+  long cur_bh = -1;
+  uint32_t phases = 0;
+  const int g = lane >> 2, t = lane & 3;
+  for (long x = lo; x < hi; ++x) {
+    const long bh = cc.bh;
+    const long b = bh / a.kv_heads, h = bh % a.kv_heads;
+    if (bh != cur_bh) {
+      if (cur_bh >= 0) attn_flush<G>(a, cur_bh, warp, sacc, acc_lo, acc_hi, mp, mrun, lrun, lane);
+      cur_bh = bh;
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        const uint2 hv = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * q_heads + h * G + hd) * 128 + 4 * lane);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+        qr[hd][0] = f0.x;
+        qr[hd][1] = f0.y;
+        qr[hd][2] = f1.x;
+        qr[hd][3] = f1.y;
+      }
+    }
+    Cursor nc = cc;
+    nc.next(I);
+
+    // ---- K: scaled scores of this item's tokens into sc[head][slot] ----------
+    bool ok = mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
+    phases ^= 1u;
+    if (!ok) {  // the copy never landed (status set): wait, bounded, for the V copy, then stop
+      mbar_wait_bounded(m.bar(1), (phases >> 1) & 1u, a.ctrl);
+      return;
+    }
+    const int kind_k = *m.kind(0);
+    int n_tok = 128;
+    bool skip = false;
+    if (kind_k == kKindTail) {
+      n_tok = a.tail_len;
+      tail_scores<G>(a, bh, qr, sc, lane);
+    } else if (kind_k == kKindInvalid) {
+      if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
+      skip = true;
+    } else {
+      const unsigned char* st = m.stage(0);
+      const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
+      const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
+      const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
+      const float2 mn1 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.y));
+      const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&scv.x));
+      const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&scv.y));
+      float cst[G], qv[G][4];
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        float part = qr[hd][0] * mn0.x;
+        part = fmaf(qr[hd][1], mn0.y, part);
+        part = fmaf(qr[hd][2], mn1.x, part);
+        part = fmaf(qr[hd][3], mn1.y, part);
+        cst[hd] = warp_sum(part);
+        qv[hd][0] = qr[hd][0] * sc0.x;
+        qv[hd][1] = qr[hd][1] * sc0.y;
+        qv[hd][2] = qr[hd][2] * sc1.x;
+        qv[hd][3] = qr[hd][3] * sc1.y;
+      }
+      if (kind_k == kKindRaw && !C::kChunked) {
+        uint32_t* tab = m.table();
+        float invf[G];
+        build_i8tab<G, NT>(tab, qv, invf, lane);
+        __syncwarp();
+        qk_i8<BITS, G>(st, tab, cst, invf, sc, 128, a.scale, lane);
+      } else {
+        float2* qp = reinterpret_cast<float2*>(m.table());
+#pragma unroll
+        for (int hd = 0; hd < G; ++hd) {
+          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane)) =
+              make_float4(qv[hd][0], qv[hd][0], qv[hd][1], qv[hd][1]);
+          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane + 2)) =
+              make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
+        }
+        __syncwarp();
+        if (kind_k == kKindRaw) {
+          if constexpr (BITS == 3) qk_raw3<G>(st, qp, cst, sc, 128, a.scale, lane);
+        } else {
+          qk_packed<G>(st, qp, cst, sc, 128, a.scale, lane);
+        }
+      }
+    }
+    __syncwarp();
+    if (x + 1 < hi) {  // the K stage is free: the next item's K record
+      if (x + 1 - wk.base >= 32) wk.load(ka, x + 1, hi, lane);
+      issue_item<BITS, G, false>(ka, m, nc, wk.get(x + 1), 0, lane);
+    }
+
+    // ---- online softmax: running max and sum of exp per head, p of this lane's slots
+    float pr[G][4];
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      float sv[4];
+      float bm = kNegInf;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        sv[i] = (!skip && r < n_tok) ? sc[hd * 128 + r] : kNegInf;
+        bm = fmaxf(bm, sv[i]);
+      }
+      bm = warp_max(bm);
+      const float m_new = fmaxf(mrun[hd], bm);
+      float ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        pr[hd][i] = sv[i] == kNegInf ? 0.f : exp2f((sv[i] - m_new) * kLog2e);
+        ps += pr[hd][i];
+      }
+      ps = warp_sum(ps);
+      if (m_new > mrun[hd]) {  // warp-uniform: rescale what was summed under the old max
+        const float alpha = mrun[hd] == kNegInf ? 0.f : exp2f((mrun[hd] - m_new) * kLog2e);
+        lrun[hd] *= alpha;
+        mp[hd] *= alpha;
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) sacc[hd * 128 + sl * 32 + lane] *= alpha;
+#pragma unroll
+        for (int jn = 0; jn < NT; ++jn) {
+          if (2 * jn + (t >> 1) == hd) {
+#pragma unroll
+            for (int T = 0; T < 8; ++T) {
+              acc_lo[jn][T] *= alpha;
+              acc_hi[jn][T] *= alpha;
+            }
+          }
+        }
+        mrun[hd] = m_new;
+      }
+      lrun[hd] += ps;
+    }
+
+    // ---- V: add the probability-weighted values -------------------------------
+    ok = mbar_wait_bounded(m.bar(1), (phases >> 1) & 1u, a.ctrl);
+    phases ^= 2u;
+    if (!ok) {
+      if (x + 1 < hi) mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
+      return;
+    }
+    const int kind_v = *m.kind(1);
+    if (kind_v == kKindTail) {
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd)
+        *reinterpret_cast<float4*>(sc + hd * 128 + 4 * lane) = make_float4(pr[hd][0], pr[hd][1], pr[hd][2], pr[hd][3]);
+      __syncwarp();
+      tail_values<G>(a, bh, sc, sacc, lane);
+    } else if (kind_v == kKindInvalid) {
+      if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
+    } else if (!skip) {
+      const unsigned char* st = m.stage(1);
+      const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
+      const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
+      const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
+      const float2 mn1 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.y));
+      const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&scv.x));
+      const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&scv.y));
+      const float mnr[4] = {mn0.x, mn0.y, mn1.x, mn1.y};
+      const float scr[4] = {sc0.x, sc0.y, sc1.x, sc1.y};
+      float pv4[G][4];
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          mp[hd] = fmaf(pr[hd][i], mnr[i], mp[hd]);
+          pv4[hd][i] = pr[hd][i] * scr[i];
+        }
+      if (kind_v == kKindRaw && !C::kChunked) {
+        uint32_t* tab = m.table();
+        float invf[G];
+        build_i8tab<G, NT>(tab, pv4, invf, lane);
+        __syncwarp();
+        pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
+      } else {
+        float* pp = reinterpret_cast<float*>(m.table());  // p'' [G][128] then group sums [G][4]
+        const bool raw = kind_v == kKindRaw;
+#pragma unroll
+        for (int hd = 0; hd < G; ++hd) {
+          float o[4];
+          float ps = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            ps += pv4[hd][i];
+            const int r15 = (4 * lane + i) & 15;  // field position of slot r in a 2-bit slice word
+            const int sg = r15 <= 10 ? 2 * r15 : 2 * r15 - 12;
+            o[i] = raw ? pv4[hd][i] * exp2i(-sg) : pv4[hd][i];
+          }
+          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+          if (!raw) {
+            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+            if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
+          }
+        }
+        __syncwarp();
+        if (raw) {
+          if constexpr (BITS == 3) pv_raw3<G>(st, pp, sacc, lane);
+        } else {
+          pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
+        }
+      }
+    }
+    __syncwarp();
+    if (x + 1 < hi) {  // the V stage is free: the next item's V record
+      if (x + 1 - wv.base >= 32) wv.load(va, x + 1, hi, lane);
+      issue_item<BITS, G, false>(va, m, nc, wv.get(x + 1), 1, lane);
+    }
+    cc = nc;
+  }
+  (void)g;
+  if (cur_bh >= 0) attn_flush<G>(a, cur_bh, warp, sacc, acc_lo, acc_hi, mp, mrun, lrun, lane);
+}
+
+// Warp whose item range holds `item` (ranges are [floor(w*N/W), floor((w+1)*N/W)), W <= N).
+__device__ __forceinline__ long attn_warp_of_item(long item, long n_items, long n_warps) {
+  return (long)(((long long)(item + 1) * n_warps + n_items - 1) / n_items) - 1;
+}
+
+// Second pass: for each output row (b, h, head), the slots of the warps that touched
+// (b, h) are merged with the log-sum-exp rule, M = max m_w, L = sum l_w e^(m_w - M),
+// out_c = sum S_w,c e^(m_w - M) / L, adding in a fixed order (deterministic).  One CTA
+// per row: warp i of 16 takes slots w0+i, w0+i+16, ...; warp 0 adds the 16 warp
+// results in order.  A row whose every record was invalid gets NaN.
+constexpr int kMergeWarps = 16;
+
+template <int G>
+__global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const AttnArgs a) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ float4 wsum[kMergeWarps][32];
+  __shared__ float wl[kMergeWarps];
+  __shared__ float wmax[kMergeWarps];
+  const long row = blockIdx.x;  // (b*kv_heads + h)*G + head
+  const long bh = row / G;
+  const int hd = (int)(row % G);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long I = a.items_per_bh;
+  const long w0 = attn_warp_of_item(bh * I, a.n_items, a.n_warps) + bh;
+  const long w1 = attn_warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps) + bh;
+  const float* base = a.partials + hd * kSlotFloats;
+  const size_t stride = (size_t)G * kSlotFloats;
+  // the overall maximum
+  float mx = kNegInf;
+  for (long w = w0 + threadIdx.x; w <= w1; w += kMergeWarps * 32) mx = fmaxf(mx, __ldcg(base + w * stride + 128));
+  mx = warp_max(mx);
+  if (lane == 0) wmax[warp] = mx;
+  __syncthreads();
+  float M = wmax[0];
+#pragma unroll
+  for (int i = 1; i < kMergeWarps; ++i) M = fmaxf(M, wmax[i]);
+  // scaled sums
+  float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  float l = 0.f;
+  for (long w = w0 + warp; w <= w1; w += kMergeWarps) {
+    const float* p = base + w * stride;
+    const float mw = __ldcg(p + 128);
+    const float e = (mw == kNegInf) ? 0.f : exp2f((mw - M) * kLog2e);
+    const float4 x = __ldcg(reinterpret_cast<const float4*>(p) + lane);
+    s.x = fmaf(x.x, e, s.x);
+    s.y = fmaf(x.y, e, s.y);
+    s.z = fmaf(x.z, e, s.z);
+    s.w = fmaf(x.w, e, s.w);
+    l = fmaf(__ldcg(p + 129), e, l);
+  }
+  wsum[warp][lane] = s;
+  if (lane == 0) wl[warp] = l;
+  __syncthreads();
+  if (warp == 0) {
+    float4 r = wsum[0][lane];
+    float L = wl[0];
+#pragma unroll
+    for (int i = 1; i < kMergeWarps; ++i) {
+      const float4 x = wsum[i][lane];
+      r.x += x.x;
+      r.y += x.y;
+      r.z += x.z;
+      r.w += x.w;
+      L += wl[i];
+    }
+    const float inv = L > 0.f ? 1.f / L : __int_as_float(0x7fc00000);
+    reinterpret_cast<float4*>(a.out + row * 128)[lane] = make_float4(r.x * inv, r.y * inv, r.z * inv, r.w * inv);
+  }
+}
+
+struct AttnKernel {
+  const void* fn;
+  int smem;
+};
+
+template <int BITS, int G>
+AttnKernel attn_info() {
+  return {reinterpret_cast<const void*>(&attn_kernel<BITS, G>), kAttnWarps * AttnCfg<BITS, G>::kWarpSmem};
+}
+
+bool attn_select(int bits, int group, AttnKernel* out) {
+#define PACKKV_ACASE(B, GG)          \
+  if (bits == B && group == GG) {    \
+    *out = attn_info<B, GG>();       \
+    return true;                     \
+  }
+  PACKKV_ACASE(4, 1) PACKKV_ACASE(4, 2) PACKKV_ACASE(4, 4) PACKKV_ACASE(4, 8)
+  PACKKV_ACASE(3, 1) PACKKV_ACASE(3, 2) PACKKV_ACASE(3, 4) PACKKV_ACASE(3, 8)
+  PACKKV_ACASE(2, 1) PACKKV_ACASE(2, 2) PACKKV_ACASE(2, 4) PACKKV_ACASE(2, 8)
+#undef PACKKV_ACASE
+  return false;
+}
+
+// Resident warps of the kernel on the current device (configures the smem limit once).
+cudaError_t attn_resident_warps(const AttnKernel& k, int* warps) {
+  static std::mutex mu;
+  static std::unordered_map<long long, int> cache;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const long long key = (long long)(reinterpret_cast<uintptr_t>(k.fn)) * 64 + dev;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) {
+    *warps = it->second;
+    return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0, sms = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k.fn, kAttnWarps * 32, k.smem);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int w = sms * per_sm * kAttnWarps;
+  cache[key] = w;
+  *warps = w;
+  return cudaSuccess;
+}
+
+int attn_max_warps() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms * 64;
+}
+
+}  // namespace
+
+size_t attention_workspace_bytes(int batch, int kv_heads, int group) {
+  const size_t bh = (size_t)batch * kv_heads;
+  return ((size_t)attn_max_warps() + bh) * group * kSlotFloats * sizeof(float);
+}
+
+cudaError_t launch_attention(AttnArgs a, cudaStream_t stream) {
+  AttnKernel k{};
+  if (!attn_select(a.bits, a.group, &k)) return cudaErrorInvalidValue;
+  int w = 0;
+  cudaError_t e = attn_resident_warps(k, &w);
+  if (e != cudaSuccess) return e;
+  if (w > attn_max_warps()) w = attn_max_warps();
+  a.n_warps = (int)(a.n_items < w ? a.n_items : w);
+  const unsigned grid = (unsigned)((a.n_warps + kAttnWarps - 1) / kAttnWarps);
+  void* args[] = {&a};
+  e = cudaLaunchKernel(k.fn, dim3(grid), dim3(kAttnWarps * 32), args, k.smem, stream);
+  if (e != cudaSuccess) return e;
+  const void* merge = nullptr;
+  switch (a.group) {
+    case 1: merge = reinterpret_cast<const void*>(&attn_merge_kernel<1>); break;
+    case 2: merge = reinterpret_cast<const void*>(&attn_merge_kernel<2>); break;
+    case 4: merge = reinterpret_cast<const void*>(&attn_merge_kernel<4>); break;
+    default: merge = reinterpret_cast<const void*>(&attn_merge_kernel<8>); break;
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)((long)a.batch * a.kv_heads * a.group));
+  cfg.blockDim = dim3(kMergeWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, merge, args);
+}
+
+}  // namespace packkv

@@ -1,0 +1,785 @@
+// Device building blocks of the fused decode products over the packed cache:
+// record staging (bulk copies into warp-private shared-memory stages, bounded
+// mbarrier waits), the 8-bit integer tensor-core decode of raw 2/4-bit records,
+// and the CUDA-core decode of raw 3-bit and compressed records (FORMAT.md
+// sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused
+// attention kernel.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace packkv {
+
+namespace {
+
+#ifndef PACKKV_WARPS_PER_CTA
+#define PACKKV_WARPS_PER_CTA 4
+#endif
+constexpr int kWarpsPerCta = PACKKV_WARPS_PER_CTA;
+#ifndef PACKKV_WARP_SMEM_KB
+#define PACKKV_WARP_SMEM_KB 10  // shared memory per warp: one 4-bit stage, five CTAs of 4 warps per SM
+#endif
+constexpr int kWarpSmemBudget = PACKKV_WARP_SMEM_KB * 1024;
+constexpr uint32_t kMagicBits = 0x4B000000u;
+constexpr float kMagic = 8388608.0f;
+constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer in the low bits
+constexpr int kRoundBits = 0x4B400000;
+
+enum ItemKind : int { kKindRaw = 0, kKindPacked = 1, kKindInvalid = 2, kKindTail = 3 };
+
+// (w & mask) | 0x4B000000 in one LOP3: the field lands in the low mantissa bits of 2^23.
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t fld(uint32_t w) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(kMagicBits));
+  return d;
+}
+
+// Two magic-number fields -> their exact values, with one packed FP32 add.
+__device__ __forceinline__ float2 pairf(uint32_t a, uint32_t b) {
+  return __fadd2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), make_float2(-kMagic, -kMagic));
+}
+
+// Field position exponent of token i (0..15) in the 2-bit decode below (value = field * 2^sig2).
+__host__ __device__ constexpr int sig2(int i) { return i <= 10 ? 2 * i : 2 * i - 12; }
+__host__ __device__ constexpr float pow2(int e) {
+  return e >= 0 ? float(1u << e) : 1.0f / float(1u << (-e));
+}
+// 2^e for a run-time e in [-126, 127], from the exponent bits (no division)
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+template <int I>
+__device__ __forceinline__ uint32_t fld2(uint32_t w, uint32_t h) {
+  if constexpr (I <= 10)
+    return fld<(3u << (2 * I))>(w);
+  else
+    return fld<(3u << (2 * I - 12))>(h);
+}
+
+// 16 two-bit fields of a 2-bit slice word as 8 pairs: field_i * 2^sig2(i)
+__device__ __forceinline__ void dec2(uint32_t w, float2 (&v)[8]) {
+  const uint32_t h = w >> 12;
+  v[0] = pairf(fld2<0>(w, h), fld2<1>(w, h));
+  v[1] = pairf(fld2<2>(w, h), fld2<3>(w, h));
+  v[2] = pairf(fld2<4>(w, h), fld2<5>(w, h));
+  v[3] = pairf(fld2<6>(w, h), fld2<7>(w, h));
+  v[4] = pairf(fld2<8>(w, h), fld2<9>(w, h));
+  v[5] = pairf(fld2<10>(w, h), fld2<11>(w, h));
+  v[6] = pairf(fld2<12>(w, h), fld2<13>(w, h));
+  v[7] = pairf(fld2<14>(w, h), fld2<15>(w, h));
+}
+
+// 3-bit raw unit, 16 tokens: 2-bit slice word w2 plus the 16 slice-1 bits at bits 0..15 of x.
+// v[p] = (field2 + 4*bit) * 2^sig2, merged with one exact packed FMA per pair.
+__device__ __forceinline__ void dec3(uint32_t w2, uint32_t x, float2 (&v)[8]) {
+  dec2(w2, v);
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const int i = 2 * p;
+    const float2 b = pairf(x & (1u << i) | kMagicBits, x & (2u << i) | kMagicBits);
+    v[p] = __ffma2_rn(b, make_float2(pow2(sig2(i) - i + 2), pow2(sig2(i + 1) - i + 1)), v[p]);
+  }
+}
+
+template <int BITS, int G, bool PV>
+struct Cfg {
+  static constexpr int kRecBytes = raw_record_bytes(BITS);
+  // b = 3 raw records are staged as 16 chunks (group g, channel quarter h: 32 units of
+  // 3 words) at a padded pitch (bank-conflict-free decode); b = 2 / 4 raw records are
+  // in fragment order and are staged in one piece, as are compressed records.
+  static constexpr bool kChunked = BITS == 3;
+  static constexpr int kChunks = 16, kChunkBytes = 384, kPitch = 400;
+  static constexpr int kStageRec = kChunked ? 528 + kChunks * kPitch : kRecBytes;  // >= every record
+  static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);              // p·V: + p rows
+  // int8 tensor-core B table: columns n = 4*head + digit (digit 3 = 0), NT n-tiles of 8
+  static constexpr int kNT = (4 * G + 7) / 8;
+  static constexpr int kI8Tab = 4 * (64 * kNT + 8) * 4;
+  // CUDA-core tables: q' pairs [G][128] (q·Kᵀ); p'' [G][128] + group sums of p' [G][4] (p·V)
+  static constexpr int kCoreTab = PV ? 512 * G + 16 * G : 1024 * G;
+  static constexpr int kTableBytes = ((kCoreTab > kI8Tab ? kCoreTab : kI8Tab) + 15) / 16 * 16;
+  static constexpr int kSumBytes = PV ? 512 * G : 0;          // p·V: [G][128] channel sums
+  static constexpr int kFixed = kTableBytes + kSumBytes;
+  static constexpr int kStages0 = (kWarpSmemBudget - kFixed - 64) / kStageBytes;
+  static constexpr int kStages = kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0);
+  static constexpr int kWarpSmem = ((kStages * kStageBytes + kFixed + kStages * 16) + 127) / 128 * 128;
+  static_assert(kStageBytes % 16 == 0 && kFixed % 16 == 0, "stage alignment");
+};
+
+// Warp-private shared memory: [stages][table][channel sums (p·V)][mbarriers][kinds].
+template <int BITS, int G, bool PV>
+struct WarpMem {
+  using C = Cfg<BITS, G, PV>;
+  unsigned char* base;
+  __device__ unsigned char* stage(int s) const { return base + s * C::kStageBytes; }
+  __device__ unsigned char* fixed() const { return base + C::kStages * C::kStageBytes; }
+  __device__ uint32_t* table() const { return reinterpret_cast<uint32_t*>(fixed()); }
+  __device__ float* sums() const { return reinterpret_cast<float*>(fixed() + C::kTableBytes); }
+  __device__ uint64_t* bar(int s) const { return reinterpret_cast<uint64_t*>(fixed() + C::kFixed) + s; }
+  __device__ int* kind(int s) const {
+    return reinterpret_cast<int*>(fixed() + C::kFixed + C::kStages * 8) + s;
+  }
+};
+
+// CUDA-core q' table of q·Kᵀ: (q'_c, q'_c) pairs; channel c = 32*h + cc sits at float2
+// index ((cc/2)*4 + h)*2 + cc%2, so that a 16-byte load gives a lane of the 3-bit
+// decode (chunk h) its next two channels.
+__device__ __forceinline__ int table_index(int c) {
+  const int h = c >> 5, cc = c & 31;
+  return ((cc >> 1) * 4 + h) * 2 + (cc & 1);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-byte shared-memory load that the compiler issues where it stands (keeps it from
+// hoisting a whole table of loop-invariant loads into registers).
+__device__ __forceinline__ float4 lds_f4(const float* p) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(smem_addr(p)));
+  return r;
+}
+
+// Position in the flat item list: (sequence*kv_heads + head, item within it).
+struct Cursor {
+  long bh;
+  int j;
+  __device__ void next(int items_per_bh) {
+    if (++j == items_per_bh) {
+      j = 0;
+      ++bh;
+    }
+  }
+};
+
+// Index entries {offset16, length16} of 32 consecutive items of a warp's range, one
+// per lane ({0, 0} for a tail item or past the range), loaded with one coalesced
+// load; any lane reads the entry of any item of the window by shuffle.
+struct EntryWindow {
+  long base;  // first item of the window
+  uint2 ent;  // entry of item base + lane
+  __device__ void load(const GemvArgs& a, long first, long hi, int lane) {
+    base = first;
+    ent = make_uint2(0u, 0u);
+    const long item = first + lane;
+    if (item < hi) {
+      const long bh = item / a.items_per_bh;
+      const int j = (int)(item % a.items_per_bh);
+      if (j < a.n_blocks) ent = *reinterpret_cast<const uint2*>(a.index + ((size_t)bh * a.max_blocks + j) * 2);
+    }
+  }
+  // Whole warp; base <= item < base + 32.
+  __device__ uint2 get(long item) const {
+    const int src = (int)(item - base);
+    return make_uint2(__shfl_sync(0xffffffffu, ent.x, src), __shfl_sync(0xffffffffu, ent.y, src));
+  }
+};
+
+// Issue the copies of item (bh, j) with index entry e into stage s of m (whole warp
+// participates); m provides stage(s), bar(s) and kind(s).
+template <int BITS, int G, bool PV, class Mem>
+__device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Cursor c, uint2 e, int s, int lane) {
+  using C = Cfg<BITS, G, PV>;
+  const long bh = c.bh;
+  const int j = c.j;
+  int kind = kKindTail;
+  uint64_t off16 = 0;
+  uint32_t len16 = 0;
+  if (j < a.n_blocks) {
+    off16 = e.x;
+    len16 = e.y;
+    const bool valid = e.x != 0xFFFFFFFFu && len16 >= 1040 / 16 && len16 * 16u <= (uint32_t)C::kRecBytes &&
+                       off16 + len16 <= a.arena16;
+    kind = !valid ? kKindInvalid : (len16 * 16u == (uint32_t)C::kRecBytes ? kKindRaw : kKindPacked);
+  }
+  unsigned char* st = m.stage(s);
+  const unsigned char* src = a.arena + off16 * 16;
+  if (lane == 0) {
+    *m.kind(s) = kind;
+    uint32_t bytes = 0;
+    if (kind == kKindRaw) bytes = C::kRecBytes;
+    if (kind == kKindPacked) bytes = len16 * 16u;
+    if (PV && bytes) bytes += 512u * G;
+    fence_async_smem();
+    if (bytes)
+      mbar_arrive_expect_tx(m.bar(s), bytes);
+    else
+      mbar_arrive(m.bar(s));
+  }
+  __syncwarp();
+  if (kind == kKindRaw && C::kChunked) {
+    if (lane < C::kChunks)
+      bulk_g2s(st + 528 + lane * C::kPitch, src + 528 + lane * C::kChunkBytes, C::kChunkBytes, m.bar(s));
+    if (lane == 16) bulk_g2s(st, src, 528, m.bar(s));
+  } else if (kind == kKindRaw) {
+    if (lane == 16) bulk_g2s(st, src, C::kRecBytes, m.bar(s));
+  } else if (kind == kKindPacked) {
+    if (lane == 16) bulk_g2s(st, src, len16 * 16u, m.bar(s));
+  }
+  if (PV && (kind == kKindRaw || kind == kKindPacked) && lane >= 24 && lane < 24 + G) {
+    const int hd = lane - 24;
+    const long b = bh / a.kv_heads, h = bh % a.kv_heads;
+    const long hq = h * G + hd;
+    const float* prow = a.p + ((size_t)b * a.kv_heads * G + hq) * a.ld + (size_t)j * 128;
+    bulk_g2s(st + C::kStageRec + hd * 512, prow, 512, m.bar(s));
+  }
+}
+
+// After a wait gave up: waits, bounded, for the warp's other copies in flight
+// (items x+1 .. prod-1) so that none lands after the warp has exited.
+template <int BITS, int G, bool PV>
+__device__ void drain_stages(const WarpMem<BITS, G, PV>& m, uint32_t phases, int s, long x, long prod,
+                             uint64_t* ctrl) {
+  using C = Cfg<BITS, G, PV>;
+  for (long i = x + 1; i < prod; ++i) {
+    const int si = (int)((s + (i - x)) % C::kStages);
+    mbar_wait_bounded(m.bar(si), (phases >> si) & 1u, ctrl);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 8-bit integer tensor-core decode of raw b = 2 / 4 records (FORMAT.md section 4)
+// ----------------------------------------------------------------------------
+// D(16x8, s32) += A(16x32, u8) * B(32x8, s8): exact integer products and sums.
+__device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Exact float of an integer |d| < 2^22.
+__device__ __forceinline__ float i2f_small(int d) { return __int_as_float(d + kRoundBits) - kRound; }
+
+// The low bytes of four floats of the form r + 1.5*2^23 (r an integer, |r| <= 127):
+// the two's-complement bytes of r, packed in order.
+__device__ __forceinline__ uint32_t pack4(float2 lo, float2 hi) {
+  const uint32_t x0 = __float_as_uint(lo.x), x1 = __float_as_uint(lo.y);
+  const uint32_t x2 = __float_as_uint(hi.x), x3 = __float_as_uint(hi.y);
+  return __byte_perm(__byte_perm(x0, x1, 0x0040), __byte_perm(x2, x3, 0x0040), 0x5410);
+}
+
+// Word of the int8 B table holding B[k = 32*kap + 16*kh + 4*t .. +3][n], read by lane
+// 4*(n%8) + t as b_kh of n-tile n/8; a lane's words for one k-step are consecutive.
+template <int NT>
+__device__ __forceinline__ int i8tab_word(int kap, int kh, int t, int n) {
+  return kap * (64 * NT + 8) + (4 * (n & 7) + t) * 2 * NT + kh * NT + (n >> 3);
+}
+
+// B table of the int8 products for one record: lane holds x[head][i] for k = 4*lane + i
+// (channel for q·Kᵀ, storage slot for p·V).  Per head f = 127 / max|x| and
+// y = x*f = d0 + d1/128 + d2/16384 with integer digits |d0| <= 127, |d1|, |d2| <= 64
+// (each the rounding of the remainder so far, so |y - sum| <= 2^-15); column
+// 4*head + i holds digit i (column 4*head + 3 and the columns of absent heads are
+// zero).  Returns 1/f per head.
+template <int G, int NT>
+__device__ __forceinline__ void build_i8tab(uint32_t* tab, const float (&x)[G][4], float (&invf)[G], int lane) {
+  const int kap = lane >> 3, kh = (lane >> 2) & 1, t = lane & 3;
+  const float2 R = make_float2(kRound, kRound), nR = make_float2(-kRound, -kRound);
+  const float2 k128 = make_float2(128.f, 128.f);
+#pragma unroll
+  for (int hd = 0; hd < 2 * NT; ++hd) {
+    uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
+    if (hd < G) {
+      const int h = hd < G ? hd : 0;
+      const float mx =
+          warp_max(fmaxf(fmaxf(fabsf(x[h][0]), fabsf(x[h][1])), fmaxf(fabsf(x[h][2]), fabsf(x[h][3]))));
+      const float f = mx > 0.f ? __fdividef(127.f, mx) : 1.f;
+      invf[h] = mx > 0.f ? __fdividef(mx, 127.f) : 1.f;
+      const float2 m128 = make_float2(-128.f, -128.f);
+      float2 t0[2], t1[2], t2[2];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float2 y = __fmul2_rn(make_float2(x[h][2 * q], x[h][2 * q + 1]), make_float2(f, f));
+        y = make_float2(fminf(fmaxf(y.x, -127.f), 127.f), fminf(fmaxf(y.y, -127.f), 127.f));
+        t0[q] = __fadd2_rn(y, R);                                          // low byte: d0 = rint(y)
+        const float2 r1 = __ffma2_rn(__fadd2_rn(t0[q], nR), m128, __fmul2_rn(y, k128));  // 128(y - d0), exact
+        t1[q] = __fadd2_rn(r1, R);                                         // low byte: d1 = rint(r1)
+        const float2 r2 = __ffma2_rn(__fadd2_rn(t1[q], nR), m128, __fmul2_rn(r1, k128));  // 128(r1 - d1), exact
+        t2[q] = __fadd2_rn(r2, R);                                         // low byte: d2 = rint(r2)
+      }
+      w0 = pack4(t0[0], t0[1]);
+      w1 = pack4(t1[0], t1[1]);
+      w2 = pack4(t2[0], t2[1]);
+    }
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 0)] = w0;
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 1)] = w1;
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 2)] = w2;
+    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 3)] = 0u;
+  }
+}
+
+// B fragments of this lane: bf[kap][j] = {b0, b1} of n-tile j at k-step kap.
+template <int NT>
+__device__ __forceinline__ void load_i8frags(const uint32_t* tab, uint32_t (&bf)[4][NT][2], int lane) {
+#pragma unroll
+  for (int kap = 0; kap < 4; ++kap) {
+    const uint32_t* p = tab + kap * (64 * NT + 8) + lane * 2 * NT;  // [kh][j] words
+    if constexpr (NT == 1) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      bf[kap][0][0] = v.x;
+      bf[kap][0][1] = v.y;
+    } else {
+#pragma unroll
+      for (int q = 0; q < NT / 2; ++q) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p + 4 * q);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int idx = 4 * q + r, kh = idx / NT, j = idx % NT;
+          bf[kap][j][kh] = w4[r];
+        }
+      }
+    }
+  }
+}
+
+// Sum of the three digit columns of an accumulator tile (thread (g, t) holds columns
+// 2t, 2t+1 = digits (0, 1) of head 2j + t/2 for even t, digit 2 and the zero column
+// for odd t): returns, in even-t threads, D0 + D1/128 + D2/16384 for rows g (lo) and
+// g + 8 (hi).
+__device__ __forceinline__ void digit_sum(const int (&d)[4], int t, float& lo, float& hi) {
+  const float w0 = (t & 1) ? 1.f / 16384.f : 1.f, w1 = (t & 1) ? 0.f : 1.f / 128.f;
+  lo = fmaf(i2f_small(d[1]), w1, i2f_small(d[0]) * w0);
+  hi = fmaf(i2f_small(d[3]), w1, i2f_small(d[2]) * w0);
+  lo += __shfl_down_sync(0xffffffffu, lo, 1);
+  hi += __shfl_down_sync(0xffffffffu, hi, 1);
+}
+
+// Selects the value of a run-time head index from a register array.
+template <int G>
+__device__ __forceinline__ float head_sel(const float (&x)[G], int head) {
+  float r = 0.f;
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd)
+    if (head == hd) r = x[hd];
+  return r;
+}
+
+// A registers of one row tile from its two fragment words (k halves kh = 0, 1).
+// b = 4: rows g (low nibbles, x1) and g + 8 (high nibbles, x16).
+__device__ __forceinline__ void afrag4(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
+  a[0] = w0 & 0x0F0F0F0Fu;
+  a[1] = w0 & 0xF0F0F0F0u;
+  a[2] = w1 & 0x0F0F0F0Fu;
+  a[3] = w1 & 0xF0F0F0F0u;
+}
+
+// b = 2: even tile rows g (x1), g + 8 (x4); odd tile rows g (x16), g + 8 (x64).
+__device__ __forceinline__ void afrag2(uint32_t w0, uint32_t w1, uint32_t (&ae)[4], uint32_t (&ao)[4]) {
+  ae[0] = w0 & 0x03030303u;
+  ae[1] = w0 & 0x0C0C0C0Cu;
+  ae[2] = w1 & 0x03030303u;
+  ae[3] = w1 & 0x0C0C0C0Cu;
+  ao[0] = w0 & 0x30303030u;
+  ao[1] = w0 & 0xC0C0C0C0u;
+  ao[2] = w1 & 0x30303030u;
+  ao[3] = w1 & 0xC0C0C0C0u;
+}
+
+// 1 / (power of two carried by the A fields) of row g (upper = 0) or g + 8 of a tile.
+template <int BITS>
+__host__ __device__ constexpr float row_unscale(int odd_tile, int upper) {
+  return BITS == 4 ? (upper ? 1.f / 16.f : 1.f)
+                   : (odd_tile ? (upper ? 1.f / 64.f : 1.f / 16.f) : (upper ? 0.25f : 1.f));
+}
+
+// Runs the tensor-core product of one raw b = 2 / 4 record: for every row tile T
+// (16 rows) calls emit(T, n-tile j, d) with the exact integer tile d.  Rows are
+// slots (q·Kᵀ, K record) or channels (p·V, V record).
+template <int BITS, int NT, class Emit>
+__device__ __forceinline__ void i8_product(const unsigned char* st, const uint32_t (&bf)[4][NT][2], int lane,
+                                           Emit&& emit) {
+  const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
+  constexpr int kRows = BITS == 4 ? 8 : 4;  // word rows: tiles (b = 4) or tile pairs (b = 2)
+#pragma unroll
+  for (int tp = 0; tp < kRows; ++tp) {
+    const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
+    // k-step kap: words (kh 0, kh 1) = (wa.x, wa.y), (wa.z, wa.w), (wb.x, wb.y), (wb.z, wb.w)
+    const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
+    if constexpr (BITS == 4) {
+      int d[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0;
+#pragma unroll
+      for (int kap = 0; kap < 4; ++kap) {
+        uint32_t a[4];
+        afrag4(w[kap][0], w[kap][1], a);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) imma16832(d[j], a, bf[kap][j][0], bf[kap][j][1]);
+      }
+#pragma unroll
+      for (int j = 0; j < NT; ++j) emit(tp, j, d[j]);
+    } else {
+      int de[NT][4], dd[NT][4];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        de[j][0] = de[j][1] = de[j][2] = de[j][3] = 0;
+        dd[j][0] = dd[j][1] = dd[j][2] = dd[j][3] = 0;
+      }
+#pragma unroll
+      for (int kap = 0; kap < 4; ++kap) {
+        uint32_t ae[4], ao[4];
+        afrag2(w[kap][0], w[kap][1], ae, ao);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          imma16832(de[j], ae, bf[kap][j][0], bf[kap][j][1]);
+          imma16832(dd[j], ao, bf[kap][j][0], bf[kap][j][1]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        emit(2 * tp, j, de[j]);
+        emit(2 * tp + 1, j, dd[j]);
+      }
+    }
+  }
+}
+
+// q·Kᵀ of one raw b = 2 / 4 K record: scores of all 128 slots for the G heads.
+template <int BITS, int G>
+__device__ __forceinline__ void qk_i8(const unsigned char* st, const uint32_t* tab, const float (&cst)[G],
+                                      const float (&invf)[G], float* sblk, long ld, float scale, int lane) {
+  constexpr int NT = (4 * G + 7) / 8;
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t bf[4][NT][2];
+  load_i8frags<NT>(tab, bf, lane);
+  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, const int (&d)[4]) {
+    float lo, hi;
+    digit_sum(d, t, lo, hi);
+    const int head = 2 * j + (t >> 1);
+    if ((t & 1) == 0 && head < G) {
+      const float f = head_sel<G>(invf, head), c = head_sel<G>(cst, head);
+      float* dst = sblk + head * ld + 16 * T + g;
+      dst[0] = scale * fmaf(lo, f * row_unscale<BITS>(T & 1, 0), c);
+      dst[8] = scale * fmaf(hi, f * row_unscale<BITS>(T & 1, 1), c);
+    }
+  });
+}
+
+// p·V of one raw b = 2 / 4 V record: adds sum_slots p'*code into the accumulators of
+// channels 16T + g (acc_lo) and 16T + g + 8 (acc_hi) of head 2j + t/2 (even t).
+template <int BITS, int G>
+__device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* tab, const float (&invf)[G],
+                                      float (&acc_lo)[(4 * G + 7) / 8][8], float (&acc_hi)[(4 * G + 7) / 8][8],
+                                      int lane) {
+  constexpr int NT = (4 * G + 7) / 8;
+  const int t = lane & 3;
+  uint32_t bf[4][NT][2];
+  load_i8frags<NT>(tab, bf, lane);
+  float f_t[NT];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) f_t[j] = head_sel<G>(invf, 2 * j + (t >> 1));
+  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, const int (&d)[4]) {
+    float lo, hi;
+    digit_sum(d, t, lo, hi);
+    acc_lo[j][T] = fmaf(lo, f_t[j] * row_unscale<BITS>(T & 1, 0), acc_lo[j][T]);
+    acc_hi[j][T] = fmaf(hi, f_t[j] * row_unscale<BITS>(T & 1, 1), acc_hi[j][T]);
+  });
+}
+
+// ----------------------------------------------------------------------------
+// q·Kᵀ on the CUDA cores
+// ----------------------------------------------------------------------------
+// One raw b = 3 K record: lane (g, k, h) decodes tokens 32g + 16k .. +15 over the 32
+// channels of chunk 4g + h (a 4-lane reduction over h finishes), heads in chunks of
+// at most four (the words are decoded once per chunk).
+template <int G>
+__device__ __forceinline__ void qk_raw3(const unsigned char* st, const float2* qp, const float (&cst)[G],
+                                        float* sblk, long ld, float scale, int lane) {
+  using C = Cfg<3, G, false>;
+  constexpr int HC = G > 4 ? 4 : G;
+  const int h = lane & 3, k = (lane >> 2) & 1, g = lane >> 3;
+  const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + h) * C::kPitch);
+#pragma unroll 1
+  for (int h0 = 0; h0 < G; h0 += HC) {
+    float2 acc[HC][8];
+#pragma unroll
+    for (int hd = 0; hd < HC; ++hd)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[hd][i] = make_float2(0.f, 0.f);
+#pragma unroll 2
+    for (int c2 = 0; c2 < 16; ++c2) {
+      float2 v0[8], v1[8];
+      dec3(wp[3 * (2 * c2) + k], wp[3 * (2 * c2) + 2] >> (16 * k), v0);
+      dec3(wp[3 * (2 * c2 + 1) + k], wp[3 * (2 * c2 + 1) + 2] >> (16 * k), v1);
+#pragma unroll
+      for (int hd = 0; hd < HC; ++hd) {
+        const float4 qq = *reinterpret_cast<const float4*>(qp + (h0 + hd) * 128 + (c2 * 4 + h) * 2);
+        const float2 q0 = make_float2(qq.x, qq.y), q1 = make_float2(qq.z, qq.w);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          acc[hd][i] = __ffma2_rn(q0, v0[i], acc[hd][i]);
+          acc[hd][i] = __ffma2_rn(q1, v1[i], acc[hd][i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int hd = 0; hd < HC; ++hd) {
+      float tt[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float x = acc[hd][i].x, y = acc[hd][i].y;
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        y += __shfl_xor_sync(0xffffffffu, y, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        y += __shfl_xor_sync(0xffffffffu, y, 2);
+        tt[2 * i] = x;
+        tt[2 * i + 1] = y;
+      }
+      float o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < 4; ++hh)
+          if (h == hh) v = tt[4 * hh + i] * pow2(-sig2(4 * hh + i));
+        o[i] = scale * (head_sel<G>(cst, h0 + hd) + v);
+      }
+      float* dst = sblk + (h0 + hd) * ld + 32 * g + 16 * k + 4 * h;
+      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// Extracts the offset of token j from a compressed unit of width w starting at word s.
+__device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, int j) {
+  uint32_t u = 0;
+  if (w == 4) {
+    u = (W[s + (j >> 3)] >> ((j & 7) * 4)) & 15u;
+  } else if (w >= 2) {
+    u = (W[s + (j >> 4)] >> ((j & 15) * 2)) & 3u;
+    if (w == 3) u |= ((W[s + 2] >> j) & 1u) << 2;
+  } else if (w == 1) {
+    u = (W[s] >> j) & 1u;
+  }
+  return u;
+}
+
+// One compressed K record, lane = token within each pack group.
+template <int G>
+__device__ __forceinline__ void qk_packed(const unsigned char* st, const float2* qp, const float (&cst)[G],
+                                          float* sblk, long ld, float scale, int lane) {
+  const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
+  const uint8_t* meta = st + kMetaOffset;
+  const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    // base term of this group: sum_c q'_c base_gc, lane covers channels 4*lane..4*lane+3
+    float bsum[G];
+    const uint32_t m4 = *reinterpret_cast<const uint32_t*>(meta + g * 128 + 4 * lane);
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        part = fmaf(qp[hd * 128 + table_index(4 * lane + i)].x, (float)((m4 >> (8 * i)) & 15u), part);
+      bsum[hd] = warp_sum(part);
+    }
+    float acc[G];
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) acc[hd] = 0.f;
+    int s = gws[g];
+#pragma unroll 1
+    for (int c4 = 0; c4 < 32; ++c4) {
+      const uint32_t mm = *reinterpret_cast<const uint32_t*>(meta + g * 128 + 4 * c4);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int w = (mm >> (8 * i + 4)) & 15u;
+        const float u = (float)unit_field(W, s, w, lane);
+        s += w;
+#pragma unroll
+        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(qp[hd * 128 + table_index(4 * c4 + i)].x, u, acc[hd]);
+      }
+    }
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) sblk[hd * ld + 32 * g + lane] = scale * (cst[hd] + bsum[hd] + acc[hd]);
+  }
+}
+
+template <int G>
+__device__ __forceinline__ void qk_tail(const GemvArgs& a, long bh, const float (&qr)[G][4], float* srow0,
+                                        int lane) {
+  const uint16_t* tail = a.tail + (size_t)bh * 128 * 128;
+  for (int t0 = 0; t0 < a.tail_len; t0 += 32) {
+    float mine[G];
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) mine[hd] = 0.f;
+    const int tn = min(32, a.tail_len - t0);
+    for (int t = 0; t < tn; ++t) {
+      const uint2 hv = *reinterpret_cast<const uint2*>(tail + (size_t)(t0 + t) * 128 + 4 * lane);
+      const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+      const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        float part = qr[hd][0] * f0.x;
+        part = fmaf(qr[hd][1], f0.y, part);
+        part = fmaf(qr[hd][2], f1.x, part);
+        part = fmaf(qr[hd][3], f1.y, part);
+        part = warp_sum(part);
+        if (lane == t) mine[hd] = part;
+      }
+    }
+    if (lane < tn) {
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) srow0[hd * a.ld + (long)a.n_blocks * 128 + t0 + lane] = a.scale * mine[hd];
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// p·V on the CUDA cores
+// ----------------------------------------------------------------------------
+// One raw b = 3 V record, lane = channel sl*32 + lane; adds into the warp's shared
+// [G][128] channel sums.  The field exponents are folded into p'' = p * scale *
+// 2^-sig (pp: [G][128] by storage slot).
+template <int G>
+__device__ __forceinline__ void pv_raw3(const unsigned char* st, const float* pp, float* sacc, int lane) {
+  using C = Cfg<3, G, true>;
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+#pragma unroll 1
+    for (int sl = 0; sl < 4; ++sl) {
+      const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 12);
+      const uint32_t w2 = wp[2];
+      float2 v[2][8];
+      dec3(wp[0], w2, v[0]);        // slots 32g .. 32g+15
+      dec3(wp[1], w2 >> 16, v[1]);  // slots 32g+16 .. 32g+31
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        float2 a0 = make_float2(0.f, 0.f), a1 = a0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 x = lds_f4(pp + hd * 128 + 32 * g + 4 * q);
+          a0 = __ffma2_rn(make_float2(x.x, x.y), v[q >> 2][2 * (q & 3)], a0);
+          a1 = __ffma2_rn(make_float2(x.z, x.w), v[q >> 2][2 * (q & 3) + 1], a1);
+        }
+        sacc[hd * 128 + sl * 32 + lane] += (a0.x + a0.y) + (a1.x + a1.y);
+      }
+    }
+  }
+}
+
+// One compressed V record, lane = channel sl*32 + lane; adds into the warp's shared
+// [G][128] channel sums.  pg[hd*4 + g] = sum of p' over pack group g.
+template <int G>
+__device__ __forceinline__ void pv_packed(const unsigned char* st, const float* pp, const float* pg, float* sacc,
+                                          int lane) {
+  const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
+  const uint8_t* meta = st + kMetaOffset;
+  const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    int carry = gws[g];
+#pragma unroll 1
+    for (int sl = 0; sl < 4; ++sl) {
+      const int c = sl * 32 + lane;
+      const uint32_t mb = meta[g * 128 + c];
+      const int w = (int)(mb >> 4), base = (int)(mb & 15u);
+      int incl = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const int start = carry + incl - w;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll 1
+      for (int hd = 0; hd < G; ++hd) {
+        const float* pr = pp + hd * 128 + 32 * g;
+        float sum = (float)base * pg[hd * 4 + g];
+        if (w == 4) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t word = W[start + q];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum = fmaf(pr[8 * q + i], (float)((word >> (4 * i)) & 15u), sum);
+          }
+        } else {
+          int at = start;
+          float lo_mul = 1.f;
+          if (w & 2) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+              const uint32_t word = W[at + q];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) sum = fmaf(pr[16 * q + i], (float)((word >> (2 * i)) & 3u), sum);
+            }
+            at += 2;
+            lo_mul = 4.f;
+          }
+          if (w & 1) {
+            const uint32_t word = W[at];
+            float s1 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s1 = fmaf(pr[i], (float)((word >> i) & 1u), s1);
+            sum = fmaf(lo_mul, s1, sum);
+          }
+        }
+        sacc[hd * 128 + c] += sum;
+      }
+    }
+  }
+}
+
+// The fp16 tail of one (sequence, head), lane = channel sl*32 + lane; adds into the
+// warp's shared [G][128] channel sums.
+template <int G>
+__device__ __forceinline__ void pv_tail(const GemvArgs& a, long bh, float* sacc, int lane) {
+  const long b = bh / a.kv_heads, h = bh % a.kv_heads;
+  const uint16_t* tail = a.tail + (size_t)bh * 128 * 128;
+  float acc[4][G];
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) acc[sl][hd] = 0.f;
+  for (int t = 0; t < a.tail_len; ++t) {
+    float vv[4];
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) {
+      const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)a.n_blocks * 128 + t];
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = fmaf(pt, vv[sl], acc[sl][hd]);
+    }
+  }
+#pragma unroll
+  for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+    for (int hd = 0; hd < G; ++hd) sacc[hd * 128 + sl * 32 + lane] += acc[sl][hd];
+}
+
+// Zeroes a warp's [G][128] channel sums.
+template <int G>
+__device__ __forceinline__ void zero_sums(float* sacc, int lane) {
+  float4* p = reinterpret_cast<float4*>(sacc);
+#pragma unroll
+  for (int i = lane; i < G * 32; i += 32) p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+}  // namespace
+
+}  // namespace packkv

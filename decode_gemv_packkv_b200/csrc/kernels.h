@@ -57,4 +57,27 @@ size_t pv_workspace_bytes(int batch, int kv_heads, int group);
 // Workspace bytes the launch of `a` by launch_pv would use (n_warps chosen as launch_pv does).
 cudaError_t pv_launch_workspace_bytes(const GemvArgs& a, size_t* bytes);
 
+// Fused decode attention over the packed cache: out = softmax(scale * q·Kᵀ) · V.
+struct AttnArgs {
+  const uint8_t* k_arena;
+  const uint8_t* v_arena;
+  const uint32_t* k_index;  // [batch][kv_heads][max_blocks][2]
+  const uint32_t* v_index;
+  const uint16_t* k_tail;   // [batch][kv_heads][128][128] fp16
+  const uint16_t* v_tail;
+  int batch, kv_heads, group, max_blocks, n_blocks, tail_len, bits;
+  uint64_t arena16;         // arena_bytes / 16
+  uint64_t* ctrl;
+  long n_items;             // batch*kv_heads*items_per_bh
+  int items_per_bh;         // n_blocks + (tail_len > 0)
+  int n_warps;              // logical warps sharing the items
+  const uint16_t* q;        // [batch][q_heads][128]
+  float scale;
+  float* out;               // [batch][q_heads][128]
+  float* partials;          // [n_warps + batch*kv_heads][group][132]: sums [128], max, sum of exp
+};
+
+cudaError_t launch_attention(AttnArgs a, cudaStream_t stream);
+size_t attention_workspace_bytes(int batch, int kv_heads, int group);
+
 }  // namespace packkv

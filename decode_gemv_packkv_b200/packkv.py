@@ -30,7 +30,8 @@ EXPORTED = [
     "packkv_abi_version", "packkv_cache_struct_size", "packkv_status_string", "packkv_record_bytes_max",
     "packkv_workspace_bytes", "packkv_cache_check", "packkv_cache_reset", "packkv_encode_block",
     "packkv_append_token", "packkv_qk_gemv", "packkv_pv_gemv", "packkv_get_status",
-    "packkv_pv_noalloc_scratch_bytes", "packkv_pv_gemv_noalloc",
+    "packkv_pv_noalloc_scratch_bytes", "packkv_pv_gemv_noalloc", "packkv_attention_workspace_bytes",
+    "packkv_attention_decode",
 ]
 
 
@@ -76,6 +77,8 @@ def _load():
         "packkv_get_status": (ctypes.c_int, [P, vp, ctypes.POINTER(u32)]),
         "packkv_pv_noalloc_scratch_bytes": (sz, []),
         "packkv_pv_gemv_noalloc": (ctypes.c_int, [P, vp, i64, i32, vp, vp]),
+        "packkv_attention_workspace_bytes": (sz, [P, i32]),
+        "packkv_attention_decode": (ctypes.c_int, [P, vp, i32, f32, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -174,6 +177,14 @@ class PackKVCache:
             self._ws[q_heads] = torch.zeros(max(n, 16), dtype=torch.uint8, device=self.k_arena.device)
         return self._ws[q_heads]
 
+    def attention_workspace(self, q_heads: int) -> torch.Tensor:
+        """Fused-attention workspace for q_heads (allocated once, reused by every call)."""
+        key = ("attn", q_heads)
+        if key not in self._ws:
+            n = int(_lib.packkv_attention_workspace_bytes(ctypes.byref(self.s), q_heads))
+            self._ws[key] = torch.zeros(max(n, 16), dtype=torch.uint8, device=self.k_arena.device)
+        return self._ws[key]
+
     def arena_used(self):
         """(K bytes, V bytes) in use; synchronises."""
         ends = self.ctrl[:2].cpu()
@@ -236,6 +247,18 @@ def packkv_pv_gemv_noalloc(cache: PackKVCache, p: torch.Tensor, out: torch.Tenso
 
 def packkv_pv_noalloc_scratch_bytes() -> int:
     return int(_lib.packkv_pv_noalloc_scratch_bytes())
+
+
+def packkv_attention_decode(cache: PackKVCache, q: torch.Tensor, scale: float, out: torch.Tensor,
+                            ws: torch.Tensor | None = None, stream=None):
+    """q: fp16 [batch, q_heads, 128]; out: fp32 [batch, q_heads, 128] = softmax(scale q·Kᵀ)·V."""
+    if q.dtype != torch.float16 or q.dim() != 3 or out.dtype != torch.float32:
+        raise ValueError("q must be fp16 [B, Hq, 128], out fp32 [B, Hq, 128]")
+    if ws is None:
+        ws = cache.attention_workspace(q.shape[1])
+    _check("packkv_attention_decode", _lib.packkv_attention_decode(ctypes.byref(cache.s), _ptr(q), q.shape[1],
+                                                                   float(scale), _ptr(out), _ptr(ws), ws.numel(),
+                                                                   _stream(stream)))
 
 
 def packkv_get_status(cache: PackKVCache, stream=None) -> int:

@@ -198,6 +198,26 @@ size_t packkv_pv_noalloc_scratch_bytes(void);
 packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, int64_t ld_p,
                                      int32_t q_heads, float* out, void* stream);
 
+/*
+ * Decode attention over the packed cache in one pass (paper page, Figure 1: the
+ * scores, the softmax and the weighted sum of values; Figure 2: decompression
+ * inside the products):
+ *   out[b][hq][c] = sum_i softmax_i(scale * q[b][hq]·k_hat[b][hq/G][i]) * v_hat[b][hq/G][i][c]
+ * over every packed block and the tail.  The scores and probabilities never
+ * reach global memory; the softmax is computed online (a running maximum and
+ * sum of exponentials per warp), split over the sequence and merged with the
+ * log-sum-exp rule by a second kernel in a fixed order (deterministic).
+ *   q:   device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8}.
+ *   out: device fp32 [batch][q_heads][128].
+ *   ws:  device, ws_bytes >= packkv_attention_workspace_bytes(cache, q_heads)
+ *        (no initialisation needed; two calls sharing ws must not overlap in time).
+ * T == 0 (nothing to attend to) is PACKKV_ERR_INVALID_ARG.  A record with an
+ * invalid index entry sets PACKKV_DEV_BAD_RECORD and its tokens are left out.
+ */
+size_t packkv_attention_workspace_bytes(const packkv_cache* cache, int32_t q_heads);
+packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t* q, int32_t q_heads,
+                                      float scale, float* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, returns PACKKV_OK if no device status bit is set,
  * else PACKKV_ERR_CAPACITY (capacity bit set) or PACKKV_ERR_DEVICE; stores
  * the bits in *bits_out (if not NULL) and clears them. */
