@@ -32,6 +32,11 @@ namespace {
 #define PACKKV_ATTN_WARPS_PER_CTA 2
 #endif
 constexpr int kAttnWarps = PACKKV_ATTN_WARPS_PER_CTA;
+#ifndef PACKKV_ATTN_ONE_STAGE
+#define PACKKV_ATTN_ONE_STAGE 0  // 1: K and V records share one stage (loaded one after the other)
+#endif
+constexpr bool kOneStage = PACKKV_ATTN_ONE_STAGE != 0;
+constexpr int kAttnStages = kOneStage ? 1 : 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSlotFloats = 132;  // per (workspace slot, head): 128 sums, running max, sum of exp, pad
 constexpr float kNegInf = -__builtin_huge_valf();
@@ -46,7 +51,7 @@ struct AttnCfg {
   static constexpr int kTableBytes = ((kI8Tab > kCoreTab ? kI8Tab : kCoreTab) + 15) / 16 * 16;
   static constexpr int kScoreBytes = 512 * G;  // [G][128] scores, then probabilities
   static constexpr int kSumBytes = 512 * G;    // [G][128] channel sums (CUDA-core and tail paths)
-  static constexpr int kFixed = 2 * kStageRec + kTableBytes + kScoreBytes + kSumBytes;
+  static constexpr int kFixed = kAttnStages * kStageRec + kTableBytes + kScoreBytes + kSumBytes;
   static constexpr int kWarpSmem = (kFixed + 32 + 127) / 128 * 128;
   static_assert(kStageRec % 16 == 0 && kFixed % 16 == 0, "stage alignment");
 };
@@ -56,10 +61,10 @@ template <int BITS, int G>
 struct AttnMem {
   using A = AttnCfg<BITS, G>;
   unsigned char* base;
-  __device__ unsigned char* stage(int s) const { return base + s * A::kStageRec; }
-  __device__ uint32_t* table() const { return reinterpret_cast<uint32_t*>(base + 2 * A::kStageRec); }
+  __device__ unsigned char* stage(int s) const { return base + (kOneStage ? 0 : s) * A::kStageRec; }
+  __device__ uint32_t* table() const { return reinterpret_cast<uint32_t*>(base + kAttnStages * A::kStageRec); }
   __device__ float* scores() const {
-    return reinterpret_cast<float*>(base + 2 * A::kStageRec + A::kTableBytes);
+    return reinterpret_cast<float*>(base + kAttnStages * A::kStageRec + A::kTableBytes);
   }
   __device__ float* sums() const { return scores() + 128 * G; }
   __device__ uint64_t* bar(int s) const { return reinterpret_cast<uint64_t*>(base + A::kFixed) + s; }
@@ -218,7 +223,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
   wk.load(ka, lo, hi, lane);
   wv.load(va, lo, hi, lane);
   issue_item<BITS, G, false>(ka, m, cc, wk.get(lo), 0, lane);
-  issue_item<BITS, G, false>(va, m, cc, wv.get(lo), 1, lane);
+  if (!kOneStage) issue_item<BITS, G, false>(va, m, cc, wv.get(lo), 1, lane);
 
   const int q_heads = a.kv_heads * G;
   float qr[G][4];
@@ -265,7 +270,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
     bool ok = mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
     phases ^= 1u;
     if (!ok) {  // the copy never landed (status set): wait, bounded, for the V copy, then stop
-      mbar_wait_bounded(m.bar(1), (phases >> 1) & 1u, a.ctrl);
+      if (!kOneStage) mbar_wait_bounded(m.bar(1), (phases >> 1) & 1u, a.ctrl);
       return;
     }
     const int kind_k = *m.kind(0);
@@ -322,7 +327,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
       }
     }
     __syncwarp();
-    if (x + 1 < hi) {  // the K stage is free: the next item's K record
+    if (kOneStage) {  // the stage is free: this item's V record
+      if (x - wv.base >= 32) wv.load(va, x, hi, lane);
+      issue_item<BITS, G, false>(va, m, cc, wv.get(x), 1, lane);
+    } else if (x + 1 < hi) {  // the K stage is free: the next item's K record
       if (x + 1 - wk.base >= 32) wk.load(ka, x + 1, hi, lane);
       issue_item<BITS, G, false>(ka, m, nc, wk.get(x + 1), 0, lane);
     }
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
     ok = mbar_wait_bounded(m.bar(1), (phases >> 1) & 1u, a.ctrl);
     phases ^= 2u;
     if (!ok) {
-      if (x + 1 < hi) mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
+      if (!kOneStage && x + 1 < hi) mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
       return;
     }
     const int kind_v = *m.kind(1);
@@ -440,9 +448,14 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
       }
     }
     __syncwarp();
-    if (x + 1 < hi) {  // the V stage is free: the next item's V record
-      if (x + 1 - wv.base >= 32) wv.load(va, x + 1, hi, lane);
-      issue_item<BITS, G, false>(va, m, nc, wv.get(x + 1), 1, lane);
+    if (x + 1 < hi) {
+      if (kOneStage) {  // the stage is free: the next item's K record
+        if (x + 1 - wk.base >= 32) wk.load(ka, x + 1, hi, lane);
+        issue_item<BITS, G, false>(ka, m, nc, wk.get(x + 1), 0, lane);
+      } else {  // the V stage is free: the next item's V record
+        if (x + 1 - wv.base >= 32) wv.load(va, x + 1, hi, lane);
+        issue_item<BITS, G, false>(va, m, nc, wv.get(x + 1), 1, lane);
+      }
     }
     cc = nc;
   }
