@@ -243,23 +243,51 @@ def frag_word_bit(bits: int, m: int, k: int):
     raise ValueError("fragment order is defined for b = 2 and b = 4")
 
 
+def frag_plane_bit(m: int, k: int):
+    """(word index within the 1-bit plane, bit offset) of A[m][k]'s high bit in a raw
+    b = 3 record (FORMAT.md section 4): the word is picked by (tile quad T div 4,
+    kappa, kh, lane), the bit by (e, T mod 4, rh)."""
+    T, rh, g = m // 16, (m // 8) % 2, m % 8
+    kappa, kh, t, e = k // 32, (k // 16) % 2, (k % 16) // 4, k % 4
+    lane = 4 * g + t
+    J, Q2 = kappa // 2, kappa % 2
+    return (((T // 4) * 2 + J) * 32 + lane) * 4 + 2 * Q2 + kh, 8 * e + 2 * (T % 4) + rh
+
+
+def frag_fields(bits: int, m: int, k: int):
+    """Where the bits of A[m][k] live in a raw record's word area: a list of
+    (word, bit offset, field width, code bit offset).  b = 2 / 4: one field of b
+    bits.  b = 3: bits 0-1 in the 2-bit plane (words 0 .. 1023, the b = 2 order),
+    bit 2 in the 1-bit plane (words 1024 .. 1535)."""
+    if bits in (2, 4):
+        w, bit = frag_word_bit(bits, m, k)
+        return [(w, bit, bits, 0)]
+    if bits == 3:
+        w0, b0 = frag_word_bit(2, m, k)
+        w1, b1 = frag_plane_bit(m, k)
+        return [(w0, b0, 2, 0), (1024 + w1, b1, 1, 2)]
+    raise ValueError("raw records hold 2, 3 or 4-bit codes")
+
+
 def pack_raw_fragment(a: np.ndarray, bits: int) -> np.ndarray:
-    """Raw word area of a b = 2 / 4 record: every code of the 128x128 matrix A at its place."""
+    """Raw word area of a record: every code of the 128x128 matrix A at its place(s)."""
     words = [0] * (512 * bits)
     for m in range(128):
         for k in range(128):
-            w, bit = frag_word_bit(bits, m, k)
-            words[w] |= int(a[m, k]) << bit
+            code = int(a[m, k])
+            for w, bit, width, shift in frag_fields(bits, m, k):
+                words[w] |= ((code >> shift) & ((1 << width) - 1)) << bit
     return np.array(words, dtype=np.uint64).astype(np.uint32)
 
 
 def unpack_raw_fragment(words: np.ndarray, bits: int) -> np.ndarray:
     a = np.zeros((128, 128), np.int64)
-    mask = (1 << bits) - 1
     for m in range(128):
         for k in range(128):
-            w, bit = frag_word_bit(bits, m, k)
-            a[m, k] = (int(words[w]) >> bit) & mask
+            code = 0
+            for w, bit, width, shift in frag_fields(bits, m, k):
+                code |= ((int(words[w]) >> bit) & ((1 << width) - 1)) << shift
+            a[m, k] = code
     return a
 
 
@@ -290,7 +318,7 @@ def build_record(codes_slot: np.ndarray, mn16: np.ndarray, sc16: np.ndarray,
             offs = codes_slot[32 * g:32 * g + 32, c] - base[g, c]
             words.append(pack_unit(offs, int(width[g, c])))
     all_words = np.concatenate(words).astype(np.uint32) if words else np.zeros(0, np.uint32)
-    if raw and bits in (2, 4):
+    if raw:
         # same header values, word area in tensor-core fragment order (K: rows = slots, V: rows = channels)
         all_words = pack_raw_fragment(codes_slot.T if is_v else codes_slot, bits)
     flags = (RAW_FLAG if raw else 0) | (V_FLAG if is_v else 0) | (FORMAT_VERSION << 8) | (bits << 16)
@@ -343,7 +371,7 @@ def parse_record(rec: bytes) -> ParsedRecord:
         width = meta >> 4
         word_at = 1040
     words = np.frombuffer(rec, dtype="<u4", count=total_words, offset=word_at).astype(np.uint64)
-    if raw and bits in (2, 4):
+    if raw:
         a = unpack_raw_fragment(words, bits)
         codes = a.T.copy() if is_v else a
         return ParsedRecord(raw, is_v, bits, mn, sc, base, width, codes, gws)

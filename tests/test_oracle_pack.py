@@ -183,15 +183,17 @@ def test_raw_fragment_order_hand_words(golden_dir):
         assert int(O.pack_raw_fragment(a, bits)[idx]) == int(want, 16), line
 
 
-@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("bits", [2, 3, 4])
 def test_raw_fragment_order_is_a_bijection(bits):
+    """Every bit of every code has its own place and the word area is filled exactly."""
     seen = set()
     for m in range(128):
         for k in range(128):
-            w, bit = O.frag_word_bit(bits, m, k)
-            assert 0 <= w < 512 * bits and bit % bits == 0 and bit + bits <= 32
-            seen.add((w, bit))
-    assert len(seen) == 128 * 128
+            for w, bit, width, _ in O.frag_fields(bits, m, k):
+                assert 0 <= w < 512 * bits and bit + width <= 32
+                for i in range(width):
+                    seen.add((w, bit + i))
+    assert len(seen) == 128 * 128 * bits
     rng = np.random.default_rng(bits)
     a = rng.integers(0, 1 << bits, (128, 128))
     assert np.array_equal(O.unpack_raw_fragment(O.pack_raw_fragment(a, bits), bits), a)
