@@ -7,9 +7,9 @@
 // over the packed blocks (storage order) and the fp16 tail.  One pass over both
 // arenas: a warp owns a contiguous range of items (blocks, then the tail) of the
 // flat (sequence, kv-head) list, as the q·Kᵀ / p·V kernels do.  Per item it
-// stages the K record and the V record (one single-stage ring each, so that the
-// next K record loads during this item's p·V and the next V record during the
-// next item's q·Kᵀ), computes the item's scores into shared memory with the
+// stages the K record, then the V record in the same shared-memory stage (the V
+// copy is issued as soon as q·Kᵀ has read the K record, the next K copy as soon
+// as p·V has read the V record), computes the item's scores into shared memory with the
 // q·Kᵀ decode paths, updates a running maximum and sum of exponentials per head
 // (online softmax), and adds the probability-weighted values with the p·V decode
 // paths.  At every (sequence, head) boundary it writes its sums, maximum and sum
@@ -29,11 +29,13 @@ namespace packkv {
 namespace {
 
 #ifndef PACKKV_ATTN_WARPS_PER_CTA
-#define PACKKV_ATTN_WARPS_PER_CTA 2
+#define PACKKV_ATTN_WARPS_PER_CTA 4
 #endif
 constexpr int kAttnWarps = PACKKV_ATTN_WARPS_PER_CTA;
 #ifndef PACKKV_ATTN_ONE_STAGE
-#define PACKKV_ATTN_ONE_STAGE 0  // 1: K and V records share one stage (loaded one after the other)
+// 1: an item's K and V records share one stage, loaded one after the other (half the
+// shared memory per warp, twice the resident warps: measured faster than two stages)
+#define PACKKV_ATTN_ONE_STAGE 1
 #endif
 constexpr bool kOneStage = PACKKV_ATTN_ONE_STAGE != 0;
 constexpr int kAttnStages = kOneStage ? 1 : 2;
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
         qv[hd][2] = qr[hd][2] * sc1.x;
         qv[hd][3] = qr[hd][3] * sc1.y;
       }
-      if (kind_k == kKindRaw && !C::kChunked) {
+      if (kind_k == kKindRaw) {
         uint32_t* tab = m.table();
         float invf[G];
         build_i8tab<G, NT>(tab, qv, invf, lane);
@@ -319,11 +321,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
               make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
         }
         __syncwarp();
-        if (kind_k == kKindRaw) {
-          if constexpr (BITS == 3) qk_raw3<G>(st, qp, cst, sc, 128, a.scale, lane);
-        } else {
-          qk_packed<G>(st, qp, cst, sc, 128, a.scale, lane);
-        }
+        qk_packed<G>(st, qp, cst, sc, 128, a.scale, lane);
       }
     }
     __syncwarp();
@@ -411,7 +409,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
           mp[hd] = fmaf(pr[hd][i], mnr[i], mp[hd]);
           pv4[hd][i] = pr[hd][i] * scr[i];
         }
-      if (kind_v == kKindRaw && !C::kChunked) {
+      if (kind_v == kKindRaw) {
         uint32_t* tab = m.table();
         float invf[G];
         build_i8tab<G, NT>(tab, pv4, invf, lane);
@@ -419,32 +417,22 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
         pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
       } else {
         float* pp = reinterpret_cast<float*>(m.table());  // p'' [G][128] then group sums [G][4]
-        const bool raw = kind_v == kKindRaw;
+        // compressed record: p' by storage slot and the per-group sums of p'
 #pragma unroll
         for (int hd = 0; hd < G; ++hd) {
-          float o[4];
           float ps = 0.f;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            ps += pv4[hd][i];
-            const int r15 = (4 * lane + i) & 15;  // field position of slot r in a 2-bit slice word
-            const int sg = r15 <= 10 ? 2 * r15 : 2 * r15 - 12;
-            o[i] = raw ? pv4[hd][i] * exp2i(-sg) : pv4[hd][i];
-          }
-          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-          if (!raw) {
-            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-            if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
-          }
+          for (int i = 0; i < 4; ++i) ps += pv4[hd][i];
+          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) =
+              make_float4(pv4[hd][0], pv4[hd][1], pv4[hd][2], pv4[hd][3]);
+          // lanes 8g .. 8g+7 hold group g
+          ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+          ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+          ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+          if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
         }
         __syncwarp();
-        if (raw) {
-          if constexpr (BITS == 3) pv_raw3<G>(st, pp, sacc, lane);
-        } else {
-          pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
-        }
+        pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
       }
     }
     __syncwarp();

@@ -1,8 +1,7 @@
 // Device building blocks of the fused decode products over the packed cache:
 // record staging (bulk copies into warp-private shared-memory stages, bounded
-// mbarrier waits), the 8-bit integer tensor-core decode of raw 2/4-bit records,
-// and the CUDA-core decode of raw 3-bit and compressed records (FORMAT.md
-// sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused
+// mbarrier waits), the 8-bit integer tensor-core decode of raw records (2, 3 and
+// 4-bit), and the CUDA-core decode of compressed records (FORMAT.md sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused
 // attention kernel.
 #pragma once
 
@@ -23,76 +22,15 @@ constexpr int kWarpsPerCta = PACKKV_WARPS_PER_CTA;
 #define PACKKV_WARP_SMEM_KB 10  // shared memory per warp: one 4-bit stage, five CTAs of 4 warps per SM
 #endif
 constexpr int kWarpSmemBudget = PACKKV_WARP_SMEM_KB * 1024;
-constexpr uint32_t kMagicBits = 0x4B000000u;
-constexpr float kMagic = 8388608.0f;
 constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer in the low bits
 constexpr int kRoundBits = 0x4B400000;
 
 enum ItemKind : int { kKindRaw = 0, kKindPacked = 1, kKindInvalid = 2, kKindTail = 3 };
 
-// (w & mask) | 0x4B000000 in one LOP3: the field lands in the low mantissa bits of 2^23.
-template <uint32_t MASK>
-__device__ __forceinline__ uint32_t fld(uint32_t w) {
-  uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(w), "n"(MASK), "r"(kMagicBits));
-  return d;
-}
-
-// Two magic-number fields -> their exact values, with one packed FP32 add.
-__device__ __forceinline__ float2 pairf(uint32_t a, uint32_t b) {
-  return __fadd2_rn(make_float2(__uint_as_float(a), __uint_as_float(b)), make_float2(-kMagic, -kMagic));
-}
-
-// Field position exponent of token i (0..15) in the 2-bit decode below (value = field * 2^sig2).
-__host__ __device__ constexpr int sig2(int i) { return i <= 10 ? 2 * i : 2 * i - 12; }
-__host__ __device__ constexpr float pow2(int e) {
-  return e >= 0 ? float(1u << e) : 1.0f / float(1u << (-e));
-}
-// 2^e for a run-time e in [-126, 127], from the exponent bits (no division)
-__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
-
-template <int I>
-__device__ __forceinline__ uint32_t fld2(uint32_t w, uint32_t h) {
-  if constexpr (I <= 10)
-    return fld<(3u << (2 * I))>(w);
-  else
-    return fld<(3u << (2 * I - 12))>(h);
-}
-
-// 16 two-bit fields of a 2-bit slice word as 8 pairs: field_i * 2^sig2(i)
-__device__ __forceinline__ void dec2(uint32_t w, float2 (&v)[8]) {
-  const uint32_t h = w >> 12;
-  v[0] = pairf(fld2<0>(w, h), fld2<1>(w, h));
-  v[1] = pairf(fld2<2>(w, h), fld2<3>(w, h));
-  v[2] = pairf(fld2<4>(w, h), fld2<5>(w, h));
-  v[3] = pairf(fld2<6>(w, h), fld2<7>(w, h));
-  v[4] = pairf(fld2<8>(w, h), fld2<9>(w, h));
-  v[5] = pairf(fld2<10>(w, h), fld2<11>(w, h));
-  v[6] = pairf(fld2<12>(w, h), fld2<13>(w, h));
-  v[7] = pairf(fld2<14>(w, h), fld2<15>(w, h));
-}
-
-// 3-bit raw unit, 16 tokens: 2-bit slice word w2 plus the 16 slice-1 bits at bits 0..15 of x.
-// v[p] = (field2 + 4*bit) * 2^sig2, merged with one exact packed FMA per pair.
-__device__ __forceinline__ void dec3(uint32_t w2, uint32_t x, float2 (&v)[8]) {
-  dec2(w2, v);
-#pragma unroll
-  for (int p = 0; p < 8; ++p) {
-    const int i = 2 * p;
-    const float2 b = pairf(x & (1u << i) | kMagicBits, x & (2u << i) | kMagicBits);
-    v[p] = __ffma2_rn(b, make_float2(pow2(sig2(i) - i + 2), pow2(sig2(i + 1) - i + 1)), v[p]);
-  }
-}
-
 template <int BITS, int G, bool PV>
 struct Cfg {
   static constexpr int kRecBytes = raw_record_bytes(BITS);
-  // b = 3 raw records are staged as 16 chunks (group g, channel quarter h: 32 units of
-  // 3 words) at a padded pitch (bank-conflict-free decode); b = 2 / 4 raw records are
-  // in fragment order and are staged in one piece, as are compressed records.
-  static constexpr bool kChunked = BITS == 3;
-  static constexpr int kChunks = 16, kChunkBytes = 384, kPitch = 400;
-  static constexpr int kStageRec = kChunked ? 528 + kChunks * kPitch : kRecBytes;  // >= every record
+  static constexpr int kStageRec = kRecBytes;                  // >= every record, staged in one piece
   static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);              // p·V: + p rows
   // int8 tensor-core B table: columns n = 4*head + digit (digit 3 = 0), NT n-tiles of 8
   static constexpr int kNT = (4 * G + 7) / 8;
@@ -123,9 +61,8 @@ struct WarpMem {
   }
 };
 
-// CUDA-core q' table of q·Kᵀ: (q'_c, q'_c) pairs; channel c = 32*h + cc sits at float2
-// index ((cc/2)*4 + h)*2 + cc%2, so that a 16-byte load gives a lane of the 3-bit
-// decode (chunk h) its next two channels.
+// CUDA-core q' table of q·Kᵀ (compressed records): (q'_c, q'_c) pairs; channel
+// c = 32*h + cc sits at float2 index ((cc/2)*4 + h)*2 + cc%2.
 __device__ __forceinline__ int table_index(int c) {
   const int h = c >> 5, cc = c & 31;
   return ((cc >> 1) * 4 + h) * 2 + (cc & 1);
@@ -149,16 +86,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 16-byte shared-memory load that the compiler issues where it stands (keeps it from
-// hoisting a whole table of loop-invariant loads into registers).
-__device__ __forceinline__ float4 lds_f4(const float* p) {
-  float4 r;
-  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
-               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
-               : "r"(smem_addr(p)));
-  return r;
 }
 
 // Position in the flat item list: (sequence*kv_heads + head, item within it).
@@ -228,11 +155,7 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Curs
       mbar_arrive(m.bar(s));
   }
   __syncwarp();
-  if (kind == kKindRaw && C::kChunked) {
-    if (lane < C::kChunks)
-      bulk_g2s(st + 528 + lane * C::kPitch, src + 528 + lane * C::kChunkBytes, C::kChunkBytes, m.bar(s));
-    if (lane == 16) bulk_g2s(st, src, 528, m.bar(s));
-  } else if (kind == kKindRaw) {
+  if (kind == kKindRaw) {
     if (lane == 16) bulk_g2s(st, src, C::kRecBytes, m.bar(s));
   } else if (kind == kKindPacked) {
     if (lane == 16) bulk_g2s(st, src, len16 * 16u, m.bar(s));
@@ -259,7 +182,7 @@ __device__ void drain_stages(const WarpMem<BITS, G, PV>& m, uint32_t phases, int
 }
 
 // ----------------------------------------------------------------------------
-// 8-bit integer tensor-core decode of raw b = 2 / 4 records (FORMAT.md section 4)
+// 8-bit integer tensor-core decode of raw records (FORMAT.md section 4)
 // ----------------------------------------------------------------------------
 // D(16x8, s32) += A(16x32, u8) * B(32x8, s8): exact integer products and sums.
 __device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -356,16 +279,32 @@ __device__ __forceinline__ void load_i8frags(const uint32_t* tab, uint32_t (&bf)
   }
 }
 
-// Sum of the three digit columns of an accumulator tile (thread (g, t) holds columns
-// 2t, 2t+1 = digits (0, 1) of head 2j + t/2 for even t, digit 2 and the zero column
-// for odd t): returns, in even-t threads, D0 + D1/128 + D2/16384 for rows g (lo) and
-// g + 8 (hi).
-__device__ __forceinline__ void digit_sum(const int (&d)[4], int t, float& lo, float& hi) {
+// Sum of the three digit columns of an accumulator tile, whose columns have already
+// been brought to the same scale (c0, c1: row g, columns 2t, 2t+1; c2, c3: row g + 8).
+// Thread (g, t) holds digits (0, 1) of head 2j + t/2 for even t, digit 2 and the zero
+// column for odd t; returns, in even-t threads, D0 + D1/128 + D2/16384 for rows g (lo)
+// and g + 8 (hi).
+__device__ __forceinline__ void digit_sum(float c0, float c1, float c2, float c3, int t, float& lo, float& hi) {
   const float w0 = (t & 1) ? 1.f / 16384.f : 1.f, w1 = (t & 1) ? 0.f : 1.f / 128.f;
-  lo = fmaf(i2f_small(d[1]), w1, i2f_small(d[0]) * w0);
-  hi = fmaf(i2f_small(d[3]), w1, i2f_small(d[2]) * w0);
+  lo = fmaf(c1, w1, c0 * w0);
+  hi = fmaf(c3, w1, c2 * w0);
   lo += __shfl_down_sync(0xffffffffu, lo, 1);
   hi += __shfl_down_sync(0xffffffffu, hi, 1);
+}
+
+// One accumulator tile whose A fields carried the powers of two 1/ug (row g) and 1/uh
+// (row g + 8): the rows' values, digits joined.
+__device__ __forceinline__ void tile_rows(const int (&d)[4], float ug, float uh, int t, float& lo, float& hi) {
+  digit_sum(i2f_small(d[0]) * ug, i2f_small(d[1]) * ug, i2f_small(d[2]) * uh, i2f_small(d[3]) * uh, t, lo, hi);
+}
+
+// Two accumulator tiles of a 3-bit record: bits 0-1 (dl, scales ul*) and bit 2 (dh,
+// scales uh*, which include the bit's weight 4).
+__device__ __forceinline__ void tile_rows2(const int (&dl)[4], const int (&dh)[4], float ulg, float ulh, float uhg,
+                                           float uhh, int t, float& lo, float& hi) {
+  digit_sum(fmaf(i2f_small(dh[0]), uhg, i2f_small(dl[0]) * ulg), fmaf(i2f_small(dh[1]), uhg, i2f_small(dl[1]) * ulg),
+            fmaf(i2f_small(dh[2]), uhh, i2f_small(dl[2]) * ulh), fmaf(i2f_small(dh[3]), uhh, i2f_small(dl[3]) * ulh),
+            t, lo, hi);
 }
 
 // Selects the value of a run-time head index from a register array.
@@ -399,27 +338,32 @@ __device__ __forceinline__ void afrag2(uint32_t w0, uint32_t w1, uint32_t (&ae)[
   ao[3] = w1 & 0xC0C0C0C0u;
 }
 
-// 1 / (power of two carried by the A fields) of row g (upper = 0) or g + 8 of a tile.
-template <int BITS>
-__host__ __device__ constexpr float row_unscale(int odd_tile, int upper) {
-  return BITS == 4 ? (upper ? 1.f / 16.f : 1.f)
-                   : (odd_tile ? (upper ? 1.f / 64.f : 1.f / 16.f) : (upper ? 0.25f : 1.f));
+// The bit-2 plane of a 3-bit record: tile T's rows g and g + 8 sit at bit 2(T mod 4)
+// and 2(T mod 4) + 1 of every byte; A registers from the plane's two words (kh 0, 1).
+template <int TQ>
+__device__ __forceinline__ void afrag1(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
+  constexpr uint32_t lo = 0x01010101u << (2 * TQ), hi = 0x02020202u << (2 * TQ);
+  a[0] = w0 & lo;
+  a[1] = w0 & hi;
+  a[2] = w1 & lo;
+  a[3] = w1 & hi;
 }
 
-// Runs the tensor-core product of one raw b = 2 / 4 record: for every row tile T
-// (16 rows) calls emit(T, n-tile j, d) with the exact integer tile d.  Rows are
-// slots (q·Kᵀ, K record) or channels (p·V, V record).
+// Runs the tensor-core product of one raw record: for every row tile T (16 rows) and
+// n-tile j calls emit(T, j, lo, hi) with the exact values of rows g (lo) and g + 8
+// (hi) of the thread's columns, digits joined (even-t threads).  Rows are slots
+// (q·Kᵀ, K record) or channels (p·V, V record).
 template <int BITS, int NT, class Emit>
 __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32_t (&bf)[4][NT][2], int lane,
                                            Emit&& emit) {
   const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
-  constexpr int kRows = BITS == 4 ? 8 : 4;  // word rows: tiles (b = 4) or tile pairs (b = 2)
+  const int t = lane & 3;
+  if constexpr (BITS == 4) {
 #pragma unroll
-  for (int tp = 0; tp < kRows; ++tp) {
-    const uint4 wa = words[(tp * 2) * 32 + lane], wb = words[(tp * 2 + 1) * 32 + lane];
-    // k-step kap: words (kh 0, kh 1) = (wa.x, wa.y), (wa.z, wa.w), (wb.x, wb.y), (wb.z, wb.w)
-    const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
-    if constexpr (BITS == 4) {
+    for (int T = 0; T < 8; ++T) {
+      const uint4 wa = words[(T * 2) * 32 + lane], wb = words[(T * 2 + 1) * 32 + lane];
+      // k-step kap: words (kh 0, kh 1) = (wa.x, wa.y), (wa.z, wa.w), (wb.x, wb.y), (wb.z, wb.w)
+      const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
       int d[NT][4];
 #pragma unroll
       for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0;
@@ -431,8 +375,17 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
         for (int j = 0; j < NT; ++j) imma16832(d[j], a, bf[kap][j][0], bf[kap][j][1]);
       }
 #pragma unroll
-      for (int j = 0; j < NT; ++j) emit(tp, j, d[j]);
-    } else {
+      for (int j = 0; j < NT; ++j) {
+        float lo, hi;
+        tile_rows(d[j], 1.f, 1.f / 16.f, t, lo, hi);  // low nibbles x1, high nibbles x16
+        emit(T, j, lo, hi);
+      }
+    }
+  } else if constexpr (BITS == 2) {
+#pragma unroll
+    for (int P = 0; P < 4; ++P) {  // tile pairs
+      const uint4 wa = words[(P * 2) * 32 + lane], wb = words[(P * 2 + 1) * 32 + lane];
+      const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
       int de[NT][4], dd[NT][4];
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
@@ -451,14 +404,64 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
       }
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
-        emit(2 * tp, j, de[j]);
-        emit(2 * tp + 1, j, dd[j]);
+        float lo, hi;
+        tile_rows(de[j], 1.f, 0.25f, t, lo, hi);  // even tile: x1, x4
+        emit(2 * P, j, lo, hi);
+        tile_rows(dd[j], 1.f / 16.f, 1.f / 64.f, t, lo, hi);  // odd tile: x16, x64
+        emit(2 * P + 1, j, lo, hi);
+      }
+    }
+  } else {
+    const uint4* hwords = words + 1024 / 4;  // bit-2 plane
+#pragma unroll
+    for (int Q = 0; Q < 2; ++Q) {  // tile quads of the bit-2 plane
+      const uint4 ha = hwords[(Q * 2) * 32 + lane], hb = hwords[(Q * 2 + 1) * 32 + lane];
+      const uint32_t hw[4][2] = {{ha.x, ha.y}, {ha.z, ha.w}, {hb.x, hb.y}, {hb.z, hb.w}};
+#pragma unroll
+      for (int pp = 0; pp < 2; ++pp) {  // tile pairs 2Q + pp: tiles 4Q + 2pp, 4Q + 2pp + 1
+        const int P = 2 * Q + pp;
+        const uint4 wa = words[(P * 2) * 32 + lane], wb = words[(P * 2 + 1) * 32 + lane];
+        const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
+        int le[NT][4], lo_[NT][4], he[NT][4], ho[NT][4];
+#pragma unroll
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) le[j][i] = lo_[j][i] = he[j][i] = ho[j][i] = 0;
+#pragma unroll
+        for (int kap = 0; kap < 4; ++kap) {
+          uint32_t ae[4], ao[4], be[4], bo[4];
+          afrag2(w[kap][0], w[kap][1], ae, ao);
+          if (pp == 0) {
+            afrag1<0>(hw[kap][0], hw[kap][1], be);
+            afrag1<1>(hw[kap][0], hw[kap][1], bo);
+          } else {
+            afrag1<2>(hw[kap][0], hw[kap][1], be);
+            afrag1<3>(hw[kap][0], hw[kap][1], bo);
+          }
+#pragma unroll
+          for (int j = 0; j < NT; ++j) {
+            imma16832(le[j], ae, bf[kap][j][0], bf[kap][j][1]);
+            imma16832(lo_[j], ao, bf[kap][j][0], bf[kap][j][1]);
+            imma16832(he[j], be, bf[kap][j][0], bf[kap][j][1]);
+            imma16832(ho[j], bo, bf[kap][j][0], bf[kap][j][1]);
+          }
+        }
+        // bit 2 weighs 4; tile 4Q + s (s = 2pp, 2pp+1) carries 2^(2s) (row g), 2^(2s+1) (row g+8)
+        const float e0 = 4.f / float(1 << (4 * pp)), e1 = 4.f / float(1 << (4 * pp + 2));
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          float lo, hi;
+          tile_rows2(le[j], he[j], 1.f, 0.25f, e0, e0 * 0.5f, t, lo, hi);
+          emit(2 * P, j, lo, hi);
+          tile_rows2(lo_[j], ho[j], 1.f / 16.f, 1.f / 64.f, e1, e1 * 0.5f, t, lo, hi);
+          emit(2 * P + 1, j, lo, hi);
+        }
       }
     }
   }
 }
 
-// q·Kᵀ of one raw b = 2 / 4 K record: scores of all 128 slots for the G heads.
+// q·Kᵀ of one raw K record: scores of all 128 slots for the G heads.
 template <int BITS, int G>
 __device__ __forceinline__ void qk_i8(const unsigned char* st, const uint32_t* tab, const float (&cst)[G],
                                       const float (&invf)[G], float* sblk, long ld, float scale, int lane) {
@@ -466,21 +469,19 @@ __device__ __forceinline__ void qk_i8(const unsigned char* st, const uint32_t* t
   const int g = lane >> 2, t = lane & 3;
   uint32_t bf[4][NT][2];
   load_i8frags<NT>(tab, bf, lane);
-  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, const int (&d)[4]) {
-    float lo, hi;
-    digit_sum(d, t, lo, hi);
+  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, float lo, float hi) {
     const int head = 2 * j + (t >> 1);
     if ((t & 1) == 0 && head < G) {
       const float f = head_sel<G>(invf, head), c = head_sel<G>(cst, head);
       float* dst = sblk + head * ld + 16 * T + g;
-      dst[0] = scale * fmaf(lo, f * row_unscale<BITS>(T & 1, 0), c);
-      dst[8] = scale * fmaf(hi, f * row_unscale<BITS>(T & 1, 1), c);
+      dst[0] = scale * fmaf(lo, f, c);
+      dst[8] = scale * fmaf(hi, f, c);
     }
   });
 }
 
-// p·V of one raw b = 2 / 4 V record: adds sum_slots p'*code into the accumulators of
-// channels 16T + g (acc_lo) and 16T + g + 8 (acc_hi) of head 2j + t/2 (even t).
+// p·V of one raw V record: adds sum_slots p'*code into the accumulators of channels
+// 16T + g (acc_lo) and 16T + g + 8 (acc_hi) of head 2j + t/2 (even t).
 template <int BITS, int G>
 __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* tab, const float (&invf)[G],
                                       float (&acc_lo)[(4 * G + 7) / 8][8], float (&acc_hi)[(4 * G + 7) / 8][8],
@@ -492,78 +493,15 @@ __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* t
   float f_t[NT];
 #pragma unroll
   for (int j = 0; j < NT; ++j) f_t[j] = head_sel<G>(invf, 2 * j + (t >> 1));
-  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, const int (&d)[4]) {
-    float lo, hi;
-    digit_sum(d, t, lo, hi);
-    acc_lo[j][T] = fmaf(lo, f_t[j] * row_unscale<BITS>(T & 1, 0), acc_lo[j][T]);
-    acc_hi[j][T] = fmaf(hi, f_t[j] * row_unscale<BITS>(T & 1, 1), acc_hi[j][T]);
+  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, float lo, float hi) {
+    acc_lo[j][T] = fmaf(lo, f_t[j], acc_lo[j][T]);
+    acc_hi[j][T] = fmaf(hi, f_t[j], acc_hi[j][T]);
   });
 }
 
 // ----------------------------------------------------------------------------
-// q·Kᵀ on the CUDA cores
+// q·Kᵀ on the CUDA cores (compressed records)
 // ----------------------------------------------------------------------------
-// One raw b = 3 K record: lane (g, k, h) decodes tokens 32g + 16k .. +15 over the 32
-// channels of chunk 4g + h (a 4-lane reduction over h finishes), heads in chunks of
-// at most four (the words are decoded once per chunk).
-template <int G>
-__device__ __forceinline__ void qk_raw3(const unsigned char* st, const float2* qp, const float (&cst)[G],
-                                        float* sblk, long ld, float scale, int lane) {
-  using C = Cfg<3, G, false>;
-  constexpr int HC = G > 4 ? 4 : G;
-  const int h = lane & 3, k = (lane >> 2) & 1, g = lane >> 3;
-  const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + h) * C::kPitch);
-#pragma unroll 1
-  for (int h0 = 0; h0 < G; h0 += HC) {
-    float2 acc[HC][8];
-#pragma unroll
-    for (int hd = 0; hd < HC; ++hd)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[hd][i] = make_float2(0.f, 0.f);
-#pragma unroll 2
-    for (int c2 = 0; c2 < 16; ++c2) {
-      float2 v0[8], v1[8];
-      dec3(wp[3 * (2 * c2) + k], wp[3 * (2 * c2) + 2] >> (16 * k), v0);
-      dec3(wp[3 * (2 * c2 + 1) + k], wp[3 * (2 * c2 + 1) + 2] >> (16 * k), v1);
-#pragma unroll
-      for (int hd = 0; hd < HC; ++hd) {
-        const float4 qq = *reinterpret_cast<const float4*>(qp + (h0 + hd) * 128 + (c2 * 4 + h) * 2);
-        const float2 q0 = make_float2(qq.x, qq.y), q1 = make_float2(qq.z, qq.w);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          acc[hd][i] = __ffma2_rn(q0, v0[i], acc[hd][i]);
-          acc[hd][i] = __ffma2_rn(q1, v1[i], acc[hd][i]);
-        }
-      }
-    }
-#pragma unroll
-    for (int hd = 0; hd < HC; ++hd) {
-      float tt[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float x = acc[hd][i].x, y = acc[hd][i].y;
-        x += __shfl_xor_sync(0xffffffffu, x, 1);
-        y += __shfl_xor_sync(0xffffffffu, y, 1);
-        x += __shfl_xor_sync(0xffffffffu, x, 2);
-        y += __shfl_xor_sync(0xffffffffu, y, 2);
-        tt[2 * i] = x;
-        tt[2 * i + 1] = y;
-      }
-      float o[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float v = 0.f;
-#pragma unroll
-        for (int hh = 0; hh < 4; ++hh)
-          if (h == hh) v = tt[4 * hh + i] * pow2(-sig2(4 * hh + i));
-        o[i] = scale * (head_sel<G>(cst, h0 + hd) + v);
-      }
-      float* dst = sblk + (h0 + hd) * ld + 32 * g + 16 * k + 4 * h;
-      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
-    }
-  }
-}
-
 // Extracts the offset of token j from a compressed unit of width w starting at word s.
 __device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, int j) {
   uint32_t u = 0;
@@ -650,38 +588,8 @@ __device__ __forceinline__ void qk_tail(const GemvArgs& a, long bh, const float 
 }
 
 // ----------------------------------------------------------------------------
-// p·V on the CUDA cores
+// p·V on the CUDA cores (compressed records)
 // ----------------------------------------------------------------------------
-// One raw b = 3 V record, lane = channel sl*32 + lane; adds into the warp's shared
-// [G][128] channel sums.  The field exponents are folded into p'' = p * scale *
-// 2^-sig (pp: [G][128] by storage slot).
-template <int G>
-__device__ __forceinline__ void pv_raw3(const unsigned char* st, const float* pp, float* sacc, int lane) {
-  using C = Cfg<3, G, true>;
-#pragma unroll 1
-  for (int g = 0; g < 4; ++g) {
-#pragma unroll 1
-    for (int sl = 0; sl < 4; ++sl) {
-      const uint32_t* wp = reinterpret_cast<const uint32_t*>(st + 528 + (4 * g + sl) * C::kPitch + lane * 12);
-      const uint32_t w2 = wp[2];
-      float2 v[2][8];
-      dec3(wp[0], w2, v[0]);        // slots 32g .. 32g+15
-      dec3(wp[1], w2 >> 16, v[1]);  // slots 32g+16 .. 32g+31
-#pragma unroll
-      for (int hd = 0; hd < G; ++hd) {
-        float2 a0 = make_float2(0.f, 0.f), a1 = a0;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 x = lds_f4(pp + hd * 128 + 32 * g + 4 * q);
-          a0 = __ffma2_rn(make_float2(x.x, x.y), v[q >> 2][2 * (q & 3)], a0);
-          a1 = __ffma2_rn(make_float2(x.z, x.w), v[q >> 2][2 * (q & 3) + 1], a1);
-        }
-        sacc[hd * 128 + sl * 32 + lane] += (a0.x + a0.y) + (a1.x + a1.y);
-      }
-    }
-  }
-}
-
 // One compressed V record, lane = channel sl*32 + lane; adds into the warp's shared
 // [G][128] channel sums.  pg[hd*4 + g] = sum of p' over pack group g.
 template <int G>

@@ -34,6 +34,12 @@ namespace {
 constexpr uint32_t kFlagAggregate = 0x80000000u;  // {x = own length16, y = flag}: prefix not known yet
 constexpr uint32_t kDone2 = 2u;                   // done counter step (bit 0: some record did not fit)
 constexpr int kEncodeThreads = 512;
+// storage-order code copies inside the (then unused) input buffers: above the first
+// 12 KiB, which hold the record being assembled (at most 528 + 2048*4 bytes)
+constexpr int kCodeCopyOffset = 12 * 1024;
+constexpr int kVtPitch = 132;  // bytes per channel row of the transposed V codes (spreads banks)
+static_assert(kCodeCopyOffset >= 528 + 2048 * 4, "records fit below the code copies");
+static_assert(kCodeCopyOffset + 128 * kVtPitch <= 128 * 128 * 2, "code copies fit in an input buffer");
 constexpr int kParts = kEncodeThreads / kBlockTokens;  // threads per channel / token in the reductions
 
 struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
@@ -281,6 +287,23 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
   }
   __syncthreads();
 
+  // ---- codes in storage order, for the fragment words of raw records ----------
+  // K: kp[slot][channel] (row copies); V: vt[channel][slot] (transposed, pitch 132).
+  // Both live in the input buffers, which the codes no longer need, above the part
+  // that later holds the records.
+  uint8_t* kp = reinterpret_cast<uint8_t*>(&s.kx[0][0]) + kCodeCopyOffset;
+  uint8_t* vt = reinterpret_cast<uint8_t*>(&s.vx[0][0]) + kCodeCopyOffset;
+  for (int i = tid; i < kBlockTokens * kHeadDim / 16; i += blockDim.x) {
+    const int r = i >> 3, q = i & 7;
+    reinterpret_cast<uint4*>(kp + r * kHeadDim)[q] = reinterpret_cast<const uint4*>(s.ck[s.perm[r]])[q];
+  }
+  for (int i = tid; i < kHeadDim * kBlockTokens / 4; i += blockDim.x) {
+    const int c = i & (kHeadDim - 1), r4 = (i >> 7) * 4;  // lanes take consecutive channels
+    const uint32_t w = (uint32_t)s.cv[s.perm[r4]][c] | ((uint32_t)s.cv[s.perm[r4 + 1]][c] << 8) |
+                       ((uint32_t)s.cv[s.perm[r4 + 2]][c] << 16) | ((uint32_t)s.cv[s.perm[r4 + 3]][c] << 24);
+    *reinterpret_cast<uint32_t*>(vt + c * kVtPitch + r4) = w;
+  }
+
   // ---- frame of reference and width of every (group, channel) unit ----------
   for (int u = tid; u < 2 * kGroups * kHeadDim; u += blockDim.x) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
@@ -385,38 +408,45 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
       }
     }
   }
-  // raw records of b = 2 / 4: words in 8-bit tensor-core fragment order (FORMAT.md section 4).
-  // A[m][k] = code of slot m, channel k (K) or of slot k, channel m (V).
-  if (a.bits != 3) {
+  // raw records: words in 8-bit tensor-core fragment order (FORMAT.md section 4).
+  // A[m][k] = code of slot m, channel k (K: kp row m) or of slot k, channel m (V: vt row
+  // m).  A word's byte e holds column k0 + e of rows (16T + 8rh + g): one 32-bit load
+  // of a storage-order row gives the four codes of a (row, byte) field set, placed by
+  // one shift.  b = 3: bits 0-1 in words 0..1023 (the b = 2 order), bit 2 in 1024..1535.
 #pragma unroll
-    for (int tensor = 0; tensor < 2; ++tensor) {
-      if (!raw[tensor]) continue;
-      uint32_t* words = rec32[tensor] + kRawWordOffset / 4;
-      for (int wi = tid; wi < 512 * a.bits; wi += blockDim.x) {
-        // wi = ((tile row or tile pair)*2 + J)*32 + lane)*4 + 2*Q2 + kh, kappa = 2J + Q2
-        const int kh = wi & 1, q2 = (wi >> 1) & 1, lane = (wi >> 2) & 31, jj = (wi >> 7) & 1, tp = wi >> 8;
-        const int kappa = 2 * jj + q2, g = lane >> 2, t = lane & 3;
-        uint32_t word = 0;
-        const int nfields = 32 / a.bits;
-        for (int f = 0; f < nfields; ++f) {
-          int e, rh, tile;
-          if (a.bits == 4) {
-            e = f >> 1, rh = f & 1, tile = tp;
-          } else {
-            e = f >> 2, rh = f & 1, tile = 2 * tp + ((f >> 1) & 1);
-          }
-          const int m = 16 * tile + 8 * rh + g, k = 32 * kappa + 16 * kh + 4 * t + e;
-          const uint32_t code = tensor ? s.cv[s.perm[k]][m] : s.ck[s.perm[m]][k];
-          word |= code << (a.bits * f);
-        }
-        words[wi] = word;
+  for (int tensor = 0; tensor < 2; ++tensor) {
+    if (!raw[tensor]) continue;
+    uint32_t* words = rec32[tensor] + kRawWordOffset / 4;
+    const uint8_t* rows = tensor ? vt : kp;
+    const int pitch = tensor ? kVtPitch : kHeadDim;
+    for (int wi = tid; wi < 512 * a.bits; wi += blockDim.x) {
+      const bool plane1 = a.bits == 3 && wi >= 1024;
+      const int wj = plane1 ? wi - 1024 : wi;
+      // wj = ((row group)*2 + J)*32 + lane)*4 + 2*Q2 + kh, kappa = 2J + Q2; the row group is
+      // the tile (b = 4), the tile pair (b = 2, low plane of b = 3) or the tile quad (bit-2 plane)
+      const int kh = wj & 1, q2 = (wj >> 1) & 1, lane = (wj >> 2) & 31, jj = (wj >> 7) & 1, tp = wj >> 8;
+      const int g = lane >> 2, t = lane & 3;
+      const uint8_t* col = rows + 32 * (2 * jj + q2) + 16 * kh + 4 * t + g * pitch;
+      auto row4 = [&](int m8) { return *reinterpret_cast<const uint32_t*>(col + m8 * 8 * pitch); };  // row 8*m8 + g
+      uint32_t word;
+      if (a.bits == 4) {
+        word = row4(2 * tp) | (row4(2 * tp + 1) << 4);  // rows 16T + g, 16T + 8 + g
+      } else if (!plane1) {
+        const uint32_t m3 = a.bits == 3 ? 0x03030303u : 0xFFFFFFFFu;
+        word = (row4(4 * tp) & m3) | ((row4(4 * tp + 1) & m3) << 2) | ((row4(4 * tp + 2) & m3) << 4) |
+               ((row4(4 * tp + 3) & m3) << 6);
+      } else {
+        word = 0u;
+#pragma unroll
+        for (int sg = 0; sg < 8; ++sg) word |= ((row4(8 * tp + sg) >> 2) & 0x01010101u) << sg;
       }
+      words[wi] = word;
     }
   }
   // pack the units: every word is owned by exactly one thread
   for (int u = tid; u < 2 * kGroups * kHeadDim; u += blockDim.x) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
-    if (raw[tensor] && a.bits != 3) continue;  // written above
+    if (raw[tensor]) continue;  // written above
     const uint8_t(*cx)[kHeadDim] = tensor ? s.cv : s.ck;
     const int w = raw[tensor] ? a.bits : s.width[tensor][g][c];
     const int base = raw[tensor] ? 0 : s.base[tensor][g][c];

@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
         qv[hd][3] = qr[hd][3] * sc1.y;
       }
       float* sblk = srow0 + (long)j * 128;
-      if (kind == kKindRaw && !C::kChunked) {
+      if (kind == kKindRaw) {
         uint32_t* tab = m.table();
         float invf[G];
         build_i8tab<G, C::kNT>(tab, qv, invf, lane);
@@ -145,11 +145,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
               make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
         }
         __syncwarp();
-        if (kind == kKindRaw) {
-          if constexpr (BITS == 3) qk_raw3<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
-        } else {
-          qk_packed<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
-        }
+        qk_packed<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
       }
     }
     __syncwarp();
@@ -343,40 +339,29 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
           pv4[hd][i] = pr[i] * scr[i];
         }
       }
-      if (kind == kKindRaw && !C::kChunked) {
+      if (kind == kKindRaw) {
         uint32_t* tab = m.table();
         float invf[G];
         build_i8tab<G, C::kNT>(tab, pv4, invf, lane);
         __syncwarp();
         pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
       } else {
-        const bool raw = kind == kKindRaw;
+        // compressed record: p' by storage slot and the per-group sums of p'
 #pragma unroll
         for (int hd = 0; hd < G; ++hd) {
-          float o[4];
           float ps = 0.f;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            ps += pv4[hd][i];
-            const int r15 = (4 * lane + i) & 15;  // field position of slot r in a 2-bit slice word
-            const int sg = r15 <= 10 ? 2 * r15 : 2 * r15 - 12;
-            o[i] = raw ? pv4[hd][i] * exp2i(-sg) : pv4[hd][i];  // exact power-of-two scaling
-          }
-          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
-          if (!raw) {
-            // per-group sum of p' (lanes 8g..8g+7 hold group g)
-            ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-            ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-            if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
-          }
+          for (int i = 0; i < 4; ++i) ps += pv4[hd][i];
+          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) =
+              make_float4(pv4[hd][0], pv4[hd][1], pv4[hd][2], pv4[hd][3]);
+          // lanes 8g .. 8g+7 hold group g
+          ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+          ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+          ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+          if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
         }
         __syncwarp();
-        if (raw) {
-          if constexpr (BITS == 3) pv_raw3<G>(st, pp, sacc, lane);
-        } else {
-          pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
-        }
+        pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
       }
     }
     __syncwarp();
