@@ -47,9 +47,9 @@ template <int BITS, int G>
 struct AttnCfg {
   using C = Cfg<BITS, G, false>;
   static constexpr int kStageRec = C::kStageRec;  // one K or one V record
-  static constexpr int kNT = (4 * G + 7) / 8;
-  static constexpr int kI8Tab = 4 * (64 * kNT + 8) * 4;
-  static constexpr int kCoreTab = 1024 * G;  // q' pairs [G][128]; p'' [G][128] + group sums [G][4] fit too
+  static constexpr int kNT = C::kNT;
+  static constexpr int kI8Tab = C::kI8Tab;
+  static constexpr int kCoreTab = 528 * G;  // q' [G][128]; p'' [G][128] + group sums [G][4]
   static constexpr int kTableBytes = ((kI8Tab > kCoreTab ? kI8Tab : kCoreTab) + 15) / 16 * 16;
   static constexpr int kScoreBytes = 512 * G;  // [G][128] scores, then probabilities
   static constexpr int kSumBytes = 512 * G;    // [G][128] channel sums (CUDA-core and tail paths)
@@ -157,18 +157,18 @@ __device__ __forceinline__ void tail_values(const AttnArgs& a, long bh, const fl
 // together), the running maximum and the running sum of exponentials.
 template <int G>
 __device__ __forceinline__ void attn_flush(const AttnArgs& a, long bh, int warp, float* sacc,
-                                           float (&acc_lo)[(4 * G + 7) / 8][8],
-                                           float (&acc_hi)[(4 * G + 7) / 8][8], float (&mp)[G], float (&mrun)[G],
+                                           float (&acc_lo)[I8Layout<G>::kNH][8],
+                                           float (&acc_hi)[I8Layout<G>::kNH][8], float (&mp)[G], float (&mrun)[G],
                                            float (&lrun)[G], int lane) {
-  constexpr int NT = (4 * G + 7) / 8;
+  using L = I8Layout<G>;
   const int g = lane >> 2, t = lane & 3;
   __syncwarp();
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int head = 2 * j + (t >> 1);
+  for (int j = 0; j < L::kNH; ++j) {
+    const int head = L::head(j, t);
 #pragma unroll
     for (int T = 0; T < 8; ++T) {
-      if ((t & 1) == 0 && head < G) {
+      if (L::owns(j, t)) {
         sacc[head * 128 + 16 * T + g] += acc_lo[j][T];
         sacc[head * 128 + 16 * T + g + 8] += acc_hi[j][T];
       }
@@ -204,6 +204,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
   using A = AttnCfg<BITS, G>;
   using C = Cfg<BITS, G, false>;
   constexpr int NT = A::kNT;
+  constexpr int NH = C::kNH;
   extern __shared__ __align__(128) unsigned char smem[];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
   const int q_heads = a.kv_heads * G;
   float qr[G][4];
   float mrun[G], lrun[G], mp[G];
-  float acc_lo[NT][8], acc_hi[NT][8];
+  float acc_lo[NH][8], acc_hi[NH][8];
 #pragma unroll
   for (int hd = 0; hd < G; ++hd) {
     mrun[hd] = kNegInf;
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
     mp[hd] = 0.f;
   }
 #pragma unroll
-  for (int jn = 0; jn < NT; ++jn)
+  for (int jn = 0; jn < NH; ++jn)
 #pragma unroll
     for (int T = 0; T < 8; ++T) acc_lo[jn][T] = acc_hi[jn][T] = 0.f;
   float* sacc = m.sums();
@@ -312,14 +313,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
         __syncwarp();
         qk_i8<BITS, G>(st, tab, cst, invf, sc, 128, a.scale, lane);
       } else {
-        float2* qp = reinterpret_cast<float2*>(m.table());
+        float* qp = reinterpret_cast<float*>(m.table());
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane)) =
-              make_float4(qv[hd][0], qv[hd][0], qv[hd][1], qv[hd][1]);
-          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane + 2)) =
-              make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
-        }
+        for (int hd = 0; hd < G; ++hd)
+          *reinterpret_cast<float4*>(qp + hd * 128 + 4 * lane) = make_float4(qv[hd][0], qv[hd][1], qv[hd][2], qv[hd][3]);
         __syncwarp();
         qk_packed<G>(st, qp, cst, sc, 128, a.scale, lane);
       }
@@ -361,8 +358,8 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl) sacc[hd * 128 + sl * 32 + lane] *= alpha;
 #pragma unroll
-        for (int jn = 0; jn < NT; ++jn) {
-          if (2 * jn + (t >> 1) == hd) {
+        for (int jn = 0; jn < NH; ++jn) {
+          if (I8Layout<G>::head(jn, t) == hd) {
 #pragma unroll
             for (int T = 0; T < 8; ++T) {
               acc_lo[jn][T] *= alpha;

@@ -27,21 +27,51 @@ constexpr int kRoundBits = 0x4B400000;
 
 enum ItemKind : int { kKindRaw = 0, kKindPacked = 1, kKindInvalid = 2, kKindTail = 3 };
 
+// Columns of the int8 tensor-core B table (q' or p' as three base-128 digits per head)
+// and which accumulator values a thread ends with.  A thread (g, t) of an m16n8
+// accumulator tile holds columns 2t and 2t + 1.
+//  * Paired (G <= 2): n-tile j holds heads 2j, 2j + 1 as columns 4*(head - 2j) + digit
+//    (digit 3 zero).  Thread t has digits 0, 1 (even t) or 2 (odd t) of head 2j + t/2;
+//    one shuffle joins them into the even-t thread.
+//  * Split (G >= 4, a multiple of 4): n-tiles 2i and 2i + 1 hold heads 4i .. 4i + 3:
+//    column 2u + d of n-tile 2i is digit d < 2 of head 4i + u, column 2u of n-tile
+//    2i + 1 its digit 2 (column 2u + 1 zero).  Thread t has all three digits of head
+//    4i + t, so every thread ends with one head's rows and no shuffle is needed.
+// kNH accumulator sets per thread, index jh: head(jh, t), owned where owns(jh, t).
+#ifndef PACKKV_SPLIT_MIN_G
+#define PACKKV_SPLIT_MIN_G 4
+#endif
+template <int G>
+struct I8Layout {
+  static constexpr bool kSplit = G >= PACKKV_SPLIT_MIN_G;
+  static_assert(!kSplit || G % 4 == 0, "split layout takes whole head quads");
+  static constexpr int kNT = kSplit ? G / 2 : (4 * G + 7) / 8;
+  static constexpr int kNH = kSplit ? G / 4 : kNT;
+  __device__ static int head(int jh, int t) { return kSplit ? 4 * jh + t : 2 * jh + (t >> 1); }
+  __device__ static bool owns(int jh, int t) { return kSplit || ((t & 1) == 0 && 2 * jh + (t >> 1) < G); }
+  // n (column over all n-tiles) of digit d of head h
+  __host__ __device__ static constexpr int column(int h, int d) {
+    return kSplit ? 16 * (h >> 2) + 2 * (h & 3) + (d & 1) + 8 * (d >> 1) : 4 * h + d;
+  }
+};
+
 template <int BITS, int G, bool PV>
 struct Cfg {
   static constexpr int kRecBytes = raw_record_bytes(BITS);
   static constexpr int kStageRec = kRecBytes;                  // >= every record, staged in one piece
-  static constexpr int kStageBytes = kStageRec + (PV ? 512 * G : 0);              // p·V: + p rows
+  static constexpr int kStageBytes = kStageRec;
   // int8 tensor-core B table: columns n = 4*head + digit (digit 3 = 0), NT n-tiles of 8
-  static constexpr int kNT = (4 * G + 7) / 8;
+  static constexpr int kNT = I8Layout<G>::kNT;
+  static constexpr int kNH = I8Layout<G>::kNH;
   static constexpr int kI8Tab = 4 * (64 * kNT + 8) * 4;
-  // CUDA-core tables: q' pairs [G][128] (q·Kᵀ); p'' [G][128] + group sums of p' [G][4] (p·V)
-  static constexpr int kCoreTab = PV ? 512 * G + 16 * G : 1024 * G;
+  // CUDA-core tables: q' [G][128] (q·Kᵀ); p'' [G][128] + group sums of p' [G][4] (p·V)
+  static constexpr int kCoreTab = PV ? 512 * G + 16 * G : 512 * G;
   static constexpr int kTableBytes = ((kCoreTab > kI8Tab ? kCoreTab : kI8Tab) + 15) / 16 * 16;
   static constexpr int kSumBytes = PV ? 512 * G : 0;          // p·V: [G][128] channel sums
   static constexpr int kFixed = kTableBytes + kSumBytes;
   static constexpr int kStages0 = (kWarpSmemBudget - kFixed - 64) / kStageBytes;
-  static constexpr int kStages = kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0);
+  // p·V keeps the p of its in-flight record in registers, one record deep: one stage
+  static constexpr int kStages = PV ? 1 : (kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0));
   static constexpr int kWarpSmem = ((kStages * kStageBytes + kFixed + kStages * 16) + 127) / 128 * 128;
   static_assert(kStageBytes % 16 == 0 && kFixed % 16 == 0, "stage alignment");
 };
@@ -60,13 +90,6 @@ struct WarpMem {
     return reinterpret_cast<int*>(fixed() + C::kFixed + C::kStages * 8) + s;
   }
 };
-
-// CUDA-core q' table of q·Kᵀ (compressed records): (q'_c, q'_c) pairs; channel
-// c = 32*h + cc sits at float2 index ((cc/2)*4 + h)*2 + cc%2.
-__device__ __forceinline__ int table_index(int c) {
-  const int h = c >> 5, cc = c & 31;
-  return ((cc >> 1) * 4 + h) * 2 + (cc & 1);
-}
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
@@ -128,7 +151,6 @@ struct EntryWindow {
 template <int BITS, int G, bool PV, class Mem>
 __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Cursor c, uint2 e, int s, int lane) {
   using C = Cfg<BITS, G, PV>;
-  const long bh = c.bh;
   const int j = c.j;
   int kind = kKindTail;
   uint64_t off16 = 0;
@@ -147,7 +169,6 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Curs
     uint32_t bytes = 0;
     if (kind == kKindRaw) bytes = C::kRecBytes;
     if (kind == kKindPacked) bytes = len16 * 16u;
-    if (PV && bytes) bytes += 512u * G;
     fence_async_smem();
     if (bytes)
       mbar_arrive_expect_tx(m.bar(s), bytes);
@@ -159,13 +180,6 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Curs
     if (lane == 16) bulk_g2s(st, src, C::kRecBytes, m.bar(s));
   } else if (kind == kKindPacked) {
     if (lane == 16) bulk_g2s(st, src, len16 * 16u, m.bar(s));
-  }
-  if (PV && (kind == kKindRaw || kind == kKindPacked) && lane >= 24 && lane < 24 + G) {
-    const int hd = lane - 24;
-    const long b = bh / a.kv_heads, h = bh % a.kv_heads;
-    const long hq = h * G + hd;
-    const float* prow = a.p + ((size_t)b * a.kv_heads * G + hq) * a.ld + (size_t)j * 128;
-    bulk_g2s(st + C::kStageRec + hd * 512, prow, 512, m.bar(s));
   }
 }
 
@@ -214,16 +228,19 @@ __device__ __forceinline__ int i8tab_word(int kap, int kh, int t, int n) {
 // B table of the int8 products for one record: lane holds x[head][i] for k = 4*lane + i
 // (channel for q·Kᵀ, storage slot for p·V).  Per head f = 127 / max|x| and
 // y = x*f = d0 + d1/128 + d2/16384 with integer digits |d0| <= 127, |d1|, |d2| <= 64
-// (each the rounding of the remainder so far, so |y - sum| <= 2^-15); column
-// 4*head + i holds digit i (column 4*head + 3 and the columns of absent heads are
-// zero).  Returns 1/f per head.
+// (each the rounding of the remainder so far, so |y - sum| <= 2^-15); digit i goes to
+// column I8Layout<G>::column(head, i), digit 3 and absent heads are zero.  Returns
+// 1/f per head.
 template <int G, int NT>
 __device__ __forceinline__ void build_i8tab(uint32_t* tab, const float (&x)[G][4], float (&invf)[G], int lane) {
+  using L = I8Layout<G>;
+  static_assert(NT == L::kNT, "n-tiles of the layout");
+  constexpr int kHeads = L::kSplit ? G : 2 * NT;  // heads with columns (absent ones zero)
   const int kap = lane >> 3, kh = (lane >> 2) & 1, t = lane & 3;
   const float2 R = make_float2(kRound, kRound), nR = make_float2(-kRound, -kRound);
   const float2 k128 = make_float2(128.f, 128.f);
 #pragma unroll
-  for (int hd = 0; hd < 2 * NT; ++hd) {
+  for (int hd = 0; hd < kHeads; ++hd) {
     uint32_t w0 = 0u, w1 = 0u, w2 = 0u;
     if (hd < G) {
       const int h = hd < G ? hd : 0;
@@ -247,10 +264,10 @@ __device__ __forceinline__ void build_i8tab(uint32_t* tab, const float (&x)[G][4
       w1 = pack4(t1[0], t1[1]);
       w2 = pack4(t2[0], t2[1]);
     }
-    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 0)] = w0;
-    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 1)] = w1;
-    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 2)] = w2;
-    tab[i8tab_word<NT>(kap, kh, t, 4 * hd + 3)] = 0u;
+    tab[i8tab_word<NT>(kap, kh, t, L::column(hd, 0))] = w0;
+    tab[i8tab_word<NT>(kap, kh, t, L::column(hd, 1))] = w1;
+    tab[i8tab_word<NT>(kap, kh, t, L::column(hd, 2))] = w2;
+    tab[i8tab_word<NT>(kap, kh, t, L::column(hd, 3))] = 0u;
   }
 }
 
@@ -279,32 +296,85 @@ __device__ __forceinline__ void load_i8frags(const uint32_t* tab, uint32_t (&bf)
   }
 }
 
-// Sum of the three digit columns of an accumulator tile, whose columns have already
-// been brought to the same scale (c0, c1: row g, columns 2t, 2t+1; c2, c3: row g + 8).
-// Thread (g, t) holds digits (0, 1) of head 2j + t/2 for even t, digit 2 and the zero
-// column for odd t; returns, in even-t threads, D0 + D1/128 + D2/16384 for rows g (lo)
-// and g + 8 (hi).
-__device__ __forceinline__ void digit_sum(float c0, float c1, float c2, float c3, int t, float& lo, float& hi) {
+// Accumulators start at the bit pattern of 1.5*2^23 (kRoundBits): an accumulated
+// integer D (|D| < 2^22) then reads as the float 1.5*2^23 + D, and
+// fmaf(that, w, -w*1.5*2^23) is w*D exactly for a power of two w; further weighted
+// digits are chained on with one rounding each.
+
+// Digit weights of a paired-layout thread: even t holds digits 0, 1 (1, 2^-7), odd t
+// digit 2 and the zero column (2^-14, 0); c = -(w0 + w1) * 1.5*2^23 (exact).
+struct PairW {
+  float w0, w1, c;
+};
+__device__ __forceinline__ PairW pair_weights(int t) {
   const float w0 = (t & 1) ? 1.f / 16384.f : 1.f, w1 = (t & 1) ? 0.f : 1.f / 128.f;
-  lo = fmaf(c1, w1, c0 * w0);
-  hi = fmaf(c3, w1, c2 * w0);
-  lo += __shfl_down_sync(0xffffffffu, lo, 1);
-  hi += __shfl_down_sync(0xffffffffu, hi, 1);
+  return {w0, w1, -(w0 + w1) * kRound};
 }
 
-// One accumulator tile whose A fields carried the powers of two 1/ug (row g) and 1/uh
-// (row g + 8): the rows' values, digits joined.
-__device__ __forceinline__ void tile_rows(const int (&d)[4], float ug, float uh, int t, float& lo, float& hi) {
-  digit_sum(i2f_small(d[0]) * ug, i2f_small(d[1]) * ug, i2f_small(d[2]) * uh, i2f_small(d[3]) * uh, t, lo, hi);
+// One row of a paired-layout tile (accumulators x0, x1 of columns 2t, 2t + 1): this
+// thread's digit terms, before the shuffle join and the row weight.
+__device__ __forceinline__ float pair_row(int x0, int x1, const PairW& w) {
+  return fmaf(__int_as_float(x1), w.w1, fmaf(__int_as_float(x0), w.w0, w.c));
 }
 
-// Two accumulator tiles of a 3-bit record: bits 0-1 (dl, scales ul*) and bit 2 (dh,
-// scales uh*, which include the bit's weight 4).
-__device__ __forceinline__ void tile_rows2(const int (&dl)[4], const int (&dh)[4], float ulg, float ulh, float uhg,
-                                           float uhh, int t, float& lo, float& hi) {
-  digit_sum(fmaf(i2f_small(dh[0]), uhg, i2f_small(dl[0]) * ulg), fmaf(i2f_small(dh[1]), uhg, i2f_small(dl[1]) * ulg),
-            fmaf(i2f_small(dh[2]), uhh, i2f_small(dl[2]) * ulh), fmaf(i2f_small(dh[3]), uhh, i2f_small(dl[3]) * ulh),
-            t, lo, hi);
+// One row of a split-layout head: digits 0, 1 (x0, x1 of n-tile 2i) and 2 (x2 of
+// n-tile 2i + 1) joined, times the row weight u (a power of two).  The first product
+// cancels all three offsets, so the running value stays below 2^23 * u.
+__device__ __forceinline__ float split_row(int x0, int x1, int x2, float u) {
+  constexpr float c = -kRound * (1.f + 1.f / 128.f + 1.f / 16384.f);  // exact: 16 significant bits
+  const float v = fmaf(__int_as_float(x0), u, c * u);
+  return fmaf(__int_as_float(x2), u * (1.f / 16384.f), fmaf(__int_as_float(x1), u * (1.f / 128.f), v));
+}
+
+// The rows of row tile T for every accumulator set jh: emit(T, jh, lo, hi) with the
+// values of rows g (lo) and g + 8 (hi), digits joined, valid where
+// I8Layout<G>::owns(jh, t).  d: the tile's accumulators over all n-tiles, whose A
+// fields carried the powers of two 1/ug (row g) and 1/uh (row g + 8).
+template <int G, class Emit>
+__device__ __forceinline__ void emit_tile(int T, const int (&d)[I8Layout<G>::kNT][4], float ug, float uh,
+                                          const PairW& w, Emit& emit) {
+  using L = I8Layout<G>;
+  if constexpr (L::kSplit) {
+#pragma unroll
+    for (int jh = 0; jh < L::kNH; ++jh)
+      emit(T, jh, split_row(d[2 * jh][0], d[2 * jh][1], d[2 * jh + 1][0], ug),
+           split_row(d[2 * jh][2], d[2 * jh][3], d[2 * jh + 1][2], uh));
+  } else {
+#pragma unroll
+    for (int j = 0; j < L::kNT; ++j) {
+      float lo = pair_row(d[j][0], d[j][1], w), hi = pair_row(d[j][2], d[j][3], w);
+      lo += __shfl_down_sync(0xffffffffu, lo, 1);
+      hi += __shfl_down_sync(0xffffffffu, hi, 1);
+      emit(T, j, lo * ug, hi * uh);
+    }
+  }
+}
+
+// As emit_tile for a 3-bit record's two planes: bits 0-1 (dl, row weights ulg, ulh) and
+// bit 2 (dh, row weights uhg, uhh, which include the bit's weight 4).
+template <int G, class Emit>
+__device__ __forceinline__ void emit_tile2(int T, const int (&dl)[I8Layout<G>::kNT][4],
+                                           const int (&dh)[I8Layout<G>::kNT][4], float ulg, float ulh, float uhg,
+                                           float uhh, const PairW& w, Emit& emit) {
+  using L = I8Layout<G>;
+  if constexpr (L::kSplit) {
+#pragma unroll
+    for (int jh = 0; jh < L::kNH; ++jh) {
+      const int a = 2 * jh, b = 2 * jh + 1;
+      emit(T, jh,
+           split_row(dl[a][0], dl[a][1], dl[b][0], ulg) + split_row(dh[a][0], dh[a][1], dh[b][0], uhg),
+           split_row(dl[a][2], dl[a][3], dl[b][2], ulh) + split_row(dh[a][2], dh[a][3], dh[b][2], uhh));
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < L::kNT; ++j) {
+      float lo = fmaf(pair_row(dh[j][0], dh[j][1], w), uhg / ulg, pair_row(dl[j][0], dl[j][1], w));
+      float hi = fmaf(pair_row(dh[j][2], dh[j][3], w), uhh / ulh, pair_row(dl[j][2], dl[j][3], w));
+      lo += __shfl_down_sync(0xffffffffu, lo, 1);
+      hi += __shfl_down_sync(0xffffffffu, hi, 1);
+      emit(T, j, lo * ulg, hi * ulh);
+    }
+  }
 }
 
 // Selects the value of a run-time head index from a register array.
@@ -350,14 +420,15 @@ __device__ __forceinline__ void afrag1(uint32_t w0, uint32_t w1, uint32_t (&a)[4
 }
 
 // Runs the tensor-core product of one raw record: for every row tile T (16 rows) and
-// n-tile j calls emit(T, j, lo, hi) with the exact values of rows g (lo) and g + 8
-// (hi) of the thread's columns, digits joined (even-t threads).  Rows are slots
-// (q·Kᵀ, K record) or channels (p·V, V record).
-template <int BITS, int NT, class Emit>
-__device__ __forceinline__ void i8_product(const unsigned char* st, const uint32_t (&bf)[4][NT][2], int lane,
-                                           Emit&& emit) {
+// accumulator set jh calls emit(T, jh, lo, hi) with the values of rows g (lo) and
+// g + 8 (hi) for head I8Layout<G>::head(jh, t), digits joined (see emit_tile).  Rows
+// are slots (q·Kᵀ, K record) or channels (p·V, V record).
+template <int BITS, int G, class Emit>
+__device__ __forceinline__ void i8_product(const unsigned char* st,
+                                           const uint32_t (&bf)[4][I8Layout<G>::kNT][2], int lane, Emit&& emit) {
+  constexpr int NT = I8Layout<G>::kNT;
   const uint4* words = reinterpret_cast<const uint4*>(st + kRawWordOffset);
-  const int t = lane & 3;
+  const PairW pw = pair_weights(lane & 3);
   if constexpr (BITS == 4) {
 #pragma unroll
     for (int T = 0; T < 8; ++T) {
@@ -366,7 +437,7 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
       const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
       int d[NT][4];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0;
+      for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = kRoundBits;
 #pragma unroll
       for (int kap = 0; kap < 4; ++kap) {
         uint32_t a[4];
@@ -374,12 +445,7 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
 #pragma unroll
         for (int j = 0; j < NT; ++j) imma16832(d[j], a, bf[kap][j][0], bf[kap][j][1]);
       }
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        float lo, hi;
-        tile_rows(d[j], 1.f, 1.f / 16.f, t, lo, hi);  // low nibbles x1, high nibbles x16
-        emit(T, j, lo, hi);
-      }
+      emit_tile<G>(T, d, 1.f, 1.f / 16.f, pw, emit);  // low nibbles x1, high nibbles x16
     }
   } else if constexpr (BITS == 2) {
 #pragma unroll
@@ -388,10 +454,9 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
       const uint32_t w[4][2] = {{wa.x, wa.y}, {wa.z, wa.w}, {wb.x, wb.y}, {wb.z, wb.w}};
       int de[NT][4], dd[NT][4];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        de[j][0] = de[j][1] = de[j][2] = de[j][3] = 0;
-        dd[j][0] = dd[j][1] = dd[j][2] = dd[j][3] = 0;
-      }
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) de[j][i] = dd[j][i] = kRoundBits;
 #pragma unroll
       for (int kap = 0; kap < 4; ++kap) {
         uint32_t ae[4], ao[4];
@@ -402,14 +467,8 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
           imma16832(dd[j], ao, bf[kap][j][0], bf[kap][j][1]);
         }
       }
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        float lo, hi;
-        tile_rows(de[j], 1.f, 0.25f, t, lo, hi);  // even tile: x1, x4
-        emit(2 * P, j, lo, hi);
-        tile_rows(dd[j], 1.f / 16.f, 1.f / 64.f, t, lo, hi);  // odd tile: x16, x64
-        emit(2 * P + 1, j, lo, hi);
-      }
+      emit_tile<G>(2 * P, de, 1.f, 0.25f, pw, emit);               // even tile: x1, x4
+      emit_tile<G>(2 * P + 1, dd, 1.f / 16.f, 1.f / 64.f, pw, emit);  // odd tile: x16, x64
     }
   } else {
     const uint4* hwords = words + 1024 / 4;  // bit-2 plane
@@ -426,7 +485,7 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
 #pragma unroll
         for (int j = 0; j < NT; ++j)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) le[j][i] = lo_[j][i] = he[j][i] = ho[j][i] = 0;
+          for (int i = 0; i < 4; ++i) le[j][i] = lo_[j][i] = he[j][i] = ho[j][i] = kRoundBits;
 #pragma unroll
         for (int kap = 0; kap < 4; ++kap) {
           uint32_t ae[4], ao[4], be[4], bo[4];
@@ -448,14 +507,8 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
         }
         // bit 2 weighs 4; tile 4Q + s (s = 2pp, 2pp+1) carries 2^(2s) (row g), 2^(2s+1) (row g+8)
         const float e0 = 4.f / float(1 << (4 * pp)), e1 = 4.f / float(1 << (4 * pp + 2));
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          float lo, hi;
-          tile_rows2(le[j], he[j], 1.f, 0.25f, e0, e0 * 0.5f, t, lo, hi);
-          emit(2 * P, j, lo, hi);
-          tile_rows2(lo_[j], ho[j], 1.f / 16.f, 1.f / 64.f, e1, e1 * 0.5f, t, lo, hi);
-          emit(2 * P + 1, j, lo, hi);
-        }
+        emit_tile2<G>(2 * P, le, he, 1.f, 0.25f, e0, e0 * 0.5f, pw, emit);
+        emit_tile2<G>(2 * P + 1, lo_, ho, 1.f / 16.f, 1.f / 64.f, e1, e1 * 0.5f, pw, emit);
       }
     }
   }
@@ -465,37 +518,43 @@ __device__ __forceinline__ void i8_product(const unsigned char* st, const uint32
 template <int BITS, int G>
 __device__ __forceinline__ void qk_i8(const unsigned char* st, const uint32_t* tab, const float (&cst)[G],
                                       const float (&invf)[G], float* sblk, long ld, float scale, int lane) {
-  constexpr int NT = (4 * G + 7) / 8;
+  using L = I8Layout<G>;
   const int g = lane >> 2, t = lane & 3;
-  uint32_t bf[4][NT][2];
-  load_i8frags<NT>(tab, bf, lane);
-  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, float lo, float hi) {
-    const int head = 2 * j + (t >> 1);
-    if ((t & 1) == 0 && head < G) {
-      const float f = head_sel<G>(invf, head), c = head_sel<G>(cst, head);
-      float* dst = sblk + head * ld + 16 * T + g;
-      dst[0] = scale * fmaf(lo, f, c);
-      dst[8] = scale * fmaf(hi, f, c);
+  uint32_t bf[4][L::kNT][2];
+  load_i8frags<L::kNT>(tab, bf, lane);
+  // per accumulator set: this thread's head with the score scale folded in
+  float sf[L::kNH], sc[L::kNH];
+#pragma unroll
+  for (int jh = 0; jh < L::kNH; ++jh) {
+    const int head = L::head(jh, t);
+    sf[jh] = scale * head_sel<G>(invf, head);
+    sc[jh] = scale * head_sel<G>(cst, head);
+  }
+  i8_product<BITS, G>(st, bf, lane, [&](int T, int jh, float lo, float hi) {
+    if (L::owns(jh, t)) {
+      float* dst = sblk + L::head(jh, t) * ld + 16 * T + g;
+      dst[0] = fmaf(lo, sf[jh], sc[jh]);
+      dst[8] = fmaf(hi, sf[jh], sc[jh]);
     }
   });
 }
 
 // p·V of one raw V record: adds sum_slots p'*code into the accumulators of channels
-// 16T + g (acc_lo) and 16T + g + 8 (acc_hi) of head 2j + t/2 (even t).
+// 16T + g (acc_lo) and 16T + g + 8 (acc_hi) of head I8Layout<G>::head(jh, t).
 template <int BITS, int G>
 __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* tab, const float (&invf)[G],
-                                      float (&acc_lo)[(4 * G + 7) / 8][8], float (&acc_hi)[(4 * G + 7) / 8][8],
+                                      float (&acc_lo)[I8Layout<G>::kNH][8], float (&acc_hi)[I8Layout<G>::kNH][8],
                                       int lane) {
-  constexpr int NT = (4 * G + 7) / 8;
+  using L = I8Layout<G>;
   const int t = lane & 3;
-  uint32_t bf[4][NT][2];
-  load_i8frags<NT>(tab, bf, lane);
-  float f_t[NT];
+  uint32_t bf[4][L::kNT][2];
+  load_i8frags<L::kNT>(tab, bf, lane);
+  float f_t[L::kNH];
 #pragma unroll
-  for (int j = 0; j < NT; ++j) f_t[j] = head_sel<G>(invf, 2 * j + (t >> 1));
-  i8_product<BITS, NT>(st, bf, lane, [&](int T, int j, float lo, float hi) {
-    acc_lo[j][T] = fmaf(lo, f_t[j], acc_lo[j][T]);
-    acc_hi[j][T] = fmaf(hi, f_t[j], acc_hi[j][T]);
+  for (int jh = 0; jh < L::kNH; ++jh) f_t[jh] = head_sel<G>(invf, L::head(jh, t));
+  i8_product<BITS, G>(st, bf, lane, [&](int T, int jh, float lo, float hi) {
+    acc_lo[jh][T] = fmaf(lo, f_t[jh], acc_lo[jh][T]);
+    acc_hi[jh][T] = fmaf(hi, f_t[jh], acc_hi[jh][T]);
   });
 }
 
@@ -518,7 +577,7 @@ __device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, 
 
 // One compressed K record, lane = token within each pack group.
 template <int G>
-__device__ __forceinline__ void qk_packed(const unsigned char* st, const float2* qp, const float (&cst)[G],
+__device__ __forceinline__ void qk_packed(const unsigned char* st, const float* qp, const float (&cst)[G],
                                           float* sblk, long ld, float scale, int lane) {
   const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
   const uint8_t* meta = st + kMetaOffset;
@@ -530,10 +589,11 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float2*
     const uint32_t m4 = *reinterpret_cast<const uint32_t*>(meta + g * 128 + 4 * lane);
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
-      float part = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        part = fmaf(qp[hd * 128 + table_index(4 * lane + i)].x, (float)((m4 >> (8 * i)) & 15u), part);
+      const float4 q4 = *reinterpret_cast<const float4*>(qp + hd * 128 + 4 * lane);
+      float part = q4.x * (float)(m4 & 15u);
+      part = fmaf(q4.y, (float)((m4 >> 8) & 15u), part);
+      part = fmaf(q4.z, (float)((m4 >> 16) & 15u), part);
+      part = fmaf(q4.w, (float)((m4 >> 24) & 15u), part);
       bsum[hd] = warp_sum(part);
     }
     float acc[G];
@@ -549,7 +609,7 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float2*
         const float u = (float)unit_field(W, s, w, lane);
         s += w;
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(qp[hd * 128 + table_index(4 * c4 + i)].x, u, acc[hd]);
+        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(qp[hd * 128 + 4 * c4 + i], u, acc[hd]);
       }
     }
 #pragma unroll

@@ -44,7 +44,7 @@ namespace packkv {
 namespace {
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, (G == 4 && BITS == 2) ? 16 / kWarpsPerCta : 0) qk_kernel(const GemvArgs a) {
   using C = Cfg<BITS, G, false>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31;
@@ -136,14 +136,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
         __syncwarp();
         qk_i8<BITS, G>(st, tab, cst, invf, sblk, a.ld, a.scale, lane);
       } else {
-        float2* qp = reinterpret_cast<float2*>(m.table());
+        float* qp = reinterpret_cast<float*>(m.table());
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane)) =
-              make_float4(qv[hd][0], qv[hd][0], qv[hd][1], qv[hd][1]);
-          *reinterpret_cast<float4*>(qp + hd * 128 + table_index(4 * lane + 2)) =
-              make_float4(qv[hd][2], qv[hd][2], qv[hd][3], qv[hd][3]);
-        }
+        for (int hd = 0; hd < G; ++hd)
+          *reinterpret_cast<float4*>(qp + hd * 128 + 4 * lane) = make_float4(qv[hd][0], qv[hd][1], qv[hd][2], qv[hd][3]);
         __syncwarp();
         qk_packed<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
       }
@@ -165,17 +161,17 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) qk_kernel(const GemvArgs a)
 // then go out with coalesced stores.
 template <int G>
 __device__ __forceinline__ void pv_flush(const GemvArgs& a, long bh, int warp, float* sacc,
-                                         float (&acc_lo)[(4 * G + 7) / 8][8], float (&acc_hi)[(4 * G + 7) / 8][8],
+                                         float (&acc_lo)[I8Layout<G>::kNH][8], float (&acc_hi)[I8Layout<G>::kNH][8],
                                          float (&mp)[G], int lane) {
-  constexpr int NT = (4 * G + 7) / 8;
+  using L = I8Layout<G>;
   const int g = lane >> 2, t = lane & 3;
   __syncwarp();
 #pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    const int head = 2 * j + (t >> 1);
+  for (int j = 0; j < L::kNH; ++j) {
+    const int head = L::head(j, t);
 #pragma unroll
     for (int T = 0; T < 8; ++T) {
-      if ((t & 1) == 0 && head < G) {
+      if (L::owns(j, t)) {
         sacc[head * 128 + 16 * T + g] += acc_lo[j][T];
         sacc[head * 128 + 16 * T + g + 8] += acc_hi[j][T];
       }
@@ -261,7 +257,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pv_reduce_kernel(const Gemv
 }
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, (G == 4 && BITS != 3) ? 16 / kWarpsPerCta : 0) pv_kernel(const GemvArgs a) {
   using C = Cfg<BITS, G, true>;
   extern __shared__ __align__(128) unsigned char smem[];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -282,15 +278,30 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
   Cursor cc = pc;
   EntryWindow win;
   win.load(a, lo, hi, lane);
-  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(I))
-    issue_item<BITS, G, true>(a, m, pc, win.get(prod), s, lane);
+  // p of the record in flight (this lane's slots 4*lane .. +3), loaded with its copy
+  float4 pn[G];
+  auto load_p = [&](Cursor c) {
+    if (c.j < a.n_blocks) {
+      const long b = c.bh / a.kv_heads, h = c.bh % a.kv_heads;
+      const float* prow = a.p + ((size_t)b * a.kv_heads * G + h * G) * a.ld + (size_t)c.j * 128;
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) pn[hd] = __ldcs(reinterpret_cast<const float4*>(prow + hd * a.ld) + lane);
+    }
+  };
+  static_assert(C::kStages == 1, "one record in flight per warp");
+  if (prod < hi) {
+    issue_item<BITS, G, true>(a, m, pc, win.get(prod), 0, lane);
+    load_p(pc);
+    ++prod;
+    pc.next(I);
+  }
 
   float mp[G];  // sum over the warp's records of p * mn (lane: slots 4*lane .. +3)
-  float acc_lo[C::kNT][8], acc_hi[C::kNT][8];  // tensor-core path
+  float acc_lo[C::kNH][8], acc_hi[C::kNH][8];  // tensor-core path
 #pragma unroll
   for (int hd = 0; hd < G; ++hd) mp[hd] = 0.f;
 #pragma unroll
-  for (int jn = 0; jn < C::kNT; ++jn)
+  for (int jn = 0; jn < C::kNH; ++jn)
 #pragma unroll
     for (int T = 0; T < 8; ++T) acc_lo[jn][T] = acc_hi[jn][T] = 0.f;
   float* sacc = m.sums();
@@ -331,7 +342,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
       float pv4[G][4];
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
-        const float4 p4 = *reinterpret_cast<const float4*>(st + C::kStageRec + hd * 512 + 16 * lane);
+        const float4 p4 = pn[hd];
         const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -368,6 +379,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32) pv_kernel(const GemvArgs a)
     if (prod < hi) {
       if (prod - win.base >= 32) win.load(a, prod, hi, lane);
       issue_item<BITS, G, true>(a, m, pc, win.get(prod), s, lane);
+      load_p(pc);
       ++prod;
       pc.next(I);
     }
