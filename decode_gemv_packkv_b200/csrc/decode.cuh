@@ -103,6 +103,12 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
+// Warp maximum of non-negative floats, which order like their bit patterns as
+// unsigned integers: one warp reduction instruction.
+__device__ __forceinline__ float warp_max_nonneg(float x) {
+  return __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(x)));
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
@@ -245,15 +251,17 @@ __device__ __forceinline__ void build_i8tab(uint32_t* tab, const float (&x)[G][4
     if (hd < G) {
       const int h = hd < G ? hd : 0;
       const float mx =
-          warp_max(fmaxf(fmaxf(fabsf(x[h][0]), fabsf(x[h][1])), fmaxf(fabsf(x[h][2]), fabsf(x[h][3]))));
-      const float f = mx > 0.f ? __fdividef(127.f, mx) : 1.f;
-      invf[h] = mx > 0.f ? __fdividef(mx, 127.f) : 1.f;
+          warp_max_nonneg(fmaxf(fmaxf(fabsf(x[h][0]), fabsf(x[h][1])), fmaxf(fabsf(x[h][2]), fabsf(x[h][3]))));
+      // |y| <= 127 (the quotient is within 2 ulp); a head whose values are all below
+      // 1e-30 gets zero digits (its products are negligible), so f stays finite
+      const bool nz = mx > 1e-30f;
+      const float f = nz ? __fdividef(127.f, mx) : 0.f;
+      invf[h] = nz ? __fdividef(mx, 127.f) : 0.f;
       const float2 m128 = make_float2(-128.f, -128.f);
       float2 t0[2], t1[2], t2[2];
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
-        float2 y = __fmul2_rn(make_float2(x[h][2 * q], x[h][2 * q + 1]), make_float2(f, f));
-        y = make_float2(fminf(fmaxf(y.x, -127.f), 127.f), fminf(fmaxf(y.y, -127.f), 127.f));
+        const float2 y = __fmul2_rn(make_float2(x[h][2 * q], x[h][2 * q + 1]), make_float2(f, f));
         t0[q] = __fadd2_rn(y, R);                                          // low byte: d0 = rint(y)
         const float2 r1 = __ffma2_rn(__fadd2_rn(t0[q], nR), m128, __fmul2_rn(y, k128));  // 128(y - d0), exact
         t1[q] = __fadd2_rn(r1, R);                                         // low byte: d1 = rint(r1)
@@ -388,12 +396,23 @@ __device__ __forceinline__ float head_sel(const float (&x)[G], int head) {
 }
 
 // A registers of one row tile from its two fragment words (k halves kh = 0, 1).
-// b = 4: rows g (low nibbles, x1) and g + 8 (high nibbles, x16).
+// b = 4: row g + 8 is the high nibbles (x16).  Row g is the low nibbles, or with
+// kWholeBytes the whole bytes, i.e. its codes plus the high nibbles x16: both rows
+// meet the same B values, so the surplus is exactly row g + 8's accumulator,
+// subtracted after the k-steps (unmask4), and a word costs one AND instead of two.
+template <bool kWholeBytes>
 __device__ __forceinline__ void afrag4(uint32_t w0, uint32_t w1, uint32_t (&a)[4]) {
-  a[0] = w0 & 0x0F0F0F0Fu;
+  a[0] = kWholeBytes ? w0 : w0 & 0x0F0F0F0Fu;
   a[1] = w0 & 0xF0F0F0F0u;
-  a[2] = w1 & 0x0F0F0F0Fu;
+  a[2] = kWholeBytes ? w1 : w1 & 0x0F0F0F0Fu;
   a[3] = w1 & 0xF0F0F0F0u;
+}
+
+// Row g of an afrag4 tile: its accumulators minus row g + 8's (columns 2t, 2t + 1),
+// keeping the 1.5*2^23 offset.  Exact: |sum over k of byte * b| <= 128*255*127 < 2^22.
+__device__ __forceinline__ void unmask4(int (&d)[4]) {
+  d[0] = d[0] - d[2] + kRoundBits;
+  d[1] = d[1] - d[3] + kRoundBits;
 }
 
 // b = 2: even tile rows g (x1), g + 8 (x4); odd tile rows g (x16), g + 8 (x64).
@@ -423,7 +442,7 @@ __device__ __forceinline__ void afrag1(uint32_t w0, uint32_t w1, uint32_t (&a)[4
 // accumulator set jh calls emit(T, jh, lo, hi) with the values of rows g (lo) and
 // g + 8 (hi) for head I8Layout<G>::head(jh, t), digits joined (see emit_tile).  Rows
 // are slots (q·Kᵀ, K record) or channels (p·V, V record).
-template <int BITS, int G, class Emit>
+template <int BITS, int G, bool kWholeBytes, class Emit>
 __device__ __forceinline__ void i8_product(const unsigned char* st,
                                            const uint32_t (&bf)[4][I8Layout<G>::kNT][2], int lane, Emit&& emit) {
   constexpr int NT = I8Layout<G>::kNT;
@@ -441,9 +460,13 @@ __device__ __forceinline__ void i8_product(const unsigned char* st,
 #pragma unroll
       for (int kap = 0; kap < 4; ++kap) {
         uint32_t a[4];
-        afrag4(w[kap][0], w[kap][1], a);
+        afrag4<kWholeBytes>(w[kap][0], w[kap][1], a);
 #pragma unroll
         for (int j = 0; j < NT; ++j) imma16832(d[j], a, bf[kap][j][0], bf[kap][j][1]);
+      }
+      if (kWholeBytes) {
+#pragma unroll
+        for (int j = 0; j < NT; ++j) unmask4(d[j]);
       }
       emit_tile<G>(T, d, 1.f, 1.f / 16.f, pw, emit);  // low nibbles x1, high nibbles x16
     }
@@ -530,7 +553,7 @@ __device__ __forceinline__ void qk_i8(const unsigned char* st, const uint32_t* t
     sf[jh] = scale * head_sel<G>(invf, head);
     sc[jh] = scale * head_sel<G>(cst, head);
   }
-  i8_product<BITS, G>(st, bf, lane, [&](int T, int jh, float lo, float hi) {
+  i8_product<BITS, G, true>(st, bf, lane, [&](int T, int jh, float lo, float hi) {
     if (L::owns(jh, t)) {
       float* dst = sblk + L::head(jh, t) * ld + 16 * T + g;
       dst[0] = fmaf(lo, sf[jh], sc[jh]);
@@ -552,7 +575,7 @@ __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* t
   float f_t[L::kNH];
 #pragma unroll
   for (int jh = 0; jh < L::kNH; ++jh) f_t[jh] = head_sel<G>(invf, L::head(jh, t));
-  i8_product<BITS, G>(st, bf, lane, [&](int T, int jh, float lo, float hi) {
+  i8_product<BITS, G, false>(st, bf, lane, [&](int T, int jh, float lo, float hi) {
     acc_lo[jh][T] = fmaf(lo, f_t[jh], acc_lo[jh][T]);
     acc_hi[jh][T] = fmaf(hi, f_t[jh], acc_hi[jh][T]);
   });

@@ -43,8 +43,18 @@ namespace packkv {
 
 namespace {
 
+// Resident CTAs of 4 warps per SM that the register budget is sized for (0: the
+// compiler's choice).  Shared memory admits 4-5 of them for the 2- and 4-bit
+// kernels; without the hint the compiler may settle below 102 registers with spills.
+constexpr int qk_min_ctas(int bits, int g) {
+  return kWarpsPerCta != 4 ? 0 : g == 1 ? 5 : g == 4 ? (bits == 2 ? 4 : bits == 4 ? 5 : 0) : 0;
+}
+constexpr int pv_min_ctas(int bits, int g) {
+  return kWarpsPerCta != 4 ? 0 : g == 1 ? 5 : g == 4 ? (bits == 3 ? 0 : 4) : 0;
+}
+
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, (G == 4 && BITS == 2) ? 16 / kWarpsPerCta : 0) qk_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G)) qk_kernel(const GemvArgs a) {
   using C = Cfg<BITS, G, false>;
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31;
@@ -257,7 +267,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pv_reduce_kernel(const Gemv
 }
 
 template <int BITS, int G>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, (G == 4 && BITS != 3) ? 16 / kWarpsPerCta : 0) pv_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_kernel(const GemvArgs a) {
   using C = Cfg<BITS, G, true>;
   extern __shared__ __align__(128) unsigned char smem[];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
