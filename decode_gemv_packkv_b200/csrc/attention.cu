@@ -456,9 +456,10 @@ __device__ __forceinline__ long attn_warp_of_item(long item, long n_items, long 
 // Second pass: for each output row (b, h, head), the slots of the warps that touched
 // (b, h) are merged with the log-sum-exp rule, M = max m_w, L = sum l_w e^(m_w - M),
 // out_c = sum S_w,c e^(m_w - M) / L, adding in a fixed order (deterministic).  One CTA
-// per row: warp i of 16 takes slots w0+i, w0+i+16, ...; warp 0 adds the 16 warp
-// results in order.  A row whose every record was invalid gets NaN.
-constexpr int kMergeWarps = 16;
+// per row: warp i of 32 takes slots w0+i, w0+i+32, ... (four loop iterations
+// unrolled, so their loads overlap); warp 0 adds the 32 warp results in order.  A row
+// whose every record was invalid gets NaN.
+constexpr int kMergeWarps = 32;
 
 template <int G>
 __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const AttnArgs a) {
@@ -487,6 +488,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   // scaled sums
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
   float l = 0.f;
+#pragma unroll 4
   for (long w = w0 + warp; w <= w1; w += kMergeWarps) {
     const float* p = base + w * stride;
     const float mw = __ldcg(p + 128);

@@ -129,26 +129,29 @@ def test_attention_rejects_an_empty_cache(pk):
     assert err.value.status == pk.ERR_INVALID_ARG
 
 
-def test_attention_full_workload_one_sequence(pk):
-    """32-head 32k-token 4-bit cache: one whole (sequence, head) against the oracle."""
-    w = synth.WORKLOADS[1]
+@pytest.mark.parametrize("wid,bits,h", [(1, 4, 5), (2, 2, 3)])
+def test_attention_full_workload_one_sequence(pk, wid, bits, h):
+    """Full-size caches (32-head 32k-token 4-bit; 8 KV heads x 4 query heads, 131k
+    tokens, 2-bit): one whole (sequence, KV head) against the oracle, in the launch
+    configuration the benchmark uses (hundreds of warps merged per output row)."""
+    w = synth.WORKLOADS[wid]
     T = w.seq
+    G = w.group
     kd = torch.empty((w.batch, w.kv_heads, T, 128), dtype=torch.float16, device="cuda")
     vd = torch.empty_like(kd)
     for b in range(w.batch):
-        for h in range(w.kv_heads):
-            ks, vs = synth.kv_slice(w.seed, w.kv_heads, b, h, T)
-            kd[b, h].copy_(torch.from_numpy(ks))
-            vd[b, h].copy_(torch.from_numpy(vs))
-    cache = pk.PackKVCache(w.batch, w.kv_heads, T // 128, 4)
+        for hh in range(w.kv_heads):
+            ks, vs = synth.kv_slice(w.seed, w.kv_heads, b, hh, T)
+            kd[b, hh].copy_(torch.from_numpy(ks))
+            vd[b, hh].copy_(torch.from_numpy(vs))
+    cache = pk.PackKVCache(w.batch, w.kv_heads, T // 128, bits)
     pk.packkv_encode_block(cache, kd, vd, T // 128)
     q = synth.queries(w, 0)
     out = torch.zeros((w.batch, w.q_heads, 128), device="cuda")
     pk.packkv_attention_decode(cache, to_dev(q), SCALE, out)
     got = out.cpu().numpy()
-    h = 5
-    oc = O.OracleCache(1, 1, T // 128, 4)
+    oc = O.OracleCache(1, 1, T // 128, bits)
     oc.encode_blocks(kd[0:1, h:h + 1].cpu().numpy(), vd[0:1, h:h + 1].cpu().numpy(), T // 128)
-    ref, terms = O.cache_attention(oc, q[0:1, h:h + 1], SCALE)
-    assert_within_terms(got[0:1, h:h + 1], ref, terms, "full-size attention, head 5")
+    ref, terms = O.cache_attention(oc, q[0:1, h * G:(h + 1) * G], SCALE)
+    assert_within_terms(got[0:1, h * G:(h + 1) * G], ref, terms, f"full-size attention, kv head {h}")
     assert np.all(np.isfinite(got))
