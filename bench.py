@@ -140,7 +140,7 @@ def measured_peaks():
 # measured by ncu on this build's kernels (dram__bytes_read.sum + dram__bytes_write.sum,
 # one capture of the 32-head 32k-token 4-bit cache; summary in profiles/).  None for
 # other workloads; to be re-measured whenever the kernel changes.
-DRAM_TRAFFIC = {("llama7b-decode mha b1 h32 d128 seq32768 4-bit", 4): 75.736064e6 + 1.610496e6}
+DRAM_TRAFFIC = {("llama7b-decode mha b1 h32 d128 seq32768 4-bit", 4): 75.735808e6 + 1.264384e6}
 
 
 # ------------------------------------------------------------------ the CUDA path
