@@ -83,8 +83,10 @@ def kv_slice(seed: int, kv_heads: int, b: int, h: int, tokens: int, start: int =
         for z in (zk, zv):
             draw = rng.integers(0, 1 << 30, (n, HEAD_DIM)) % levels[None, :]
             hold = (np.arange(n)[:, None] % runs[0][None, :]) != 0
-            for t in range(1, n):
-                draw[t] = np.where(hold[t], draw[t - 1], draw[t])
+            # each held position repeats the draw of the last position not held
+            src = np.where(hold, 0, np.arange(n)[:, None])
+            src = np.maximum.accumulate(src, axis=0)
+            draw = np.take_along_axis(draw, src, axis=0)
             z[:] = (draw.astype(np.float32) - levels[None, :] / 2.0) / 4.0
     k = (mu[None, :] + sigma[None, :] * zk[start:]).astype(np.float16)
     v = zv[start:].astype(np.float16)
