@@ -584,6 +584,10 @@ __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* t
 // ----------------------------------------------------------------------------
 // q·Kᵀ on the CUDA cores (compressed records)
 // ----------------------------------------------------------------------------
+// Exact float of an unsigned integer u < 2^23: u in the mantissa of 2^23, minus 2^23
+// (two full-rate instructions instead of an integer-to-float conversion).
+__device__ __forceinline__ float small_u2f(uint32_t u) { return __uint_as_float(u | 0x4B000000u) - 8388608.f; }
+
 // Extracts the offset of token j from a compressed unit of width w starting at word s.
 __device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, int j) {
   uint32_t u = 0;
@@ -613,10 +617,10 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float* 
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
       const float4 q4 = *reinterpret_cast<const float4*>(qp + hd * 128 + 4 * lane);
-      float part = q4.x * (float)(m4 & 15u);
-      part = fmaf(q4.y, (float)((m4 >> 8) & 15u), part);
-      part = fmaf(q4.z, (float)((m4 >> 16) & 15u), part);
-      part = fmaf(q4.w, (float)((m4 >> 24) & 15u), part);
+      float part = q4.x * small_u2f(m4 & 15u);
+      part = fmaf(q4.y, small_u2f((m4 >> 8) & 15u), part);
+      part = fmaf(q4.z, small_u2f((m4 >> 16) & 15u), part);
+      part = fmaf(q4.w, small_u2f((m4 >> 24) & 15u), part);
       bsum[hd] = warp_sum(part);
     }
     float acc[G];
@@ -626,13 +630,22 @@ __device__ __forceinline__ void qk_packed(const unsigned char* st, const float* 
 #pragma unroll 1
     for (int c4 = 0; c4 < 32; ++c4) {
       const uint32_t mm = *reinterpret_cast<const uint32_t*>(meta + g * 128 + 4 * c4);
+      float q4[G][4];
+#pragma unroll
+      for (int hd = 0; hd < G; ++hd) {
+        const float4 v = *reinterpret_cast<const float4*>(qp + hd * 128 + 4 * c4);
+        q4[hd][0] = v.x;
+        q4[hd][1] = v.y;
+        q4[hd][2] = v.z;
+        q4[hd][3] = v.w;
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int w = (mm >> (8 * i + 4)) & 15u;
-        const float u = (float)unit_field(W, s, w, lane);
+        const float u = small_u2f(unit_field(W, s, w, lane));
         s += w;
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(qp[hd * 128 + 4 * c4 + i], u, acc[hd]);
+        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(q4[hd][i], u, acc[hd]);
       }
     }
 #pragma unroll
@@ -697,39 +710,49 @@ __device__ __forceinline__ void pv_packed(const unsigned char* st, const float* 
       }
       const int start = carry + incl - w;
       carry += __shfl_sync(0xffffffffu, incl, 31);
+      // this lane's unit (group g, channel c), eight tokens at a time: their offsets,
+      // then p' * offset for a block of HB heads (one head at a time from G = 4 on, which
+      // decodes the unit again per head but keeps the registers of the wider kernels)
+      constexpr int HB = G >= 4 ? 1 : G;
+      const int bit_word = start + ((w & 2) ? 2 : 0);  // the 1-bit slice follows the 2-bit one
+      const uint32_t bit_hi = (w & 2) ? 2u : 0u;       // and is bit 2 of a width-3 unit
 #pragma unroll 1
-      for (int hd = 0; hd < G; ++hd) {
-        const float* pr = pp + hd * 128 + 32 * g;
-        float sum = (float)base * pg[hd * 4 + g];
-        if (w == 4) {
+      for (int h0 = 0; h0 < G; h0 += HB) {
+        float sum[HB];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t word = W[start + q];
+        for (int h = 0; h < HB; ++h) sum[h] = (float)base * pg[(h0 + h) * 4 + g];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) sum = fmaf(pr[8 * q + i], (float)((word >> (4 * i)) & 15u), sum);
+        for (int k = 0; k < 4; ++k) {  // tokens 8k .. 8k+7
+          float u[8];
+          if (w == 4) {
+            const uint32_t word = W[start + k];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = small_u2f((word >> (4 * i)) & 15u);
+          } else {
+            uint32_t two = 0u, one = 0u;
+            if (w & 2) two = W[start + (k >> 1)] >> (16 * (k & 1));
+            if (w & 1) one = W[bit_word] >> (8 * k);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) u[i] = small_u2f(((two >> (2 * i)) & 3u) | (((one >> i) & 1u) << bit_hi));
           }
-        } else {
-          int at = start;
-          float lo_mul = 1.f;
-          if (w & 2) {
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-              const uint32_t word = W[at + q];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) sum = fmaf(pr[16 * q + i], (float)((word >> (2 * i)) & 3u), sum);
-            }
-            at += 2;
-            lo_mul = 4.f;
-          }
-          if (w & 1) {
-            const uint32_t word = W[at];
-            float s1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s1 = fmaf(pr[i], (float)((word >> i) & 1u), s1);
-            sum = fmaf(lo_mul, s1, sum);
+          for (int h = 0; h < HB; ++h) {
+            const float4* pr4 = reinterpret_cast<const float4*>(pp + (h0 + h) * 128 + 32 * g + 8 * k);
+            const float4 pa = pr4[0], pb = pr4[1];
+            float t = sum[h];
+            t = fmaf(pa.x, u[0], t);
+            t = fmaf(pa.y, u[1], t);
+            t = fmaf(pa.z, u[2], t);
+            t = fmaf(pa.w, u[3], t);
+            t = fmaf(pb.x, u[4], t);
+            t = fmaf(pb.y, u[5], t);
+            t = fmaf(pb.z, u[6], t);
+            t = fmaf(pb.w, u[7], t);
+            sum[h] = t;
           }
         }
-        sacc[hd * 128 + c] += sum;
+#pragma unroll
+        for (int h = 0; h < HB; ++h) sacc[(h0 + h) * 128 + c] += sum[h];
       }
     }
   }
