@@ -213,9 +213,6 @@ __device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Exact float of an integer |d| < 2^22.
-__device__ __forceinline__ float i2f_small(int d) { return __int_as_float(d + kRoundBits) - kRound; }
-
 // The low bytes of four floats of the form r + 1.5*2^23 (r an integer, |r| <= 127):
 // the two's-complement bytes of r, packed in order.
 __device__ __forceinline__ uint32_t pack4(float2 lo, float2 hi) {

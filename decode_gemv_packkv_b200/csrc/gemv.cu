@@ -17,16 +17,15 @@
 //  * Dequantization is folded out of the inner loop: k_hat = mn_c + s_c*code
 //    gives score = scale*(sum_c q_c mn_c + sum_c (q_c s_c) code); v_hat =
 //    mn_r + s_r*code gives out_c = sum_r p_r mn_r + sum_r (p_r s_r) code.
-//  * Raw 2/4-bit records (the common case) hold their codes in the fragment
-//    order of an 8-bit integer tensor-core operand: one AND per 32-bit word
-//    yields a whole A register of four codes (times a known power of two), and
-//    mma.sync m16n8k32 (u8 x s8 -> s32, exact) multiplies them by q' or p'
-//    written as three base-128 digits of q'*f (f = 127 / max|q'| per record and
-//    head; about 22 significant bits, the digits in three B columns).
-//  * 3-bit raw records and compressed (frame-of-reference) records are decoded
-//    on the CUDA cores: magic-number decode (LOP3 into the mantissa of 2^23,
-//    packed FP32 add) for raw 3-bit units, per-unit field extraction for
-//    compressed units.
+//  * Raw records (2, 3 and 4 bits; the common case) hold their codes in the
+//    fragment order of an 8-bit integer tensor-core operand: one AND per 32-bit
+//    word yields a whole A register of four codes (times a known power of two;
+//    3-bit records as a 2-bit plane and a 1-bit plane), and mma.sync m16n8k32
+//    (u8 x s8 -> s32, exact) multiplies them by q' or p' written as three
+//    base-128 digits of q'*f (f = 127 / max|q'| per record and head; about 22
+//    significant bits, the digits in three B columns).
+//  * Compressed (frame-of-reference) records are decoded on the CUDA cores by
+//    per-unit field extraction.
 //  * p·V: a warp sums its item range into per-channel fp32 partials and writes
 //    them to the workspace at every (sequence, head) boundary (split-K over the
 //    sequence); a second-pass kernel, launched as a programmatic dependent so
@@ -117,7 +116,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G)) qk_ke
         for (int i = lane; i < 128; i += 32) srow0[hd * a.ld + (long)j * 128 + i] = __int_as_float(0x7fc00000);
     } else {
       // per record: the min term sum_c q_c * mn_c, then q' = q * scale_c as the
-      // int8 tensor-core B table (raw b = 2 / 4) or the CUDA-core q' table
+      // int8 tensor-core B table (raw records) or the CUDA-core q' table
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
