@@ -72,6 +72,18 @@ def test_attention_tail_only_and_large_scores(pk):
         assert_within_terms(got, ref, terms, f"tail-only attention, scale {scale}")
 
 
+@pytest.mark.parametrize("bits", [2, 4])
+def test_attention_peaked_softmax_over_blocks(pk, bits):
+    """A large scale over several blocks: most probabilities underflow to zero, so whole
+    records see p = 0 (zero digit tables) next to records that carry all the weight."""
+    k, v, q = synth.small_case(65 + bits, 1, 2, 4, 5 * 128 + 19)
+    cache, ocache = _build(pk, k, v, bits)
+    got = _attn(pk, cache, q, 4.0)
+    ref, terms = O.cache_attention(ocache, q, 4.0)
+    assert_within_terms(got, ref, terms, "peaked attention")
+    assert pk.packkv_get_status(cache) == 0
+
+
 def test_attention_many_items_per_warp_and_determinism(pk):
     """A long sequence over few (sequence, head) pairs: every warp spans several
     records and (sequence, head) boundaries; two calls agree bit for bit, also with

@@ -128,6 +128,25 @@ def test_pv_parity(pk, bits, group, structured):
     assert_within_terms(got2, ref2, terms2, "p·V (signed p)")
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_pv_zero_and_tiny_weights(pk, bits):
+    """Whole records with p = 0, records with p far below any useful magnitude
+    (1e-35, under the digit-scale floor) and ordinary records side by side: the
+    result stays finite and within the tolerance (the tiny terms are negligible)."""
+    k, v, q = synth.small_case(40 + bits, 1, 2, 2, 4 * 128 + 9)
+    cache, ocache = _build(pk, k, v, bits)
+    rng = np.random.default_rng(bits)
+    p = np.zeros((1, 4, cache.tokens), np.float32)
+    p[..., 0:128] = rng.random((1, 4, 128)).astype(np.float32)      # block 0: ordinary
+    p[..., 256:384] = np.float32(1e-35)                             # block 2: tiny
+    p[..., 512:] = rng.random((1, 4, cache.tokens - 512)).astype(np.float32)  # the tail
+    got = _pv(pk, cache, p)
+    assert np.all(np.isfinite(got))
+    ref, terms = O.cache_pv(ocache, p)
+    assert_within_terms(got, ref, terms, "p·V (zero and tiny records)")
+    assert pk.packkv_get_status(cache) == 0
+
+
 def test_pv_is_deterministic_with_a_dirty_workspace(pk):
     k, v, q = synth.small_case(12, 2, 4, 2, 20 * 128 + 3)
     cache, _ = _build(pk, k, v, 4, keep_perm=False)
