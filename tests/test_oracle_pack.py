@@ -208,3 +208,32 @@ def test_raw_v_record_stores_the_transpose():
     codes = O.quantize_block_v(v[0, 0], 4)[0][perm]      # [slot, channel]
     w0 = int(np.frombuffer(v_rec, "<u4", 1, 528)[0])
     assert w0 & 0xF == codes[0, 0] and (w0 >> 4) & 0xF == codes[0, 8] and (w0 >> 8) & 0xF == codes[1, 0]
+
+
+def test_plain_quant_ratio_closed_form():
+    """Plain b-bit quantization of a 128x128 fp16 block: 2*16384 bytes over the codes
+    (16384*b/8) plus fp16 min and scale for 128 rows (512 bytes)."""
+    assert O.plain_quant_ratio(4) == pytest.approx(32768 / 8704, rel=1e-15)
+    assert O.plain_quant_ratio(3) == pytest.approx(32768 / 6656, rel=1e-15)
+    assert O.plain_quant_ratio(2) == pytest.approx(32768 / 4608, rel=1e-15)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_compression_ratio_of_raw_and_packed_caches(bits):
+    """i.i.d. Gaussian blocks never pack below b bits, so every record is raw and the
+    ratio is exactly 32768 / (528 + 2048 b + 8) per block; run-structured blocks pack,
+    their arena is smaller than all-raw, and with the identity key (runs kept in token
+    order) the ratio beats plain quantization."""
+    nb, T = 4, 4 * 128
+    k, v, _ = synth.small_case(90 + bits, 1, 1, 1, T)
+    oc = O.OracleCache(1, 1, nb, bits, O.KEY_K_SUM)
+    oc.encode_blocks(k, v, nb)
+    raw = O.raw_record_bytes(bits)
+    assert len(oc.k_arena) == nb * raw and len(oc.v_arena) == nb * raw
+    assert O.compression_ratio(T, len(oc.k_arena), nb * 8) == pytest.approx(32768 / (raw + 8), rel=1e-15)
+    ks, vs, _ = synth.small_case(90 + bits, 1, 1, 1, T, structured=True)
+    os_ = O.OracleCache(1, 1, nb, bits, O.KEY_IDENTITY)
+    os_.encode_blocks(ks, vs, nb)
+    for arena in (os_.k_arena, os_.v_arena):
+        assert len(arena) < nb * raw
+        assert O.compression_ratio(T, len(arena), nb * 8) > O.plain_quant_ratio(bits)
