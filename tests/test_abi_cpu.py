@@ -103,3 +103,14 @@ def test_host_checks_reject_before_launch(pk):
     assert lib.packkv_pv_gemv(ctypes.byref(s), k, 256, 2, k, k, 0, None) == pk.ERR_INVALID_ARG  # ws too small
     s = _fake_cache(pk)  # empty cache: q·Kᵀ is a no-op
     assert lib.packkv_qk_gemv(ctypes.byref(s), k, 2, 1.0, k, 0, None, 0, None) == pk.OK
+    # fused attention: an empty cache has no softmax; bad grouping; misaligned output;
+    # a workspace below the size the library reports
+    att = lib.packkv_attention_decode
+    assert att(ctypes.byref(s), k, 2, 1.0, k, k, 1 << 30, None) == pk.ERR_INVALID_ARG
+    s = _fake_cache(pk, n_blocks=2)
+    assert att(ctypes.byref(s), k, 3, 1.0, k, k, 1 << 30, None) == pk.ERR_INVALID_ARG
+    assert att(ctypes.byref(s), k, 6, 1.0, k, k, 1 << 30, None) == pk.ERR_UNSUPPORTED
+    assert att(ctypes.byref(s), k, 2, 1.0, ctypes.c_void_p(0x20000004), k, 1 << 30, None) == pk.ERR_INVALID_ARG
+    need = lib.packkv_attention_workspace_bytes(ctypes.byref(s), 2)
+    assert need > 0
+    assert att(ctypes.byref(s), k, 2, 1.0, k, k, need - 16, None) == pk.ERR_INVALID_ARG
