@@ -33,6 +33,22 @@ def test_header_declares_the_four_calls():
         assert call in names
 
 
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++17")])
+def test_header_is_plain_c_and_cxx(lang, std, tmp_path):
+    """include/*.h compile on their own as strict C99 and as C++ (no torch or CUDA types)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = tmp_path / ("use.c" if lang == "c" else "use.cc")
+        src.write_text(f'#include "{os.path.basename(hdr)}"\nint main(void) {{ return 0; }}\n')
+        r = subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-pedantic", "-fsyntax-only",
+                            "-I", os.path.dirname(hdr), str(src)], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_library_exports_every_declared_symbol(pk):
     lib = ctypes.CDLL(pk.LIB_PATH)
     missing = [n for n in _declared_functions() if not hasattr(lib, n)]
