@@ -1,6 +1,6 @@
 // Device-side helpers shared by the PackKV kernels (sm_100a).
 //
-// Record layout constants follow FORMAT.md section 4 (version 1).  The async
+// Record layout constants follow packed-cache format v1, section 4 (version 1).  The async
 // copy helpers wrap the Hopper/Blackwell bulk-copy engine (cp.async.bulk with an
 // mbarrier completion, never multicast) and the bounded mbarrier wait used by
 // every kernel that stages records in shared memory.

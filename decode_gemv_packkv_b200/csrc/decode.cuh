@@ -1,7 +1,7 @@
 // Device building blocks of the fused decode products over the packed cache:
 // record staging (bulk copies into warp-private shared-memory stages, bounded
 // mbarrier waits), the 8-bit integer tensor-core decode of raw records (2, 3 and
-// 4-bit), and the CUDA-core decode of compressed records (FORMAT.md sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused
+// 4-bit), and the CUDA-core decode of compressed records (packed-cache format v1, sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused
 // attention kernel.
 #pragma once
 
@@ -202,7 +202,7 @@ __device__ void drain_stages(const WarpMem<BITS, G, PV>& m, uint32_t phases, int
 }
 
 // ----------------------------------------------------------------------------
-// 8-bit integer tensor-core decode of raw records (FORMAT.md section 4)
+// 8-bit integer tensor-core decode of raw records (packed-cache format v1, section 4)
 // ----------------------------------------------------------------------------
 // D(16x8, s32) += A(16x32, u8) * B(32x8, s8): exact integer products and sums.
 __device__ __forceinline__ void imma16832(int (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {

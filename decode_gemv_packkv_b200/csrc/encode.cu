@@ -1,5 +1,5 @@
 // PackKV encoder: block quantization, joint token reorder, channel-direction
-// bit-packing (FORMAT.md sections 1-4; PackKV paper page, Figure 2 steps (1)
+// bit-packing (packed-cache format v1, sections 1-4; PackKV paper page, Figure 2 steps (1)
 // and (2), Figure 5 granularities, TL;DR).
 //
 // One encode call is one pass over the input: a CTA per (sequence, head, block)
@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
       }
     }
   }
-  // raw records: words in 8-bit tensor-core fragment order (FORMAT.md section 4).
+  // raw records: words in 8-bit tensor-core fragment order (packed-cache format v1, section 4).
   // A[m][k] = code of slot m, channel k (K: kp row m) or of slot k, channel m (V: vt row
   // m).  A word's byte e holds column k0 + e of rows (16T + 8rh + g): one 32-bit load
   // of a storage-order row gives the four codes of a (row, byte) field set, placed by

@@ -11,7 +11,7 @@
  *     bound together), bit-pack the integer codes along the channel direction;
  *     decompression inside the matrix-vector multiply, no write-back;
  *   - Figure 5: token-wise and channel-wise quantization granularity.
- * Every parameter the pages leave open is fixed by FORMAT.md (version 1).
+ * Every parameter the pages leave open is fixed by the packed-cache format, version 1.
  *
  * Conventions for every call:
  *   - Pointers named "device" are CUDA device pointers; all must be 16-byte
@@ -59,7 +59,7 @@ typedef enum {
 #define PACKKV_DEV_BAD_RECORD 0x4u /* a GEMV met an invalid index entry; its outputs are NaN/skipped */
 #define PACKKV_DEV_TIMEOUT 0x8u    /* a kernel's bounded wait on an async copy gave up */
 
-/* Reorder keys (FORMAT.md section 2). */
+/* Reorder keys (packed-cache format v1, section 2). */
 #define PACKKV_KEY_IDENTITY 0u
 #define PACKKV_KEY_K_SUM 1u
 #define PACKKV_KEY_KV_SUM 2u
@@ -86,7 +86,7 @@ typedef struct {
   int32_t n_blocks;    /* host counter: packed blocks per (sequence, head), uniform over the batch */
   int32_t tail_len;    /* host counter: tokens in the uncompressed tail, 0..127 */
   int32_t reserved0;
-  uint8_t* k_arena;    /* device, arena_bytes: K records (FORMAT.md section 4) */
+  uint8_t* k_arena;    /* device, arena_bytes: K records (packed-cache format v1, section 4) */
   uint8_t* v_arena;    /* device, arena_bytes: V records */
   uint64_t arena_bytes;/* capacity of EACH arena; multiple of 16, at most 2^36 */
   uint32_t* k_index;   /* device u32 [batch][kv_heads][max_blocks][2] = {offset16, length16} */
@@ -119,7 +119,7 @@ packkv_status packkv_cache_reset(packkv_cache* cache, void* stream);
 
 /*
  * Encode n_blocks full blocks per (sequence, head) and append them to the cache
- * (quantize, joint token reorder, channel-direction bit-packing: FORMAT.md
+ * (quantize, joint token reorder, channel-direction bit-packing: packed-cache format v1,
  * sections 1-4; paper page Figures 2 and 5).
  *   k, v: device fp16 [batch][kv_heads][n_blocks*128][128], row-major.
  * Records go to the arenas in ascending (sequence, head, block) order.
@@ -149,7 +149,7 @@ packkv_status packkv_append_token(packkv_cache* cache, const uint16_t* k, const 
 /*
  * scores[b][hq][i] = scale * sum_c q[b][hq][c] * k_hat[b][hq/G][i][c]  (fp32 accumulate)
  * over the packed blocks in storage order, then the tail in arrival order
- * (FORMAT.md sections 6-7; paper page Figure 1, Figure 2 fused decompression).
+ * (packed-cache format v1, sections 6-7; paper page Figure 1, Figure 2 fused decompression).
  *   q:      device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8}.
  *   scores: device fp32, row (b, hq) starts at (b*q_heads + hq) * ld_scores;
  *           ld_scores >= T = n_blocks*128 + tail_len, multiple of 4.

@@ -3,7 +3,7 @@
 TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
 only the tests, the smoke check and the benchmark's CPU-baseline leg do.  It
 shares no code, tables or constants with the CUDA library; both follow the
-written format (FORMAT.md in the repository root) independently.
+written packed-cache format (version 1) independently.
 
 Sources (the PackKV pages; cited by page title and figure/section):
   [Abs]    "PackKV: Reducing KV Cache Memory Footprint through LLM-Aware Lossy
@@ -22,7 +22,7 @@ Sources (the PackKV pages; cited by page title and figure/section):
 The pages fix none of the numbers; the readings taken (block 128, group 32,
 K per channel / V per token, min-max quantizer with an fp16 scale rounded up,
 K-code-sum reorder key, frame-of-reference + width packing in power-of-two
-slices) are the ones written in FORMAT.md.
+slices) are the ones the packed-cache format v1 fixes.
 
 Floating point: the quantizer is defined in fp32 (single IEEE operations, as the
 GPU performs them) so that integer codes agree bit for bit; decoding and both
@@ -212,7 +212,7 @@ def unpack_unit(words: np.ndarray, w: int) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
-# Step 4: record assembly (FORMAT.md section 4)
+# Step 4: record assembly (packed-cache format v1, section 4)
 # ----------------------------------------------------------------------------
 def raw_record_bytes(bits: int) -> int:
     return 16 + 512 + 2048 * bits
@@ -226,7 +226,7 @@ def record_bytes_max(bits: int) -> int:
 def frag_word_bit(bits: int, m: int, k: int):
     """(word index, bit offset) of A[m][k] in the raw fragment order (b = 2, 4).
 
-    Restates FORMAT.md section 4: m = 16T + 8rh + g, k = 32kappa + 16kh + 4t + e,
+    Restates packed-cache format v1, section 4: m = 16T + 8rh + g, k = 32kappa + 16kh + 4t + e,
     lane = 4g + t; the word is picked by (row tile T (b = 4) or tile pair T div 2
     (b = 2), kappa, kh, lane) and the field inside it by (e, rh) (and the tile
     row parity for b = 2): byte e of the word holds row g in its low field(s)
@@ -245,7 +245,7 @@ def frag_word_bit(bits: int, m: int, k: int):
 
 def frag_plane_bit(m: int, k: int):
     """(word index within the 1-bit plane, bit offset) of A[m][k]'s high bit in a raw
-    b = 3 record (FORMAT.md section 4): the word is picked by (tile quad T div 4,
+    b = 3 record (packed-cache format v1, section 4): the word is picked by (tile quad T div 4,
     kappa, kh, lane), the bit by (e, T mod 4, rh)."""
     T, rh, g = m // 16, (m // 8) % 2, m % 8
     kappa, kh, t, e = k // 32, (k // 16) % 2, (k % 16) // 4, k % 4
@@ -362,6 +362,9 @@ def parse_record(rec: bytes) -> ParsedRecord:
     mn = np.frombuffer(rec, dtype="<f2", count=128, offset=16).astype(np.float16)
     sc = np.frombuffer(rec, dtype="<f2", count=128, offset=272).astype(np.float16)
     if raw:
+        # a raw record keeps the header values of the unit layout with every width = b
+        if gws != [g * 128 * bits for g in range(4)] or total_words != 512 * bits:
+            raise ValueError("raw record header does not match the unit layout")
         base = np.zeros((4, 128), np.int64)
         width = np.full((4, 128), bits, np.int64)
         word_at = 528
@@ -416,7 +419,7 @@ def dequant_v(rec: ParsedRecord) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
-# The cache: arenas, index, tail (FORMAT.md section 5)
+# The cache: arenas, index, tail (packed-cache format v1, section 5)
 # ----------------------------------------------------------------------------
 class OracleCache:
     """Mirror of the packed cache state: two arenas, two index tables, the tail."""

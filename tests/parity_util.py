@@ -1,7 +1,7 @@
 """Shared helpers of the GPU parity tests: run the CUDA path through the C ABI
 and the CPU oracle on the same seeded inputs, and compare.
 
-Acceptance (FORMAT.md section 7): encoder output bit-exact; scores and outputs
+Acceptance (packed-cache format v1, section 7): encoder output bit-exact; scores and outputs
 within 1e-3 * sum|terms| per element (exact 0 where sum|terms| = 0).
 """
 from __future__ import annotations

@@ -1,7 +1,7 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
 
 Encoder: records, index, arena ends and permutations bit-exact.  GEMVs: every
-element within 1e-3 * sum|terms| (FORMAT.md section 7).  Small cases span
+element within 1e-3 * sum|terms| (packed-cache format v1, section 7).  Small cases span
 several blocks, pack groups and a ragged tail; the full workload sizes are
 checked in the launch configuration the benchmark times, on sampled blocks the
 oracle computes one by one.

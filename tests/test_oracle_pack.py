@@ -1,9 +1,10 @@
 """Pins for the oracle's reorder, bit-packing and record layout (CPU only).
 
-Format: FORMAT.md sections 2-4 (PackKV paper page, Figure 2 steps 1 and 2;
+Format: packed-cache format v1, sections 2-4 (PackKV paper page, Figure 2 steps 1 and 2;
 TL;DR: reorder with K and V bound together, light lossless encoding).
 """
 import os
+import re
 import struct
 
 import numpy as np
@@ -76,6 +77,18 @@ def _k1_block():
     return k
 
 
+def _expand(txt):
+    """Comma-separated hex items; `x*n` repeats an item, `[x,y]*n` a bracketed list."""
+    vals = []
+    for m in re.finditer(r"\[([^\]]*)\]\*(\d+)|([^,\[\]]+)", txt):
+        if m.group(1) is not None:
+            vals += [int(v, 16) for v in m.group(1).split(",")] * int(m.group(2))
+        else:
+            v, _, n = m.group(3).strip().partition("*")
+            vals += [int(v, 16)] * (int(n) if n else 1)
+    return vals
+
+
 def _expected_record(spec):
     f = dict(t.strip().split("=", 1) for t in spec.split("|")[1:])
     out = bytearray()
@@ -83,10 +96,7 @@ def _expected_record(spec):
     out += struct.pack("<II", int(f["flags"], 16), int(f["total_words"]))
 
     def expand16(txt):
-        vals = []
-        for item in txt.split(","):
-            v, _, n = item.partition("*")
-            vals += [int(v, 16)] * (int(n) if n else 1)
+        vals = _expand(txt)
         assert len(vals) == 128
         return struct.pack("<128H", *vals)
     out += expand16(f["min"]) + expand16(f["scale"])
@@ -97,8 +107,7 @@ def _expected_record(spec):
         meta[int(g) * 128 + int(c)] = int(val, 16)
     out += meta
     if f["words"]:
-        w, _, n = f["words"].partition("*")
-        out += struct.pack("<I", int(w, 16)) * int(n)
+        out += struct.pack(f"<{len(_expand(f['words']))}I", *_expand(f["words"]))
     out += b"\x00" * (int(f["len"]) - len(out))
     return bytes(out)
 
@@ -114,6 +123,47 @@ def test_records_hand_layout(golden_dir):
             assert perm.tolist() == list(range(0, 128, 2)) + list(range(1, 128, 2))
         else:
             assert perm.tolist() == list(range(128))
+
+
+def _kv_block():
+    """Block KV of the record goldens: K as block K1; V[t, c] = 1 for 1 <= c <= n_t with
+    n_t = 2, 0, 1, 1 for t % 4 = 0, 1, 2, 3."""
+    n = np.array([2, 0, 1, 1])[np.arange(128) % 4]
+    v = (np.arange(128)[None, :] >= 1) & (np.arange(128)[None, :] <= n[:, None])
+    return _k1_block(), v.astype(np.float16)
+
+
+def test_records_kv_sum_key(golden_dir):
+    """The K+V code-sum reorder key (key 2): permutation and both records by hand."""
+    specs = {line.split("|")[0].strip(): line for line in _lines(os.path.join(golden_dir, "records.txt"))}
+    k, v = _kv_block()
+    k_rec, v_rec, perm = O.encode_block(k, v, 4, O.KEY_KV_SUM)
+    want_perm = [int(x) for x in specs["KV_perm"].split("|")[1].split(",")]
+    assert perm.tolist() == want_perm
+    assert k_rec == _expected_record(specs["KV_key2_K"])
+    assert v_rec == _expected_record(specs["KV_key2_V"])
+    # the other keys order this block differently, so the golden pins the key itself
+    assert O.encode_block(k, v, 4, O.KEY_K_SUM)[2].tolist() != want_perm
+    assert O.encode_block(k, v, 4, O.KEY_IDENTITY)[2].tolist() != want_perm
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_raw_record_headers(golden_dir, bits):
+    """Raw K and V records: header words (group_word_start, flags with the V bit,
+    total_words) and length by hand; parse_record rejects a raw header that differs."""
+    specs = {line.split("|")[0].strip(): line for line in _lines(os.path.join(golden_dir, "records.txt"))}
+    k, v, _ = synth.small_case(70 + bits, 1, 1, 1, 128)
+    k_rec, v_rec, _ = O.encode_block(k[0, 0], v[0, 0], bits)
+    for rec, which in ((k_rec, "k"), (v_rec, "v")):
+        f = dict(t.strip().split("=", 1) for t in specs[f"RAW_b{bits}_{which}"].split("|")[1:])
+        assert len(rec) == int(f["len"])
+        want = struct.pack("<4H", *[int(x) for x in f["gws"].split(",")]) + \
+            struct.pack("<II", int(f["flags"], 16), int(f["total_words"]))
+        assert rec[:16] == want, which
+        for bad_at, bad in ((2, b"\x01\x00"), (12, b"\x00\x00\x00\x00")):
+            broken = rec[:bad_at] + bad + rec[bad_at + len(bad):]
+            with pytest.raises(ValueError):
+                O.parse_record(broken)
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4])

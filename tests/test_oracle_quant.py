@@ -1,6 +1,6 @@
 """Pins for the oracle's fp16 round-up and quantizer (CPU only).
 
-Format: FORMAT.md section 1 (PackKV paper page, Figure 5 granularities;
+Format: packed-cache format v1, section 1 (PackKV paper page, Figure 5 granularities;
 Figure 2 / TL;DR quantization step).
 """
 import bisect
