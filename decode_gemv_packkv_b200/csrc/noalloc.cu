@@ -51,8 +51,6 @@ bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr
 
 extern "C" {
 
-size_t packkv_pv_noalloc_scratch_bytes(void) { return PACKKV_PV_NOALLOC_SCRATCH_BYTES; }
-
 packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, int64_t ld_p, int32_t q_heads,
                                      float* out, void* stream) {
   const packkv_status st = packkv_cache_check(cache);

@@ -30,7 +30,7 @@ EXPORTED = [
     "packkv_abi_version", "packkv_cache_struct_size", "packkv_status_string", "packkv_record_bytes_max",
     "packkv_workspace_bytes", "packkv_cache_check", "packkv_cache_reset", "packkv_encode_block",
     "packkv_append_token", "packkv_qk_gemv", "packkv_pv_gemv", "packkv_get_status",
-    "packkv_pv_noalloc_scratch_bytes", "packkv_pv_gemv_noalloc", "packkv_attention_workspace_bytes",
+    "packkv_pv_gemv_noalloc", "packkv_attention_workspace_bytes",
     "packkv_attention_decode",
 ]
 
@@ -75,7 +75,6 @@ def _load():
         "packkv_qk_gemv": (ctypes.c_int, [P, vp, i32, f32, vp, i64, vp, sz, vp]),
         "packkv_pv_gemv": (ctypes.c_int, [P, vp, i64, i32, vp, vp, sz, vp]),
         "packkv_get_status": (ctypes.c_int, [P, vp, ctypes.POINTER(u32)]),
-        "packkv_pv_noalloc_scratch_bytes": (sz, []),
         "packkv_pv_gemv_noalloc": (ctypes.c_int, [P, vp, i64, i32, vp, vp]),
         "packkv_attention_workspace_bytes": (sz, [P, i32]),
         "packkv_attention_decode": (ctypes.c_int, [P, vp, i32, f32, vp, vp, sz, vp]),
@@ -238,15 +237,15 @@ def packkv_pv_gemv(cache: PackKVCache, p: torch.Tensor, out: torch.Tensor, ws: t
 def packkv_pv_gemv_noalloc(cache: PackKVCache, p: torch.Tensor, out: torch.Tensor, stream=None):
     """p·V with the library's own fixed scratch instead of a workspace, for callers that
     cannot allocate device memory.  Raises PackKVError (capacity) if the call needs more
-    scratch than packkv_pv_noalloc_scratch_bytes(); overlapping calls share the scratch."""
+    scratch than PV_NOALLOC_SCRATCH_BYTES; overlapping calls share the scratch."""
     if p.dtype != torch.float32 or p.dim() != 3 or out.dtype != torch.float32:
         raise ValueError("p must be fp32 [B, Hq, ld], out fp32 [B, Hq, 128]")
     _check("packkv_pv_gemv_noalloc", _lib.packkv_pv_gemv_noalloc(ctypes.byref(cache.s), _ptr(p), p.shape[2],
                                                                  p.shape[1], _ptr(out), _stream(stream)))
 
 
-def packkv_pv_noalloc_scratch_bytes() -> int:
-    return int(_lib.packkv_pv_noalloc_scratch_bytes())
+# size of the library's fixed p·V scratch (PACKKV_PV_NOALLOC_SCRATCH_BYTES in packkv.h)
+PV_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def packkv_attention_decode(cache: PackKVCache, q: torch.Tensor, scale: float, out: torch.Tensor,

@@ -183,18 +183,23 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
  * because it synchronises the device.
  * Same arguments and result as packkv_pv_gemv minus ws/ws_bytes.  The split-K
  * partials live in a static device array of PACKKV_PV_NOALLOC_SCRATCH_BYTES
- * that every GPU loading the library holds until the process exits; the call
- * allocates nothing.  Returns PACKKV_ERR_CAPACITY, without launching, if the
- * call would need more scratch than that (the need is packkv_workspace_bytes-
- * like: (CTAs launched + batch*kv_heads) * G * 512 bytes, with at most four
- * CTAs per SM; e.g. with G = 4 about 3500 (sequence, kv head) pairs fit on a
- * B200).  The first call
- * on a device looks up the array's device address (a one-time set-up); make
- * that first call before any stream capture.  All calls share the one array:
- * calls that overlap in time on the GPU race.  Nothing in it needs clearing.
+ * (8 MiB) that every GPU loading the library holds until the process exits;
+ * the call allocates nothing.  It needs
+ *     (W + batch*kv_heads) * G * 512 bytes,
+ * W = the warps it launches = min(batch*kv_heads*items per pair, resident warps
+ * of the p·V kernel: SMs x CTAs per SM x 4); e.g. on a B200 with G = 4 (4 CTAs
+ * per SM, W = 2368 once the cache has that many items) about 1700
+ * (sequence, kv head) pairs fit.  A call that needs more returns
+ * PACKKV_ERR_CAPACITY without launching anything.
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up, cached per device); make that first call before any stream capture.
+ * The cached address belongs to the device's current context: after a
+ * cudaDeviceReset in the same process this entry point must not be used again.
+ * All calls share the one array, and it keeps the last call's partials: calls
+ * that overlap in time on the GPU race.  Nothing in it needs clearing (every
+ * partial is written before it is read).  With T == 0, out is set to zero.
  */
 #define PACKKV_PV_NOALLOC_SCRATCH_BYTES (8u << 20)
-size_t packkv_pv_noalloc_scratch_bytes(void);
 packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, int64_t ld_p,
                                      int32_t q_heads, float* out, void* stream);
 

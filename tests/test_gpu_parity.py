@@ -286,6 +286,7 @@ def _sampled_check(pk, w, bits, kd, vd, cache, samples, full_bh):
     assert_within_terms(out.cpu().numpy()[b:b + 1, h * G:(h + 1) * G], ref_o, terms_o, "p·V, whole sequence")
     assert np.all(np.isfinite(s_np))
     assert pk.packkv_get_status(cache) == 0
+    return ocache
 
 
 @pytest.mark.parametrize("wid,bits", [(0, 4), (1, 4), (2, 4), (2, 2), (3, 3)])
@@ -355,4 +356,94 @@ def test_streaming_workload(pk, bits):
         for i in range(w.seq // 128, o.n_blocks):
             assert gpu_record(karena, kindex, b, h, i) == o.record("k", 0, 0, i)
             assert gpu_record(varena, vindex, b, h, i) == o.record("v", 0, 0, i)
+    assert pk.packkv_get_status(cache) == 0
+
+
+# ----------------------------------------------------------------------------- compressed records at scale
+@pytest.mark.parametrize("bits", [4, 2])
+def test_full_size_structured_cache(pk, bits):
+    """The 32-head 32k-token shape on run-structured inputs, where most records are
+    compressed (unit widths 0..b) and some raw, so warps run compressed and raw records
+    back to back in the launch configuration the benchmark uses: records on sampled
+    blocks bit-exact, q·Kᵀ and p·V on sampled blocks and one whole sequence, and the
+    fused attention over that sequence."""
+    w = synth.WORKLOADS[1]
+    kd, vd = _upload(w, w.seq, structured=True)
+    nb = w.seq // 128
+    cache = pk.PackKVCache(w.batch, w.kv_heads, nb, bits)
+    pk.packkv_encode_block(cache, kd, vd, nb)
+    raw = O.raw_record_bytes(bits) // 16
+    for which in ("k", "v"):
+        lens = gpu_records(cache, which)[1][..., 1]
+        assert np.any(lens < raw), f"{which}: no compressed record"
+    assert np.any(gpu_records(cache, "k")[1][..., 1] == raw), "K: no raw record"
+    rng = np.random.default_rng(100 + bits)
+    samples = {(0, int(rng.integers(w.kv_heads)), int(rng.integers(nb))) for _ in range(6)}
+    samples |= {(0, 0, 0), (0, w.kv_heads - 1, nb - 1)}
+    h = 7
+    oc = _sampled_check(pk, w, bits, kd, vd, cache, sorted(samples), (0, h))
+    q = synth.queries(w)
+    out = torch.zeros((w.batch, w.q_heads, 128), device="cuda")
+    pk.packkv_attention_decode(cache, to_dev(q), SCALE, out)
+    ref, terms = O.cache_attention(oc, q[0:1, h:h + 1], SCALE)
+    assert_within_terms(out.cpu().numpy()[0:1, h:h + 1], ref, terms, "attention, whole structured sequence")
+    assert pk.packkv_get_status(cache) == 0
+
+
+@pytest.mark.parametrize("bits,group", [(4, 1), (2, 4), (3, 2)])
+def test_many_items_per_warp(pk, bits, group):
+    """2048 (sequence, head) pairs of 64 blocks plus a 57-token tail: 133k items, about
+    45 per warp, so every warp crosses many (sequence, head) boundaries, reloads its
+    window of index entries and runs compressed records, raw records and tails in one
+    pass.  Eight distinct structured sequences are tiled over the pairs (the oracle
+    decodes each once); scores, outputs and the fused attention are checked on a
+    contiguous run of pairs and on scattered ones."""
+    B, H, nb, tail, n_distinct = 64, 32, 64, 57, 8
+    T = nb * 128 + tail
+    G = group
+    ks, vs = [], []
+    for i in range(n_distinct):
+        k1, v1 = synth.kv_slice(7000 + 10 * bits + G, n_distinct, 0, i, T, structured=True)
+        ks.append(torch.from_numpy(k1))
+        vs.append(torch.from_numpy(v1))
+    kd = torch.empty((B, H, T, 128), dtype=torch.float16, device="cuda")
+    vd = torch.empty_like(kd)
+    for p_ in range(B * H):
+        kd.view(B * H, T, 128)[p_].copy_(ks[p_ % n_distinct], non_blocking=True)
+        vd.view(B * H, T, 128)[p_].copy_(vs[p_ % n_distinct], non_blocking=True)
+    cache = pk.PackKVCache(B, H, nb + 1, bits)
+    pk.packkv_encode_block(cache, kd[:, :, :nb * 128].contiguous(), vd[:, :, :nb * 128].contiguous(), nb)
+    for t in range(nb * 128, T):
+        pk.packkv_append_token(cache, kd[:, :, t].contiguous(), vd[:, :, t].contiguous())
+    del kd, vd
+    oc = []
+    for i in range(n_distinct):
+        o = O.OracleCache(1, 1, nb + 1, bits)
+        o.encode_blocks(ks[i][:nb * 128].numpy()[None, None], vs[i][:nb * 128].numpy()[None, None], nb)
+        for t in range(nb * 128, T):
+            o.append_token(ks[i][t].numpy()[None, None], vs[i][t].numpy()[None, None])
+        oc.append(o)
+    rng = np.random.default_rng(bits * 10 + G)
+    q = rng.standard_normal((B, H * G, 128)).astype(np.float16)
+    ld = (T + 3) // 4 * 4
+    scores = torch.empty((B, H * G, ld), device="cuda")
+    pk.packkv_qk_gemv(cache, to_dev(q), SCALE, scores)
+    p = rng.random((B, H * G, ld)).astype(np.float32)
+    p[:, :, T:] = 0
+    out = torch.empty((B, H * G, 128), device="cuda")
+    pk.packkv_pv_gemv(cache, to_dev(p), out)
+    att = torch.empty((B, H * G, 128), device="cuda")
+    pk.packkv_attention_decode(cache, to_dev(q), SCALE, att)
+    s_np, o_np, a_np = scores.cpu().numpy(), out.cpu().numpy(), att.cpu().numpy()
+    pairs = list(range(600, 760)) + [int(x) for x in rng.integers(0, B * H, 40)] + [0, B * H - 1]
+    for pr in sorted(set(pairs)):
+        b, h = divmod(pr, H)
+        o = oc[pr % n_distinct]
+        hs = slice(h * G, (h + 1) * G)
+        ref, terms = O.cache_qk(o, q[b:b + 1, hs], SCALE)
+        assert_within_terms(s_np[b:b + 1, hs, :T], ref, terms, f"scores of pair {pr}")
+        ref, terms = O.cache_pv(o, p[b:b + 1, hs, :T])
+        assert_within_terms(o_np[b:b + 1, hs], ref, terms, f"p·V of pair {pr}")
+        ref, terms = O.cache_attention(o, q[b:b + 1, hs], SCALE)
+        assert_within_terms(a_np[b:b + 1, hs], ref, terms, f"attention of pair {pr}")
     assert pk.packkv_get_status(cache) == 0
