@@ -11,9 +11,12 @@
 
 namespace {
 
+using packkv::AttnArgs;
 using packkv::EncodeArgs;
 using packkv::GemvArgs;
-using packkv::AttnArgs;
+using packkv::RaggedAppendPlan;
+using packkv::RaggedEncodePlan;
+using packkv::RaggedPlan;
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -41,7 +44,65 @@ packkv_status check_cache(const packkv_cache* c) {
     return PACKKV_ERR_INVALID_ARG;
   if (c->arena_bytes == 0 || (c->arena_bytes & 15u) != 0 || c->arena_bytes > kMaxArenaBytes)
     return PACKKV_ERR_INVALID_ARG;
+  if ((c->seq_blocks == nullptr) != (c->seq_tail == nullptr)) return PACKKV_ERR_INVALID_ARG;
+  if (c->block_table != nullptr && (reinterpret_cast<uintptr_t>(c->block_table) & 3u) != 0)
+    return PACKKV_ERR_INVALID_ARG;
+  if (c->seq_blocks != nullptr) {
+    if (c->batch > PACKKV_RAGGED_MAX_BATCH) return PACKKV_ERR_UNSUPPORTED;
+    if (c->n_blocks != 0 || c->tail_len != 0) return PACKKV_ERR_INVALID_ARG;
+    for (int b = 0; b < c->batch; ++b)
+      if (c->seq_blocks[b] < 0 || c->seq_blocks[b] > c->max_blocks || c->seq_tail[b] < 0 ||
+          c->seq_tail[b] >= PACKKV_BLOCK_TOKENS)
+        return PACKKV_ERR_INVALID_ARG;
+  }
   return PACKKV_OK;
+}
+
+bool is_ragged(const packkv_cache* c) { return c->seq_blocks != nullptr; }
+
+// Plans live in thread-local host storage: a launch copies its parameters when it is
+// enqueued, so the storage is free again when the call returns.
+RaggedPlan& plan_storage() {
+  thread_local RaggedPlan p;
+  return p;
+}
+RaggedEncodePlan& encode_plan_storage() {
+  thread_local RaggedEncodePlan p;
+  return p;
+}
+RaggedAppendPlan& append_plan_storage() {
+  thread_local RaggedAppendPlan p;
+  return p;
+}
+
+// The flat item list of a ragged cache: per sequence its first item and tail; returns
+// the item count and the longest sequence (tokens).
+RaggedPlan& build_plan(const packkv_cache* c, long* n_items, int64_t* t_max) {
+  RaggedPlan& p = plan_storage();
+  long acc = 0;
+  int64_t tm = 0;
+  for (int b = 0; b < c->batch; ++b) {
+    p.base[b] = (int32_t)acc;
+    p.tail[b] = c->seq_tail[b];
+    acc += (long)(c->seq_blocks[b] + (c->seq_tail[b] > 0 ? 1 : 0)) * c->kv_heads;
+    const int64_t tb = (int64_t)c->seq_blocks[b] * PACKKV_BLOCK_TOKENS + c->seq_tail[b];
+    tm = tb > tm ? tb : tm;
+  }
+  p.base[c->batch] = (int32_t)acc;
+  *n_items = acc;
+  *t_max = tm;
+  return p;
+}
+
+// Tokens of the longest sequence (uniform: every sequence).
+int64_t max_tokens(const packkv_cache* c) {
+  if (!is_ragged(c)) return (int64_t)c->n_blocks * PACKKV_BLOCK_TOKENS + c->tail_len;
+  int64_t tm = 0;
+  for (int b = 0; b < c->batch; ++b) {
+    const int64_t tb = (int64_t)c->seq_blocks[b] * PACKKV_BLOCK_TOKENS + c->seq_tail[b];
+    tm = tb > tm ? tb : tm;
+  }
+  return tm;
 }
 
 EncodeArgs encode_args(const packkv_cache* c, const uint16_t* k, const uint16_t* v, int nb) {
@@ -62,6 +123,8 @@ EncodeArgs encode_args(const packkv_cache* c, const uint16_t* k, const uint16_t*
   a.arena_bytes = c->arena_bytes;
   a.perm = c->perm;
   a.ctrl = c->ctrl;
+  a.block_table = c->block_table;
+  a.ragged = false;
   return a;
 }
 
@@ -89,7 +152,19 @@ GemvArgs gemv_args(const packkv_cache* c, int group, const uint8_t* arena, const
   a.ctrl = c->ctrl;
   a.items_per_bh = c->n_blocks + (c->tail_len > 0 ? 1 : 0);
   a.n_items = (long)c->batch * c->kv_heads * a.items_per_bh;
+  a.block_table = c->block_table;
+  a.ragged = is_ragged(c);
   return a;
+}
+
+// The ragged plan of a launch (nullptr for a uniform batch); sets a.n_items.
+template <class A>
+const RaggedPlan* launch_plan(const packkv_cache* c, A& a) {
+  if (!is_ragged(c)) return nullptr;
+  int64_t tm = 0;
+  RaggedPlan& p = build_plan(c, &a.n_items, &tm);
+  a.items_per_bh = 1;  // unused by ragged launches
+  return &p;
 }
 
 }  // namespace
@@ -133,6 +208,8 @@ packkv_status packkv_cache_reset(packkv_cache* cache, void* stream) {
   if (e != cudaSuccess) return PACKKV_ERR_CUDA;
   cache->n_blocks = 0;
   cache->tail_len = 0;
+  if (is_ragged(cache))
+    for (int b = 0; b < cache->batch; ++b) cache->seq_blocks[b] = cache->seq_tail[b] = 0;
   return PACKKV_OK;
 }
 
@@ -140,14 +217,70 @@ packkv_status packkv_encode_block(packkv_cache* cache, const uint16_t* k, const 
                                   void* stream) {
   const packkv_status st = check_cache(cache);
   if (st != PACKKV_OK) return st;
-  if (n_blocks < 0 || cache->tail_len != 0) return PACKKV_ERR_INVALID_ARG;
+  if (n_blocks < 0) return PACKKV_ERR_INVALID_ARG;
+  if (!is_ragged(cache) && cache->tail_len != 0) return PACKKV_ERR_INVALID_ARG;
   if (n_blocks == 0) return PACKKV_OK;
   if (!aligned16(k) || !aligned16(v)) return PACKKV_ERR_INVALID_ARG;
-  if ((int64_t)cache->n_blocks + n_blocks > cache->max_blocks) return PACKKV_ERR_CAPACITY;
   if ((int64_t)cache->batch * cache->kv_heads * n_blocks > 0x7fffffffLL) return PACKKV_ERR_INVALID_ARG;
-  const cudaError_t e = packkv::launch_encode(encode_args(cache, k, v, n_blocks), as_stream(stream));
+  if (!is_ragged(cache)) {
+    if ((int64_t)cache->n_blocks + n_blocks > cache->max_blocks) return PACKKV_ERR_CAPACITY;
+    const cudaError_t e = packkv::launch_encode(encode_args(cache, k, v, n_blocks), nullptr, as_stream(stream));
+    if (e != cudaSuccess) return PACKKV_ERR_CUDA;
+    cache->n_blocks += n_blocks;
+    return PACKKV_OK;
+  }
+  for (int b = 0; b < cache->batch; ++b) {
+    if (cache->seq_tail[b] != 0) return PACKKV_ERR_INVALID_ARG;
+    if ((int64_t)cache->seq_blocks[b] + n_blocks > cache->max_blocks) return PACKKV_ERR_CAPACITY;
+  }
+  RaggedEncodePlan& plan = encode_plan_storage();
+  for (int b = 0; b < cache->batch; ++b) {
+    plan.seq[b] = b;
+    plan.first_block[b] = cache->seq_blocks[b];
+  }
+  EncodeArgs a = encode_args(cache, k, v, n_blocks);
+  a.ragged = true;
+  const cudaError_t e = packkv::launch_encode(a, &plan, as_stream(stream));
   if (e != cudaSuccess) return PACKKV_ERR_CUDA;
-  cache->n_blocks += n_blocks;
+  for (int b = 0; b < cache->batch; ++b) cache->seq_blocks[b] += n_blocks;
+  return PACKKV_OK;
+}
+
+// One token for the sequences with active[b] (all if active is NULL) of a ragged cache.
+packkv_status append_ragged(packkv_cache* cache, const uint16_t* k, const uint16_t* v, const uint8_t* active,
+                            cudaStream_t stream) {
+  RaggedAppendPlan& ap = append_plan_storage();
+  RaggedEncodePlan& ep = encode_plan_storage();
+  int n_done = 0;
+  for (int b = 0; b < cache->batch; ++b) {
+    const bool on = active == nullptr || active[b] != 0;
+    ap.pos[b] = on ? cache->seq_tail[b] : -1;
+    if (on && cache->seq_tail[b] + 1 == PACKKV_BLOCK_TOKENS) {
+      if (cache->seq_blocks[b] >= cache->max_blocks) return PACKKV_ERR_CAPACITY;
+      ep.seq[n_done] = b;
+      ep.first_block[n_done] = cache->seq_blocks[b];
+      ++n_done;
+    }
+  }
+  cudaError_t e = packkv::launch_append_ragged(k, v, cache->k_tail, cache->v_tail, cache->batch, cache->kv_heads,
+                                               ap, stream);
+  if (e != cudaSuccess) return PACKKV_ERR_CUDA;
+  if (n_done > 0) {
+    EncodeArgs a = encode_args(cache, cache->k_tail, cache->v_tail, 1);
+    a.batch = n_done;
+    a.ragged = true;
+    e = packkv::launch_encode(a, &ep, stream);
+    if (e != cudaSuccess) return PACKKV_ERR_CUDA;
+  }
+  for (int b = 0; b < cache->batch; ++b) {
+    if (ap.pos[b] < 0) continue;
+    if (cache->seq_tail[b] + 1 == PACKKV_BLOCK_TOKENS) {
+      cache->seq_blocks[b] += 1;
+      cache->seq_tail[b] = 0;
+    } else {
+      cache->seq_tail[b] += 1;
+    }
+  }
   return PACKKV_OK;
 }
 
@@ -155,6 +288,7 @@ packkv_status packkv_append_token(packkv_cache* cache, const uint16_t* k, const 
   const packkv_status st = check_cache(cache);
   if (st != PACKKV_OK) return st;
   if (!aligned16(k) || !aligned16(v)) return PACKKV_ERR_INVALID_ARG;
+  if (is_ragged(cache)) return append_ragged(cache, k, v, nullptr, as_stream(stream));
   const bool completes = cache->tail_len + 1 == PACKKV_BLOCK_TOKENS;
   if (completes && cache->n_blocks >= cache->max_blocks) return PACKKV_ERR_CAPACITY;
   cudaError_t e = packkv::launch_append(k, v, cache->k_tail, cache->v_tail, cache->batch * cache->kv_heads,
@@ -164,11 +298,20 @@ packkv_status packkv_append_token(packkv_cache* cache, const uint16_t* k, const 
     cache->tail_len += 1;
     return PACKKV_OK;
   }
-  e = packkv::launch_encode(encode_args(cache, cache->k_tail, cache->v_tail, 1), as_stream(stream));
+  e = packkv::launch_encode(encode_args(cache, cache->k_tail, cache->v_tail, 1), nullptr, as_stream(stream));
   if (e != cudaSuccess) return PACKKV_ERR_CUDA;
   cache->n_blocks += 1;
   cache->tail_len = 0;
   return PACKKV_OK;
+}
+
+packkv_status packkv_append_token_masked(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
+                                         const uint8_t* active, void* stream) {
+  const packkv_status st = check_cache(cache);
+  if (st != PACKKV_OK) return st;
+  if (!is_ragged(cache)) return PACKKV_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || active == nullptr) return PACKKV_ERR_INVALID_ARG;
+  return append_ragged(cache, k, v, active, as_stream(stream));
 }
 
 packkv_status packkv_qk_gemv(const packkv_cache* cache, const uint16_t* q, int32_t q_heads, float scale,
@@ -180,15 +323,16 @@ packkv_status packkv_qk_gemv(const packkv_cache* cache, const uint16_t* q, int32
   int g = 0;
   if (q_heads < 1 || q_heads % cache->kv_heads != 0) return PACKKV_ERR_INVALID_ARG;
   if (!group_ok(cache, q_heads, &g)) return PACKKV_ERR_UNSUPPORTED;
-  const int64_t T = (int64_t)cache->n_blocks * PACKKV_BLOCK_TOKENS + cache->tail_len;
+  const int64_t T = max_tokens(cache);
   if (!aligned16(q) || !aligned16(scores) || ld_scores < T || ld_scores % 4 != 0) return PACKKV_ERR_INVALID_ARG;
   if (T == 0) return PACKKV_OK;
   GemvArgs a = gemv_args(cache, g, cache->k_arena, cache->k_index, cache->k_tail);
+  const RaggedPlan* plan = launch_plan(cache, a);
   a.q = q;
   a.scores = scores;
   a.ld = ld_scores;
   a.scale = scale;
-  return cuda_status(packkv::launch_qk(a, as_stream(stream)));
+  return cuda_status(packkv::launch_qk(a, plan, as_stream(stream)));
 }
 
 packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t ld_p, int32_t q_heads, float* out,
@@ -198,7 +342,7 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
   int g = 0;
   if (q_heads < 1 || q_heads % cache->kv_heads != 0) return PACKKV_ERR_INVALID_ARG;
   if (!group_ok(cache, q_heads, &g)) return PACKKV_ERR_UNSUPPORTED;
-  const int64_t T = (int64_t)cache->n_blocks * PACKKV_BLOCK_TOKENS + cache->tail_len;
+  const int64_t T = max_tokens(cache);
   if (!aligned16(p) || !aligned16(out) || ld_p < T || ld_p % 4 != 0) return PACKKV_ERR_INVALID_ARG;
   if (T == 0) {
     const size_t bytes = (size_t)cache->batch * q_heads * PACKKV_HEAD_DIM * sizeof(float);
@@ -207,11 +351,12 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
   const size_t need = packkv::pv_workspace_bytes(cache->batch, cache->kv_heads, g);
   if (!aligned16(ws) || ws_bytes < need) return PACKKV_ERR_INVALID_ARG;
   GemvArgs a = gemv_args(cache, g, cache->v_arena, cache->v_index, cache->v_tail);
+  const RaggedPlan* plan = launch_plan(cache, a);
   a.p = p;
   a.ld = ld_p;
   a.out = out;
   a.partials = reinterpret_cast<float*>(ws);
-  return cuda_status(packkv::launch_pv(a, as_stream(stream)));
+  return cuda_status(packkv::launch_pv(a, plan, as_stream(stream)));
 }
 
 size_t packkv_attention_workspace_bytes(const packkv_cache* cache, int32_t q_heads) {
@@ -228,8 +373,8 @@ packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t*
   int g = 0;
   if (q_heads < 1 || q_heads % cache->kv_heads != 0) return PACKKV_ERR_INVALID_ARG;
   if (!group_ok(cache, q_heads, &g)) return PACKKV_ERR_UNSUPPORTED;
-  const int64_t T = (int64_t)cache->n_blocks * PACKKV_BLOCK_TOKENS + cache->tail_len;
-  if (T == 0 || !aligned16(q) || !aligned16(out)) return PACKKV_ERR_INVALID_ARG;
+  const int64_t T = max_tokens(cache);
+  if ((T == 0 && !is_ragged(cache)) || !aligned16(q) || !aligned16(out)) return PACKKV_ERR_INVALID_ARG;
   const size_t need = packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, g);
   if (!aligned16(ws) || ws_bytes < need) return PACKKV_ERR_INVALID_ARG;
   AttnArgs a{};
@@ -250,11 +395,14 @@ packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t*
   a.ctrl = cache->ctrl;
   a.items_per_bh = cache->n_blocks + (cache->tail_len > 0 ? 1 : 0);
   a.n_items = (long)cache->batch * cache->kv_heads * a.items_per_bh;
+  a.block_table = cache->block_table;
+  a.ragged = is_ragged(cache);
+  const RaggedPlan* plan = launch_plan(cache, a);
   a.q = q;
   a.scale = scale;
   a.out = out;
   a.partials = reinterpret_cast<float*>(ws);
-  return cuda_status(packkv::launch_attention(a, as_stream(stream)));
+  return cuda_status(packkv::launch_attention(a, plan, as_stream(stream)));
 }
 
 packkv_status packkv_get_status(const packkv_cache* cache, void* stream, uint32_t* bits_out) {

@@ -49,8 +49,7 @@ struct AttnCfg {
   static constexpr int kStageRec = C::kStageRec;  // one K or one V record
   static constexpr int kNT = C::kNT;
   static constexpr int kI8Tab = C::kI8Tab;
-  static constexpr int kCoreTab = 528 * G;  // q' [G][128]; p'' [G][128] + group sums [G][4]
-  static constexpr int kTableBytes = ((kI8Tab > kCoreTab ? kI8Tab : kCoreTab) + 15) / 16 * 16;
+  static constexpr int kTableBytes = (kI8Tab + 15) / 16 * 16;
   static constexpr int kScoreBytes = 512 * G;  // [G][128] scores, then probabilities
   static constexpr int kSumBytes = 512 * G;    // [G][128] channel sums (CUDA-core and tail paths)
   static constexpr int kFixed = kAttnStages * kStageRec + kTableBytes + kScoreBytes + kSumBytes;
@@ -92,19 +91,21 @@ __device__ __forceinline__ GemvArgs tensor_view(const AttnArgs& a, bool v) {
   g.n_items = a.n_items;
   g.items_per_bh = a.items_per_bh;
   g.n_warps = a.n_warps;
+  g.block_table = a.block_table;
+  g.ragged = a.ragged;
   return g;
 }
 
 // Scaled scores of the fp16 tail tokens of (sequence, head) bh into sc[head*128 + t].
 template <int G>
-__device__ __forceinline__ void tail_scores(const AttnArgs& a, long bh, const float (&qr)[G][4], float* sc,
+__device__ __forceinline__ void tail_scores(const AttnArgs& a, long bh, int tl, const float (&qr)[G][4], float* sc,
                                             int lane) {
   const uint16_t* tail = a.k_tail + (size_t)bh * 128 * 128;
-  for (int t0 = 0; t0 < a.tail_len; t0 += 32) {
+  for (int t0 = 0; t0 < tl; t0 += 32) {
     float mine[G];
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) mine[hd] = 0.f;
-    const int tn = min(32, a.tail_len - t0);
+    const int tn = min(32, tl - t0);
     for (int t = 0; t < tn; ++t) {
       const uint2 hv = *reinterpret_cast<const uint2*>(tail + (size_t)(t0 + t) * 128 + 4 * lane);
       const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
@@ -128,14 +129,15 @@ __device__ __forceinline__ void tail_scores(const AttnArgs& a, long bh, const fl
 
 // Adds sum_t p[head][t] * v_tail[t][c] into the channel sums (lane = channel sl*32 + lane).
 template <int G>
-__device__ __forceinline__ void tail_values(const AttnArgs& a, long bh, const float* p, float* sacc, int lane) {
+__device__ __forceinline__ void tail_values(const AttnArgs& a, long bh, int tl, const float* p, float* sacc,
+                                            int lane) {
   const uint16_t* tail = a.v_tail + (size_t)bh * 128 * 128;
   float acc[4][G];
 #pragma unroll
   for (int sl = 0; sl < 4; ++sl)
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) acc[sl][hd] = 0.f;
-  for (int t = 0; t < a.tail_len; ++t) {
+  for (int t = 0; t < tl; ++t) {
     float vv[4];
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
@@ -199,8 +201,13 @@ __device__ __forceinline__ void attn_flush(const AttnArgs& a, long bh, int warp,
   __syncwarp();
 }
 
-template <int BITS, int G>
-__global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a) {
+// Resident CTAs per SM the register budget is sized for: shared memory admits five
+// 4-warp CTAs of the 2- and 4-bit single-head kernels, which then need <= 102 registers.
+constexpr int attn_min_ctas(int bits, int g) { return kAttnWarps == 4 && g == 1 && bits != 3 ? 5 : 0; }
+
+template <int BITS, int G, class Plan>
+__global__ void __launch_bounds__(kAttnWarps * 32, attn_min_ctas(BITS, G))
+    attn_kernel(const AttnArgs a, const __grid_constant__ Plan plan) {
   using A = AttnCfg<BITS, G>;
   using C = Cfg<BITS, G, false>;
   constexpr int NT = A::kNT;
@@ -214,17 +221,17 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
   const GemvArgs ka = tensor_view(a, false), va = tensor_view(a, true);
   const long lo = (long)((long long)a.n_items * warp / a.n_warps);
   const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
-  const int I = a.items_per_bh;
   if (lane == 0) {
     mbar_init(m.bar(0), 1);
     mbar_init(m.bar(1), 1);
     fence_mbar_init();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's results are visible
   __syncwarp();
-  Cursor cc{lo / I, (int)(lo % I)};
+  Cursor cc = cursor_at(a, plan, lo);
   EntryWindow wk, wv;
-  wk.load(ka, lo, hi, lane);
-  wv.load(va, lo, hi, lane);
+  wk.load(ka, plan, lo, hi, lane);
+  wv.load(va, plan, lo, hi, lane);
   issue_item<BITS, G, false>(ka, m, cc, wk.get(lo), 0, lane);
   if (!kOneStage) issue_item<BITS, G, false>(va, m, cc, wv.get(lo), 1, lane);
 
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
       }
     }
     Cursor nc = cc;
-    nc.next(I);
+    cursor_next(a, plan, nc);
 
     // ---- K: scaled scores of this item's tokens into sc[head][slot] ----------
     bool ok = mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
@@ -276,17 +283,18 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
       if (!kOneStage) mbar_wait_bounded(m.bar(1), (phases >> 1) & 1u, a.ctrl);
       return;
     }
-    const int kind_k = *m.kind(0);
+    const int kind_len_k = *m.kind(0);
+    const int kind_k = kind_len_k & 0xFF;
     int n_tok = 128;
     bool skip = false;
     if (kind_k == kKindTail) {
-      n_tok = a.tail_len;
-      tail_scores<G>(a, bh, qr, sc, lane);
+      n_tok = cc.tl;
+      tail_scores<G>(a, bh, cc.tl, qr, sc, lane);
     } else if (kind_k == kKindInvalid) {
       if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
       skip = true;
     } else {
-      const unsigned char* st = m.stage(0);
+      unsigned char* st = m.stage(0);
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -306,27 +314,24 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
         qv[hd][2] = qr[hd][2] * sc1.x;
         qv[hd][3] = qr[hd][3] * sc1.y;
       }
+      uint32_t* tab = m.table();
+      float invf[G];
+      build_i8tab<G, NT>(tab, qv, invf, lane);
+      __syncwarp();
       if (kind_k == kKindRaw) {
-        uint32_t* tab = m.table();
-        float invf[G];
-        build_i8tab<G, NT>(tab, qv, invf, lane);
-        __syncwarp();
         qk_i8<BITS, G>(st, tab, cst, invf, sc, 128, a.scale, lane);
-      } else {
-        float* qp = reinterpret_cast<float*>(m.table());
-#pragma unroll
-        for (int hd = 0; hd < G; ++hd)
-          *reinterpret_cast<float4*>(qp + hd * 128 + 4 * lane) = make_float4(qv[hd][0], qv[hd][1], qv[hd][2], qv[hd][3]);
-        __syncwarp();
-        qk_packed<G>(st, qp, cst, sc, 128, a.scale, lane);
+      } else if (!qk_packed_tc<BITS, G>(st, (uint32_t)(kind_len_k >> 8) * 16u, tab, qv, cst, invf, sc, 128, a.scale,
+                                         lane)) {
+        if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
+        skip = true;
       }
     }
     __syncwarp();
     if (kOneStage) {  // the stage is free: this item's V record
-      if (x - wv.base >= 32) wv.load(va, x, hi, lane);
+      if (x - wv.base >= 32) wv.load(va, plan, x, hi, lane);
       issue_item<BITS, G, false>(va, m, cc, wv.get(x), 1, lane);
     } else if (x + 1 < hi) {  // the K stage is free: the next item's K record
-      if (x + 1 - wk.base >= 32) wk.load(ka, x + 1, hi, lane);
+      if (x + 1 - wk.base >= 32) wk.load(ka, plan, x + 1, hi, lane);
       issue_item<BITS, G, false>(ka, m, nc, wk.get(x + 1), 0, lane);
     }
 
@@ -379,17 +384,18 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
       if (!kOneStage && x + 1 < hi) mbar_wait_bounded(m.bar(0), phases & 1u, a.ctrl);
       return;
     }
-    const int kind_v = *m.kind(1);
+    const int kind_len_v = *m.kind(1);
+    const int kind_v = kind_len_v & 0xFF;
     if (kind_v == kKindTail) {
 #pragma unroll
       for (int hd = 0; hd < G; ++hd)
         *reinterpret_cast<float4*>(sc + hd * 128 + 4 * lane) = make_float4(pr[hd][0], pr[hd][1], pr[hd][2], pr[hd][3]);
       __syncwarp();
-      tail_values<G>(a, bh, sc, sacc, lane);
+      tail_values<G>(a, bh, cc.tl, sc, sacc, lane);
     } else if (kind_v == kKindInvalid) {
       if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
     } else if (!skip) {
-      const unsigned char* st = m.stage(1);
+      unsigned char* st = m.stage(1);
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -399,46 +405,39 @@ __global__ void __launch_bounds__(kAttnWarps * 32) attn_kernel(const AttnArgs a)
       const float mnr[4] = {mn0.x, mn0.y, mn1.x, mn1.y};
       const float scr[4] = {sc0.x, sc0.y, sc1.x, sc1.y};
       float pv4[G][4];
+      float mpr[G];
 #pragma unroll
-      for (int hd = 0; hd < G; ++hd)
+      for (int hd = 0; hd < G; ++hd) {
+        mpr[hd] = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          mp[hd] = fmaf(pr[hd][i], mnr[i], mp[hd]);
+          mpr[hd] = fmaf(pr[hd][i], mnr[i], mpr[hd]);
           pv4[hd][i] = pr[hd][i] * scr[i];
         }
-      if (kind_v == kKindRaw) {
-        uint32_t* tab = m.table();
-        float invf[G];
-        build_i8tab<G, NT>(tab, pv4, invf, lane);
-        __syncwarp();
+      }
+      uint32_t* tab = m.table();
+      float invf[G];
+      build_i8tab<G, NT>(tab, pv4, invf, lane);
+      __syncwarp();
+      bool ok = true;
+      if (kind_v == kKindRaw)
         pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
-      } else {
-        float* pp = reinterpret_cast<float*>(m.table());  // p'' [G][128] then group sums [G][4]
-        // compressed record: p' by storage slot and the per-group sums of p'
+      else
+        ok = pv_packed_tc<BITS, G>(st, (uint32_t)(kind_len_v >> 8) * 16u, tab, pv4, invf, sacc, lane);
+      if (ok) {
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          float ps = 0.f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ps += pv4[hd][i];
-          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) =
-              make_float4(pv4[hd][0], pv4[hd][1], pv4[hd][2], pv4[hd][3]);
-          // lanes 8g .. 8g+7 hold group g
-          ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-          ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-          ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-          if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
-        }
-        __syncwarp();
-        pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
+        for (int hd = 0; hd < G; ++hd) mp[hd] += mpr[hd];
+      } else if (lane == 0) {
+        set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
       }
     }
     __syncwarp();
     if (x + 1 < hi) {
       if (kOneStage) {  // the stage is free: the next item's K record
-        if (x + 1 - wk.base >= 32) wk.load(ka, x + 1, hi, lane);
+        if (x + 1 - wk.base >= 32) wk.load(ka, plan, x + 1, hi, lane);
         issue_item<BITS, G, false>(ka, m, nc, wk.get(x + 1), 0, lane);
       } else {  // the V stage is free: the next item's V record
-        if (x + 1 - wv.base >= 32) wv.load(va, x + 1, hi, lane);
+        if (x + 1 - wv.base >= 32) wv.load(va, plan, x + 1, hi, lane);
         issue_item<BITS, G, false>(va, m, nc, wv.get(x + 1), 1, lane);
       }
     }
@@ -461,8 +460,10 @@ __device__ __forceinline__ long attn_warp_of_item(long item, long n_items, long 
 // whose every record was invalid gets NaN.
 constexpr int kMergeWarps = 32;
 
-template <int G>
-__global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const AttnArgs a) {
+template <int G, class Plan>
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    attn_merge_kernel(const AttnArgs a, const __grid_constant__ Plan plan) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 wsum[kMergeWarps][32];
   __shared__ float wl[kMergeWarps];
@@ -471,9 +472,14 @@ __global__ void __launch_bounds__(kMergeWarps * 32) attn_merge_kernel(const Attn
   const long bh = row / G;
   const int hd = (int)(row % G);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long I = a.items_per_bh;
-  const long w0 = attn_warp_of_item(bh * I, a.n_items, a.n_warps) + bh;
-  const long w1 = attn_warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps) + bh;
+  long first = 0, n = 0;
+  row_items(a, plan, bh, &first, &n);
+  if (n == 0) {  // a sequence without tokens (ragged batches): its output is zero
+    if (warp == 0) reinterpret_cast<float4*>(a.out + row * 128)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const long w0 = attn_warp_of_item(first, a.n_items, a.n_warps) + bh;
+  const long w1 = attn_warp_of_item(first + n - 1, a.n_items, a.n_warps) + bh;
   const float* base = a.partials + hd * kSlotFloats;
   const size_t stride = (size_t)G * kSlotFloats;
   // the overall maximum
@@ -525,16 +531,17 @@ struct AttnKernel {
   int smem;
 };
 
-template <int BITS, int G>
+template <int BITS, int G, class Plan>
 AttnKernel attn_info() {
-  return {reinterpret_cast<const void*>(&attn_kernel<BITS, G>), kAttnWarps * AttnCfg<BITS, G>::kWarpSmem};
+  return {reinterpret_cast<const void*>(&attn_kernel<BITS, G, Plan>), kAttnWarps * AttnCfg<BITS, G>::kWarpSmem};
 }
 
+template <class Plan>
 bool attn_select(int bits, int group, AttnKernel* out) {
-#define PACKKV_ACASE(B, GG)          \
-  if (bits == B && group == GG) {    \
-    *out = attn_info<B, GG>();       \
-    return true;                     \
+#define PACKKV_ACASE(B, GG)            \
+  if (bits == B && group == GG) {      \
+    *out = attn_info<B, GG, Plan>();   \
+    return true;                       \
   }
   PACKKV_ACASE(4, 1) PACKKV_ACASE(4, 2) PACKKV_ACASE(4, 4) PACKKV_ACASE(4, 8)
   PACKKV_ACASE(3, 1) PACKKV_ACASE(3, 2) PACKKV_ACASE(3, 4) PACKKV_ACASE(3, 8)
@@ -584,25 +591,40 @@ size_t attention_workspace_bytes(int batch, int kv_heads, int group) {
   return ((size_t)attn_max_warps() + bh) * group * kSlotFloats * sizeof(float);
 }
 
-cudaError_t launch_attention(AttnArgs a, cudaStream_t stream) {
+template <int G, class Plan>
+const void* merge_fn() {
+  return reinterpret_cast<const void*>(&attn_merge_kernel<G, Plan>);
+}
+
+template <class Plan>
+cudaError_t launch_attention_t(AttnArgs a, const Plan* plan, cudaStream_t stream) {
   AttnKernel k{};
-  if (!attn_select(a.bits, a.group, &k)) return cudaErrorInvalidValue;
+  if (!attn_select<Plan>(a.bits, a.group, &k)) return cudaErrorInvalidValue;
   int w = 0;
   cudaError_t e = attn_resident_warps(k, &w);
   if (e != cudaSuccess) return e;
   if (w > attn_max_warps()) w = attn_max_warps();
   a.n_warps = (int)(a.n_items < w ? a.n_items : w);
+  if (a.n_warps < 1) a.n_warps = 1;
   const unsigned grid = (unsigned)((a.n_warps + kAttnWarps - 1) / kAttnWarps);
-  void* args[] = {&a};
-  e = cudaLaunchKernel(k.fn, dim3(grid), dim3(kAttnWarps * 32), args, k.smem, stream);
-  if (e != cudaSuccess) return e;
-  const void* merge = nullptr;
-  switch (a.group) {
-    case 1: merge = reinterpret_cast<const void*>(&attn_merge_kernel<1>); break;
-    case 2: merge = reinterpret_cast<const void*>(&attn_merge_kernel<2>); break;
-    case 4: merge = reinterpret_cast<const void*>(&attn_merge_kernel<4>); break;
-    default: merge = reinterpret_cast<const void*>(&attn_merge_kernel<8>); break;
+  void* args[] = {&a, const_cast<Plan*>(plan)};
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  if (a.n_items > 0) {
+    // a programmatic dependent of whatever precedes it (griddepcontrol.wait in the kernel)
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(grid);
+    lc.blockDim = dim3(kAttnWarps * 32);
+    lc.dynamicSmemBytes = (size_t)k.smem;
+    lc.stream = stream;
+    lc.attrs = pdl;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelExC(&lc, k.fn, args);
+    if (e != cudaSuccess) return e;
   }
+  const void* merge = a.group == 1 ? merge_fn<1, Plan>() : a.group == 2 ? merge_fn<2, Plan>()
+                    : a.group == 4 ? merge_fn<4, Plan>() : merge_fn<8, Plan>();
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)((long)a.batch * a.kv_heads * a.group));
   cfg.blockDim = dim3(kMergeWarps * 32);
@@ -612,8 +634,13 @@ cudaError_t launch_attention(AttnArgs a, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.n_items > 0 ? 1 : 0;
   return cudaLaunchKernelExC(&cfg, merge, args);
+}
+
+cudaError_t launch_attention(AttnArgs a, const RaggedPlan* plan, cudaStream_t stream) {
+  static const NoPlan none{};
+  return plan ? launch_attention_t<RaggedPlan>(a, plan, stream) : launch_attention_t<NoPlan>(a, &none, stream);
 }
 
 }  // namespace packkv

@@ -1,8 +1,8 @@
 // Device building blocks of the fused decode products over the packed cache:
 // record staging (bulk copies into warp-private shared-memory stages, bounded
 // mbarrier waits), the 8-bit integer tensor-core decode of raw records (2, 3 and
-// 4-bit), and the CUDA-core decode of compressed records (packed-cache format v1, sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused
-// attention kernel.
+// 4-bit) and of compressed records (units sorted by width; packed-cache format v1,
+// sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused attention kernel.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -64,9 +64,7 @@ struct Cfg {
   static constexpr int kNT = I8Layout<G>::kNT;
   static constexpr int kNH = I8Layout<G>::kNH;
   static constexpr int kI8Tab = 4 * (64 * kNT + 8) * 4;
-  // CUDA-core tables: q' [G][128] (q·Kᵀ); p'' [G][128] + group sums of p' [G][4] (p·V)
-  static constexpr int kCoreTab = PV ? 512 * G + 16 * G : 512 * G;
-  static constexpr int kTableBytes = ((kCoreTab > kI8Tab ? kCoreTab : kI8Tab) + 15) / 16 * 16;
+  static constexpr int kTableBytes = (kI8Tab + 15) / 16 * 16;
   static constexpr int kSumBytes = PV ? 512 * G : 0;          // p·V: [G][128] channel sums
   static constexpr int kFixed = kTableBytes + kSumBytes;
   static constexpr int kStages0 = (kWarpSmemBudget - kFixed - 64) / kStageBytes;
@@ -117,32 +115,118 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Position in the flat item list: (sequence*kv_heads + head, item within it).
+// The flat item list of a launch: for every (sequence, head) its packed blocks and then,
+// if it has one, its tail.  Uniform batches (NoPlan): every sequence has a.n_blocks
+// blocks and a.tail_len tail tokens.  Ragged batches: the RaggedPlan passed with the
+// launch gives each sequence's first item and tail length.
+struct NoPlan {};
+
 struct Cursor {
-  long bh;
-  int j;
-  __device__ void next(int items_per_bh) {
-    if (++j == items_per_bh) {
-      j = 0;
-      ++bh;
-    }
-  }
+  long bh;  // sequence * kv_heads + head
+  int j;    // item within the (sequence, head)
+  int n;    // items of the (sequence, head)
+  int nb;   // packed blocks of the sequence (item j < nb is block j, item nb the tail)
+  int tl;   // tail tokens of the sequence
 };
+
+template <class A>
+__device__ __forceinline__ Cursor cursor_at(const A& a, const NoPlan&, long x) {
+  Cursor c;
+  c.n = a.items_per_bh;
+  c.nb = a.n_blocks;
+  c.tl = a.tail_len;
+  c.bh = x / c.n;
+  c.j = (int)(x % c.n);
+  return c;
+}
+
+template <class A>
+__device__ __forceinline__ Cursor cursor_at(const A& a, const RaggedPlan& p, long x) {
+  int lo = 0, hi = a.batch;  // the last sequence whose first item is <= x has items
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.base[mid] <= x) lo = mid; else hi = mid;
+  }
+  Cursor c;
+  c.n = (p.base[lo + 1] - p.base[lo]) / a.kv_heads;
+  c.tl = p.tail[lo];
+  c.nb = c.n - (c.tl > 0 ? 1 : 0);
+  const long r = x - p.base[lo];
+  c.bh = (long)lo * a.kv_heads + r / c.n;
+  c.j = (int)(r % c.n);
+  return c;
+}
+
+template <class A>
+__device__ __forceinline__ void cursor_next(const A& a, const NoPlan&, Cursor& c) {
+  if (++c.j == c.n) {
+    c.j = 0;
+    ++c.bh;
+  }
+}
+
+template <class A>
+__device__ __forceinline__ void cursor_next(const A& a, const RaggedPlan& p, Cursor& c) {
+  if (++c.j < c.n) return;
+  c.j = 0;
+  ++c.bh;
+  if (c.bh % a.kv_heads == 0) {  // the next sequence that has items
+    int b = (int)(c.bh / a.kv_heads);
+    while (b < a.batch && p.base[b + 1] == p.base[b]) ++b;
+    if (b < a.batch) {
+      c.n = (p.base[b + 1] - p.base[b]) / a.kv_heads;
+      c.tl = p.tail[b];
+      c.nb = c.n - (c.tl > 0 ? 1 : 0);
+    }
+    c.bh = (long)b * a.kv_heads;
+  }
+}
+
+// Items [first, first + n) of (sequence, head) row bh (n = 0: the row has none).
+template <class A>
+__device__ __forceinline__ void row_items(const A& a, const NoPlan&, long bh, long* first, long* n) {
+  *first = bh * a.items_per_bh;
+  *n = a.items_per_bh;
+}
+
+template <class A>
+__device__ __forceinline__ void row_items(const A& a, const RaggedPlan& p, long bh, long* first, long* n) {
+  const long b = bh / a.kv_heads, h = bh % a.kv_heads;
+  *n = (p.base[b + 1] - p.base[b]) / a.kv_heads;
+  *first = p.base[b] + h * *n;
+}
+
+// Index entry {offset16, length16} of block j of row bh: through the block table if the
+// cache has one (a physical block outside the index reads as an invalid entry).
+template <class A>
+__device__ __forceinline__ uint2 block_entry(const A& a, long bh, int j) {
+  size_t at;
+  if (a.block_table == nullptr) {
+    at = (size_t)bh * a.max_blocks + j;
+  } else {
+    const long b = bh / a.kv_heads, h = bh % a.kv_heads;
+    const int p = a.block_table[(size_t)b * a.max_blocks + j];
+    if (p < 0 || (long)p >= (long)a.batch * a.max_blocks) return make_uint2(0xFFFFFFFFu, 0u);
+    at = ((size_t)(p / a.max_blocks) * a.kv_heads + h) * a.max_blocks + p % a.max_blocks;
+  }
+  return *reinterpret_cast<const uint2*>(a.index + at * 2);
+}
 
 // Index entries {offset16, length16} of 32 consecutive items of a warp's range, one
 // per lane ({0, 0} for a tail item or past the range), loaded with one coalesced
-// load; any lane reads the entry of any item of the window by shuffle.
+// load (uniform batches without a block table); any lane reads the entry of any item of
+// the window by shuffle.
 struct EntryWindow {
   long base;  // first item of the window
   uint2 ent;  // entry of item base + lane
-  __device__ void load(const GemvArgs& a, long first, long hi, int lane) {
+  template <class A, class Plan>
+  __device__ void load(const A& a, const Plan& plan, long first, long hi, int lane) {
     base = first;
     ent = make_uint2(0u, 0u);
     const long item = first + lane;
     if (item < hi) {
-      const long bh = item / a.items_per_bh;
-      const int j = (int)(item % a.items_per_bh);
-      if (j < a.n_blocks) ent = *reinterpret_cast<const uint2*>(a.index + ((size_t)bh * a.max_blocks + j) * 2);
+      const Cursor c = cursor_at(a, plan, item);
+      if (c.j < c.nb) ent = block_entry(a, c.bh, c.j);
     }
   }
   // Whole warp; base <= item < base + 32.
@@ -152,16 +236,17 @@ struct EntryWindow {
   }
 };
 
-// Issue the copies of item (bh, j) with index entry e into stage s of m (whole warp
-// participates); m provides stage(s), bar(s) and kind(s).
+// Issue the copies of item c with index entry e into stage s of m (whole warp
+// participates); m provides stage(s), bar(s) and kind(s).  The kind slot gets the item
+// kind in bits 0..7 and the record's length in 16-byte units above.
 template <int BITS, int G, bool PV, class Mem>
-__device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Cursor c, uint2 e, int s, int lane) {
+__device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, const Cursor& c, uint2 e, int s,
+                                           int lane) {
   using C = Cfg<BITS, G, PV>;
-  const int j = c.j;
   int kind = kKindTail;
   uint64_t off16 = 0;
   uint32_t len16 = 0;
-  if (j < a.n_blocks) {
+  if (c.j < c.nb) {
     off16 = e.x;
     len16 = e.y;
     const bool valid = e.x != 0xFFFFFFFFu && len16 >= 1040 / 16 && len16 * 16u <= (uint32_t)C::kRecBytes &&
@@ -171,7 +256,7 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, Curs
   unsigned char* st = m.stage(s);
   const unsigned char* src = a.arena + off16 * 16;
   if (lane == 0) {
-    *m.kind(s) = kind;
+    *m.kind(s) = kind | (int)(len16 << 8);  // kind in bits 0..7, record length (16-B units) above
     uint32_t bytes = 0;
     if (kind == kKindRaw) bytes = C::kRecBytes;
     if (kind == kKindPacked) bytes = len16 * 16u;
@@ -579,86 +664,287 @@ __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* t
 }
 
 // ----------------------------------------------------------------------------
-// q·Kᵀ on the CUDA cores (compressed records)
+// Compressed records on the 8-bit integer tensor cores
 // ----------------------------------------------------------------------------
-// Exact float of an unsigned integer u < 2^23: u in the mantissa of 2^23, minus 2^23
-// (two full-rate instructions instead of an integer-to-float conversion).
+// A compressed unit (pack group g, channel c) holds the 32 offsets of its slots in w
+// words: power-of-two slices of 4, 2 and 1 bits (packed-cache format v1, section 3).
+// A tensor-core A register takes four codes, so lanes must decode units with the same
+// instructions: the units of a group are sorted by width (classes 4, 3, 2, 1; a unit of
+// width 0 carries only its base and is left out), each class padded with dummy units to
+// a multiple of 16, and every run of 16 sorted units then has one width.
+//  * q·Kᵀ: a run is one k half (16 channels) of an m16n8k32 product.  Lane (g8, t) takes
+//    the channels at run positions 4t..4t+3 and slots 4g8..4g8+3 of the group (rows g8 and
+//    g8 + 8 of the group's two 16-slot tiles), joins the four units' slot runs with byte
+//    permutes and separates the codes with masks.  The B operand (q' digits, in natural
+//    channel order in the table of build_i8tab) is gathered through the sort.
+//  * p·V: a run is one 16-row tile (rows = channels, k = the group's 32 slots).  Lane t
+//    decodes 8 slots of two units with shifts and masks.  The rows change from group to
+//    group, so a group's tile results are added into the warp's channel sums.
+// The sorted descriptors (word start | tag << 16) live in the stage: the prologue reads
+// the record's meta into registers, after which bytes [0, 1040) of the stage (header,
+// params, meta) are free.  Words [1024, 1040) are zeroed; a dummy unit starts there
+// (word index -4 of the word area), so it decodes to zero codes.
+constexpr int kZeroUnitStart = -4;
+
+// Reads and checks a staged compressed record: widths <= BITS, total_words = the sum of
+// the widths, and a record length that matches it (so that every word a unit of the
+// record can name lies inside the staged bytes).  m4[g] = the meta bytes of this lane's
+// channels 4*lane .. 4*lane + 3 in group g.  Whole warp; returns the same verdict to all.
+template <int BITS>
+__device__ __forceinline__ bool packed_prologue(unsigned char* st, uint32_t len, uint32_t (&m4)[4], int lane) {
+  const uint32_t* meta = reinterpret_cast<const uint32_t*>(st + kMetaOffset);
+  uint32_t wsum = 0u, bad = 0u;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    m4[g] = meta[g * 32 + lane];
+    const uint32_t w = (m4[g] >> 4) & 0x0F0F0F0Fu;
+    wsum = __dp4a(w, 0x01010101u, wsum);
+    bad |= (w + (0x7Fu - BITS) * 0x01010101u) & 0x80808080u;  // a width above BITS sets bit 7
+  }
+  int tot = (int)wsum;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  const uint32_t total_words = reinterpret_cast<const uint32_t*>(st)[3];
+  const bool ok = !__any_sync(0xffffffffu, bad != 0u) && (uint32_t)tot == total_words &&
+                  ((1040u + 4u * (uint32_t)tot + 15u) & ~15u) == len;
+  __syncwarp();  // every lane has read the header and meta: [0, 1040) may be overwritten
+  if (lane < 4) reinterpret_cast<uint32_t*>(st + 1024)[lane] = 0u;
+  return ok;
+}
+
+// Run positions of one group after the sort: nblk runs of 16, classes 4, 3, 2 end
+// (padded) at end4, end3, end2 and class 1 fills the rest.
+struct SortedGroup {
+  int nblk, end4, end3, end2;
+  __device__ int width(int blk) const {
+    const int p = 16 * blk;
+    return p < end4 ? 4 : (p < end3 ? 3 : (p < end2 ? 2 : 1));
+  }
+};
+
+// Sorts the units of one group by width into desc[] (whole warp).  m4: this lane's meta
+// bytes (channels 4*lane + i); wbase: word index where the group starts (advanced by the
+// group's words); tag(c): the descriptor's high half for channel c.  Counting sort: a
+// packed per-class count (byte 4 - w for width w) is scanned over the warp together with
+// the widths (word starts in channel order).
+template <class Tag>
+__device__ __forceinline__ SortedGroup sort_group(uint32_t m4, int& wbase, uint32_t* desc, uint32_t dummy, Tag tag,
+                                                  int lane) {
+  uint32_t w[4];
+  int ls = 0;
+  uint32_t cnt = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    w[i] = (m4 >> (8 * i + 4)) & 15u;
+    ls += (int)w[i];
+    cnt += w[i] ? 1u << (32u - 8u * w[i]) : 0u;
+  }
+  int incl = ls;
+  uint32_t cincl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    const uint32_t cy = __shfl_up_sync(0xffffffffu, cincl, o);
+    if (lane >= o) {
+      incl += y;
+      cincl += cy;
+    }
+  }
+  const int gtot = __shfl_sync(0xffffffffu, incl, 31);
+  const uint32_t ctot = __shfl_sync(0xffffffffu, cincl, 31);
+  int s = wbase + incl - ls;
+  wbase += gtot;
+  const uint32_t n0 = ctot & 255u, n1 = (ctot >> 8) & 255u, n2 = (ctot >> 16) & 255u, n3 = ctot >> 24;
+  const uint32_t p0 = (n0 + 15u) & ~15u, p1 = (n1 + 15u) & ~15u, p2 = (n2 + 15u) & ~15u, p3 = (n3 + 15u) & ~15u;
+  const uint32_t b1 = p0, b2 = b1 + p1, b3 = b2 + p2;
+  // per class byte: the position of this lane's next unit of that class (<= 187: no carries)
+  uint32_t at = ((b1 << 8) | (b2 << 16) | (b3 << 24)) + (cincl - cnt);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (w[i]) {
+      const uint32_t sh = 32u - 8u * w[i];
+      desc[(at >> sh) & 255u] = ((uint32_t)s & 0xFFFFu) | (tag(4 * lane + i) << 16);
+      at += 1u << sh;
+    }
+    s += (int)w[i];
+  }
+  // dummies fill each class up to its padded size
+  if ((uint32_t)lane < p0 - n0) desc[n0 + lane] = dummy;
+  if ((uint32_t)lane < p1 - n1) desc[b1 + n1 + lane] = dummy;
+  if ((uint32_t)lane < p2 - n2) desc[b2 + n2 + lane] = dummy;
+  if ((uint32_t)lane < p3 - n3) desc[b3 + n3 + lane] = dummy;
+  SortedGroup r;
+  r.nblk = (int)((b3 + p3) >> 4);
+  r.end4 = (int)b1;
+  r.end3 = (int)b2;
+  r.end2 = (int)b3;
+  return r;
+}
+
+__device__ __forceinline__ int desc_start(uint32_t d) { return (int)(int16_t)(d & 0xFFFFu); }
+
+// Exact float of a small unsigned integer (< 2^23): it goes into the mantissa of 2^23.
 __device__ __forceinline__ float small_u2f(uint32_t u) { return __uint_as_float(u | 0x4B000000u) - 8388608.f; }
 
-// Extracts the offset of token j from a compressed unit of width w starting at word s.
-__device__ __forceinline__ uint32_t unit_field(const uint32_t* W, int s, int w, int j) {
-  uint32_t u = 0;
-  if (w == 4) {
-    u = (W[s + (j >> 3)] >> ((j & 7) * 4)) & 15u;
-  } else if (w >= 2) {
-    u = (W[s + (j >> 4)] >> ((j & 15) * 2)) & 3u;
-    if (w == 3) u |= ((W[s + 2] >> j) & 1u) << 2;
-  } else if (w == 1) {
-    u = (W[s] >> j) & 1u;
+// q·Kᵀ: A registers of one 16-unit run of width W for lane (g8, t): R[i] = the codes of
+// slot 4*g8 + i of the four units d (run positions 4t .. 4t+3), one byte per unit.
+template <int W>
+__device__ __forceinline__ void qk_run(const uint32_t* words, const uint4 d, int g8, uint32_t (&R)[4]) {
+  const int s0 = desc_start(d.x), s1 = desc_start(d.y), s2 = desc_start(d.z), s3 = desc_start(d.w);
+  if constexpr (W == 4) {
+    // slots 4*g8 .. +3: the 16-bit half g8 & 1 of word g8 >> 1 (a nibble per slot)
+    const int o = g8 >> 1;
+    const uint32_t sel = (g8 & 1) ? 0x7632u : 0x5410u;
+    const uint32_t y01 = __byte_perm(words[s0 + o], words[s1 + o], sel);
+    const uint32_t y23 = __byte_perm(words[s2 + o], words[s3 + o], sel);
+    const uint32_t p0 = __byte_perm(y01, y23, 0x6420u), p1 = __byte_perm(y01, y23, 0x7531u);
+    R[0] = p0 & 0x0F0F0F0Fu;
+    R[1] = (p0 >> 4) & 0x0F0F0F0Fu;
+    R[2] = p1 & 0x0F0F0F0Fu;
+    R[3] = (p1 >> 4) & 0x0F0F0F0Fu;
+  } else {
+    // 2-bit slice: byte g8 & 3 of word g8 >> 1 ... >> 2; 1-bit slice: nibble g8 & 1 of byte g8 >> 1
+    uint32_t p2 = 0u, p1 = 0u;
+    if constexpr (W == 2 || W == 3) {
+      const int o = g8 >> 2;
+      const uint32_t b = (uint32_t)(g8 & 3), sel = b | ((b + 4u) << 4);
+      const uint32_t y01 = __byte_perm(words[s0 + o], words[s1 + o], sel);
+      const uint32_t y23 = __byte_perm(words[s2 + o], words[s3 + o], sel);
+      p2 = __byte_perm(y01, y23, 0x5410u);
+    }
+    if constexpr (W == 1 || W == 3) {
+      const int o = W == 3 ? 2 : 0;
+      const uint32_t b = (uint32_t)(g8 >> 1), sel = b | ((b + 4u) << 4);
+      const uint32_t y01 = __byte_perm(words[s0 + o], words[s1 + o], sel);
+      const uint32_t y23 = __byte_perm(words[s2 + o], words[s3 + o], sel);
+      p1 = __byte_perm(y01, y23, 0x5410u) >> (4 * (g8 & 1));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t r = 0u;
+      if constexpr (W == 2 || W == 3) r = (p2 >> (2 * i)) & 0x03030303u;
+      if constexpr (W == 1) r = (p1 >> i) & 0x01010101u;
+      if constexpr (W == 3) r |= ((p1 >> i) & 0x01010101u) << 2;
+      R[i] = r;
+    }
   }
-  return u;
 }
 
-// One compressed K record, lane = token within each pack group.
-template <int G>
-__device__ __forceinline__ void qk_packed(const unsigned char* st, const float* qp, const float (&cst)[G],
-                                          float* sblk, long ld, float scale, int lane) {
-  const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
-  const uint8_t* meta = st + kMetaOffset;
-  const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
-#pragma unroll 1
-  for (int g = 0; g < 4; ++g) {
-    // base term of this group: sum_c q'_c base_gc, lane covers channels 4*lane..4*lane+3
-    float bsum[G];
-    const uint32_t m4 = *reinterpret_cast<const uint32_t*>(meta + g * 128 + 4 * lane);
+// Byte `off` past each of the four units' B-table bases (the descriptors' high halves),
+// packed in order.
+__device__ __forceinline__ uint32_t gather4(const uint8_t* t8, const uint4 d, int off) {
+  const uint32_t x0 = t8[(d.x >> 16) + off], x1 = t8[(d.y >> 16) + off];
+  const uint32_t x2 = t8[(d.z >> 16) + off], x3 = t8[(d.w >> 16) + off];
+  return __byte_perm(__byte_perm(x0, x1, 0x0040u), __byte_perm(x2, x3, 0x0040u), 0x5410u);
+}
+
+// q·Kᵀ of one compressed K record on the tensor cores.  tab: the int8 B table of q'
+// (build_i8tab, natural channel order); qv: this lane's q' = q * scale_c for channels
+// 4*lane .. +3; cst: sum_c q_c mn_c per head.  Writes the 128 scores of every head:
+// scale * (cst + sum_c q'_c base_gc + sum_c q'_c offset).
+// Returns false (nothing written) if the record fails the prologue's checks.
+template <int BITS, int G>
+__device__ __forceinline__ bool qk_packed_tc(unsigned char* st, uint32_t len, const uint32_t* tab,
+                                             const float (&qv)[G][4], const float (&cst)[G], const float (&invf)[G],
+                                             float* sblk, long ld, float scale, int lane) {
+  using L = I8Layout<G>;
+  constexpr int NT = L::kNT;
+  uint32_t m4[4];
+  if (!packed_prologue<BITS>(st, len, m4, lane)) return false;
+  const int g8 = lane >> 2, t = lane & 3;
+  uint32_t* desc = reinterpret_cast<uint32_t*>(st);
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
+  const uint8_t* t8 = reinterpret_cast<const uint8_t*>(tab);
+  // byte of channel c's B digits in the table (column n adds 4 * (8 NT (n & 7) + (n >> 3)))
+  auto tag = [](int c) -> uint32_t {
+    return 4u * (uint32_t)((c >> 5) * (64 * NT + 8) + ((c >> 2) & 3) * 2 * NT + ((c >> 4) & 1) * NT) + (uint32_t)(c & 3);
+  };
+  const uint32_t dummy = (uint32_t)kZeroUnitStart & 0xFFFFu;
+  // base terms of the four groups, sum_c q'_c base_gc, kept in the free stage bytes
+  // [768, 1024) (qv is then dead, which keeps the register count of the raw path)
+  float* bsm = reinterpret_cast<float*>(st + 768);
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
-      const float4 q4 = *reinterpret_cast<const float4*>(qp + hd * 128 + 4 * lane);
-      float part = q4.x * small_u2f(m4 & 15u);
-      part = fmaf(q4.y, small_u2f((m4 >> 8) & 15u), part);
-      part = fmaf(q4.z, small_u2f((m4 >> 16) & 15u), part);
-      part = fmaf(q4.w, small_u2f((m4 >> 24) & 15u), part);
-      bsum[hd] = warp_sum(part);
+      float part = qv[hd][0] * small_u2f(m4[g] & 15u);
+      part = fmaf(qv[hd][1], small_u2f((m4[g] >> 8) & 15u), part);
+      part = fmaf(qv[hd][2], small_u2f((m4[g] >> 16) & 15u), part);
+      part = fmaf(qv[hd][3], small_u2f((m4[g] >> 24) & 15u), part);
+      part = warp_sum(part);
+      if (lane == 0) bsm[g * G + hd] = part + cst[hd];
     }
-    float acc[G];
+  const PairW pw = pair_weights(t);
+  float sf[L::kNH];
 #pragma unroll
-    for (int hd = 0; hd < G; ++hd) acc[hd] = 0.f;
-    int s = gws[g];
+  for (int jh = 0; jh < L::kNH; ++jh) sf[jh] = scale * head_sel<G>(invf, L::head(jh, t));
+  int wbase = 0;
 #pragma unroll 1
-    for (int c4 = 0; c4 < 32; ++c4) {
-      const uint32_t mm = *reinterpret_cast<const uint32_t*>(meta + g * 128 + 4 * c4);
-      float q4[G][4];
+  for (int g = 0; g < 4; ++g) {
+    __syncwarp();  // the previous group's runs are decoded: desc may be rewritten
+    const SortedGroup sg = sort_group(m4[g], wbase, desc, dummy, tag, lane);
+    float sc_[L::kNH];
 #pragma unroll
-      for (int hd = 0; hd < G; ++hd) {
-        const float4 v = *reinterpret_cast<const float4*>(qp + hd * 128 + 4 * c4);
-        q4[hd][0] = v.x;
-        q4[hd][1] = v.y;
-        q4[hd][2] = v.z;
-        q4[hd][3] = v.w;
+    for (int jh = 0; jh < L::kNH; ++jh) sc_[jh] = scale * bsm[g * G + L::head(jh, t)];
+    __syncwarp();  // desc of this group written
+    int acc[2][NT][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int j = 0; j < NT; ++j) acc[u][j][0] = acc[u][j][1] = acc[u][j][2] = acc[u][j][3] = kRoundBits;
+#pragma unroll 1
+    for (int blk0 = 0; blk0 < sg.nblk; blk0 += 2) {
+      uint32_t R[2][4], bf[2][NT];
+#pragma unroll
+      for (int kh = 0; kh < 2; ++kh) {
+        const int blk = blk0 + kh;
+        if (blk < sg.nblk) {
+          const uint4 d = *reinterpret_cast<const uint4*>(desc + 16 * blk + 4 * t);
+          switch (sg.width(blk)) {  // warp-uniform
+            case 4: qk_run<4>(words, d, g8, R[kh]); break;
+            case 3: qk_run<3>(words, d, g8, R[kh]); break;
+            case 2: qk_run<2>(words, d, g8, R[kh]); break;
+            default: qk_run<1>(words, d, g8, R[kh]); break;
+          }
+#pragma unroll
+          for (int j = 0; j < NT; ++j) bf[kh][j] = gather4(t8, d, 4 * (8 * NT * g8 + j));
+        } else {
+          R[kh][0] = R[kh][1] = R[kh][2] = R[kh][3] = 0u;
+#pragma unroll
+          for (int j = 0; j < NT; ++j) bf[kh][j] = 0u;
+        }
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int w = (mm >> (8 * i + 4)) & 15u;
-        const float u = small_u2f(unit_field(W, s, w, lane));
-        s += w;
+      for (int u = 0; u < 2; ++u) {  // the group's two tiles: rows g8 / g8 + 8 = slots 4 g8 + 2u / + 1
+        const uint32_t a[4] = {R[0][2 * u], R[0][2 * u + 1], R[1][2 * u], R[1][2 * u + 1]};
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) acc[hd] = fmaf(q4[hd][i], u, acc[hd]);
+        for (int j = 0; j < NT; ++j) imma16832(acc[u][j], a, bf[0][j], bf[1][j]);
       }
     }
 #pragma unroll
-    for (int hd = 0; hd < G; ++hd) sblk[hd * ld + 32 * g + lane] = scale * (cst[hd] + bsum[hd] + acc[hd]);
+    for (int u = 0; u < 2; ++u) {
+      auto emit = [&](int, int jh, float lo, float hi) {
+        if (L::owns(jh, t)) {
+          float* dst = sblk + L::head(jh, t) * ld + 32 * g + 4 * g8 + 2 * u;
+          *reinterpret_cast<float2*>(dst) = make_float2(fmaf(lo, sf[jh], sc_[jh]), fmaf(hi, sf[jh], sc_[jh]));
+        }
+      };
+      emit_tile<G>(u, acc[u], 1.f, 1.f, pw, emit);
+    }
   }
+  return true;
 }
 
+// The fp16 tail (tl tokens, after the sequence's nb blocks) of row bh: scaled scores.
 template <int G>
-__device__ __forceinline__ void qk_tail(const GemvArgs& a, long bh, const float (&qr)[G][4], float* srow0,
-                                        int lane) {
+__device__ __forceinline__ void qk_tail(const GemvArgs& a, long bh, int nb, int tl, const float (&qr)[G][4],
+                                        float* srow0, int lane) {
   const uint16_t* tail = a.tail + (size_t)bh * 128 * 128;
-  for (int t0 = 0; t0 < a.tail_len; t0 += 32) {
+  for (int t0 = 0; t0 < tl; t0 += 32) {
     float mine[G];
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) mine[hd] = 0.f;
-    const int tn = min(32, a.tail_len - t0);
+    const int tn = min(32, tl - t0);
     for (int t = 0; t < tn; ++t) {
       const uint2 hv = *reinterpret_cast<const uint2*>(tail + (size_t)(t0 + t) * 128 + 4 * lane);
       const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
@@ -675,90 +961,183 @@ __device__ __forceinline__ void qk_tail(const GemvArgs& a, long bh, const float 
     }
     if (lane < tn) {
 #pragma unroll
-      for (int hd = 0; hd < G; ++hd) srow0[hd * a.ld + (long)a.n_blocks * 128 + t0 + lane] = a.scale * mine[hd];
+      for (int hd = 0; hd < G; ++hd) srow0[hd * a.ld + (long)nb * 128 + t0 + lane] = a.scale * mine[hd];
     }
   }
 }
 
-// ----------------------------------------------------------------------------
-// p·V on the CUDA cores (compressed records)
-// ----------------------------------------------------------------------------
-// One compressed V record, lane = channel sl*32 + lane; adds into the warp's shared
-// [G][128] channel sums.  pg[hd*4 + g] = sum of p' over pack group g.
-template <int G>
-__device__ __forceinline__ void pv_packed(const unsigned char* st, const float* pp, const float* pg, float* sacc,
-                                          int lane) {
-  const uint16_t* gws = reinterpret_cast<const uint16_t*>(st);
-  const uint8_t* meta = st + kMetaOffset;
-  const uint32_t* W = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
-#pragma unroll 1
-  for (int g = 0; g < 4; ++g) {
-    int carry = gws[g];
-#pragma unroll 1
-    for (int sl = 0; sl < 4; ++sl) {
-      const int c = sl * 32 + lane;
-      const uint32_t mb = meta[g * 128 + c];
-      const int w = (int)(mb >> 4), base = (int)(mb & 15u);
-      int incl = w;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+// p·V: A registers (rows = two units, k = the group's 32 slots) of lane t from a unit
+// of width W starting at word s.  The k position (kh, t, e) of a register holds
+//   slot 8t + 2e + kh  (order A: one word per lane for the 4-bit slice), or
+//   slot t + 8e + 4kh  (order B: one shift and mask per register for 2- and 1-bit slices).
+// a[0] / a[1]: the kh = 0 / kh = 1 registers.
+template <int W, bool kOrderA>
+__device__ __forceinline__ void pv_unit(const uint32_t* words, int s, int t, uint32_t (&a)[2]) {
+  if constexpr (kOrderA) {
+    if constexpr (W == 4) {
+      const uint32_t x = words[s + t];  // slots 8t .. 8t+7, a nibble each
+      a[0] = x & 0x0F0F0F0Fu;
+      a[1] = (x >> 4) & 0x0F0F0F0Fu;
+    } else {
+      uint32_t r0 = 0u, r1 = 0u;
+      if constexpr (W == 2 || W == 3) {  // slots 8t .. 8t+7: bits 16(t & 1) .. +15 of word t >> 1
+        const uint32_t z = __byte_perm(words[s + (t >> 1)], 0u, (t & 1) ? 0x3322u : 0x1100u);
+        r0 = (z & 0x00030003u) | ((z >> 4) & 0x03000300u);
+        r1 = ((z >> 2) & 0x00030003u) | ((z >> 6) & 0x03000300u);
       }
-      const int start = carry + incl - w;
-      carry += __shfl_sync(0xffffffffu, incl, 31);
-      // this lane's unit (group g, channel c), eight tokens at a time: their offsets,
-      // then p' * offset for a block of HB heads (one head at a time from G = 4 on, which
-      // decodes the unit again per head but keeps the registers of the wider kernels)
-      constexpr int HB = G >= 4 ? 1 : G;
-      const int bit_word = start + ((w & 2) ? 2 : 0);  // the 1-bit slice follows the 2-bit one
-      const uint32_t bit_hi = (w & 2) ? 2u : 0u;       // and is bit 2 of a width-3 unit
-#pragma unroll 1
-      for (int h0 = 0; h0 < G; h0 += HB) {
-        float sum[HB];
-#pragma unroll
-        for (int h = 0; h < HB; ++h) sum[h] = (float)base * pg[(h0 + h) * 4 + g];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {  // tokens 8k .. 8k+7
-          float u[8];
-          if (w == 4) {
-            const uint32_t word = W[start + k];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = small_u2f((word >> (4 * i)) & 15u);
-          } else {
-            uint32_t two = 0u, one = 0u;
-            if (w & 2) two = W[start + (k >> 1)] >> (16 * (k & 1));
-            if (w & 1) one = W[bit_word] >> (8 * k);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) u[i] = small_u2f(((two >> (2 * i)) & 3u) | (((one >> i) & 1u) << bit_hi));
-          }
-#pragma unroll
-          for (int h = 0; h < HB; ++h) {
-            const float4* pr4 = reinterpret_cast<const float4*>(pp + (h0 + h) * 128 + 32 * g + 8 * k);
-            const float4 pa = pr4[0], pb = pr4[1];
-            float t = sum[h];
-            t = fmaf(pa.x, u[0], t);
-            t = fmaf(pa.y, u[1], t);
-            t = fmaf(pa.z, u[2], t);
-            t = fmaf(pa.w, u[3], t);
-            t = fmaf(pb.x, u[4], t);
-            t = fmaf(pb.y, u[5], t);
-            t = fmaf(pb.z, u[6], t);
-            t = fmaf(pb.w, u[7], t);
-            sum[h] = t;
-          }
-        }
-#pragma unroll
-        for (int h = 0; h < HB; ++h) sacc[(h0 + h) * 128 + c] += sum[h];
+      if constexpr (W == 1 || W == 3) {  // slots 8t .. 8t+7: byte t; bit 2e -> byte e by one multiply
+        const uint32_t x = words[s + (W == 3 ? 2 : 0)] >> (8 * t);
+        const uint32_t b0 = ((x & 0x55u) * 0x41041u) & 0x01010101u;
+        const uint32_t b1 = (((x >> 1) & 0x55u) * 0x41041u) & 0x01010101u;
+        r0 |= W == 3 ? b0 << 2 : b0;
+        r1 |= W == 3 ? b1 << 2 : b1;
       }
+      a[0] = r0;
+      a[1] = r1;
+    }
+  } else {
+    static_assert(W != 4, "order B serves widths 1 to 3");
+    uint32_t r0 = 0u, r1 = 0u;
+    if constexpr (W == 2 || W == 3) {  // slot t + 8e + 4kh: byte 2(e & 1) + kh of word e >> 1, bits 2t
+      const uint32_t w0 = words[s], w1 = words[s + 1];
+      r0 = (__byte_perm(w0, w1, 0x6420u) >> (2 * t)) & 0x03030303u;
+      r1 = (__byte_perm(w0, w1, 0x7531u) >> (2 * t)) & 0x03030303u;
+    }
+    if constexpr (W == 1 || W == 3) {  // bit t + 8e + 4kh
+      const uint32_t x = words[s + (W == 3 ? 2 : 0)] >> t;
+      const uint32_t b0 = x & 0x01010101u, b1 = (x >> 4) & 0x01010101u;
+      r0 |= W == 3 ? b0 << 2 : b0;
+      r1 |= W == 3 ? b1 << 2 : b1;
+    }
+    a[0] = r0;
+    a[1] = r1;
+  }
+}
+
+// B fragments of group g in the two k orders of pv_unit, gathered from the int8 B table
+// of p' (build_i8tab, natural slot order: byte k & 3 of word i8tab_word(k >> 5,
+// (k >> 4) & 1, (k >> 2) & 3, n) holds slot k).  bA/bB[kh][j] for n-tile j.
+template <int NT>
+__device__ __forceinline__ void pv_group_frags(const uint32_t* tab, int g, int lane, uint32_t (&bA)[2][NT],
+                                               uint32_t (&bB)[2][NT]) {
+  const int g8 = lane >> 2, t = lane & 3;
+  const uint8_t* t8 = reinterpret_cast<const uint8_t*>(tab);
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    const int n = 8 * j + g8;
+    // order A: slot 8t + 2e + kh = natural (kh' = t >> 1, t' = 2(t & 1) + (e >> 1), e' = 2(e & 1) + kh)
+    const uint32_t w0 = tab[i8tab_word<NT>(g, t >> 1, 2 * (t & 1), n)];
+    const uint32_t w1 = tab[i8tab_word<NT>(g, t >> 1, 2 * (t & 1) + 1, n)];
+    bA[0][j] = __byte_perm(w0, w1, 0x6420u);
+    bA[1][j] = __byte_perm(w0, w1, 0x7531u);
+    // order B: slot t + 8e + 4kh = natural (kh' = e >> 1, t' = 2(e & 1) + kh, e' = t)
+#pragma unroll
+    for (int kh = 0; kh < 2; ++kh) {
+      const uint32_t x0 = t8[4 * i8tab_word<NT>(g, 0, kh, n) + t], x1 = t8[4 * i8tab_word<NT>(g, 0, 2 + kh, n) + t];
+      const uint32_t x2 = t8[4 * i8tab_word<NT>(g, 1, kh, n) + t], x3 = t8[4 * i8tab_word<NT>(g, 1, 2 + kh, n) + t];
+      bB[kh][j] = __byte_perm(__byte_perm(x0, x1, 0x0040u), __byte_perm(x2, x3, 0x0040u), 0x5410u);
     }
   }
+}
+
+// One 16-unit run of width W as a p·V tile: rows g8 / g8 + 8 = the units at run positions
+// g8 / g8 + 8; adds each row's products, digits joined and times invf, into sacc (the
+// warp's [G][128] channel sums).
+template <int W, int G>
+__device__ __forceinline__ void pv_run(const uint32_t* words, const uint32_t* desc, int blk,
+                                       const uint32_t (&bA)[2][I8Layout<G>::kNT],
+                                       const uint32_t (&bB)[2][I8Layout<G>::kNT], const float (&f_t)[I8Layout<G>::kNH],
+                                       const PairW& pw, float* sacc, int lane) {
+  using L = I8Layout<G>;
+  constexpr int NT = L::kNT;
+  constexpr bool kA = W == 4;
+  const int g8 = lane >> 2, t = lane & 3;
+  const uint32_t dlo = desc[16 * blk + g8], dhi = desc[16 * blk + 8 + g8];
+  uint32_t alo[2], ahi[2];
+  pv_unit<W, kA>(words, desc_start(dlo), t, alo);
+  pv_unit<W, kA>(words, desc_start(dhi), t, ahi);
+  const uint32_t a[4] = {alo[0], ahi[0], alo[1], ahi[1]};
+  int d[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) {
+    d[j][0] = d[j][1] = d[j][2] = d[j][3] = kRoundBits;
+    imma16832(d[j], a, kA ? bA[0][j] : bB[0][j], kA ? bA[1][j] : bB[1][j]);
+  }
+  const uint32_t clo = dlo >> 16, chi = dhi >> 16;  // channels (0xFFFF: dummy)
+  auto emit = [&](int, int jh, float lo, float hi) {
+    if (L::owns(jh, t)) {
+      float* row = sacc + L::head(jh, t) * 128;
+      if (clo < 128u) row[clo] = fmaf(lo, f_t[jh], row[clo]);
+      if (chi < 128u) row[chi] = fmaf(hi, f_t[jh], row[chi]);
+    }
+  };
+  emit_tile<G>(0, d, 1.f, 1.f, pw, emit);
+}
+
+// p·V of one compressed V record on the tensor cores.  tab: the int8 B table of p'
+// (build_i8tab, natural slot order); pv4: this lane's p' = p * scale_r for slots
+// 4*lane .. +3; invf: per head.  Adds sum_r p'_r code[r][c] into sacc.  Returns false
+// (nothing added) if the record fails the prologue's checks.
+template <int BITS, int G>
+__device__ __forceinline__ bool pv_packed_tc(unsigned char* st, uint32_t len, const uint32_t* tab,
+                                             const float (&pv4)[G][4], const float (&invf)[G], float* sacc, int lane) {
+  using L = I8Layout<G>;
+  constexpr int NT = L::kNT;
+  uint32_t m4[4];
+  if (!packed_prologue<BITS>(st, len, m4, lane)) return false;
+  const int t = lane & 3;
+  uint32_t* desc = reinterpret_cast<uint32_t*>(st);
+  const uint32_t* words = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
+  const uint32_t dummy = ((uint32_t)kZeroUnitStart & 0xFFFFu) | 0xFFFF0000u;
+  const PairW pw = pair_weights(t);
+  float f_t[L::kNH];
+#pragma unroll
+  for (int jh = 0; jh < L::kNH; ++jh) f_t[jh] = head_sel<G>(invf, L::head(jh, t));
+  // base terms first: channel c gets sum_g base_gc * (sum of p' over group g); lanes
+  // 8g .. 8g+7 hold group g.  (Every later addition into sacc commutes with these.)
+#pragma unroll
+  for (int hd = 0; hd < G; ++hd) {
+    float ps = (pv4[hd][0] + pv4[hd][1]) + (pv4[hd][2] + pv4[hd][3]);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+    float bacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const float pg = __shfl_sync(0xffffffffu, ps, 8 * g);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bacc[i] = fmaf(small_u2f((m4[g] >> (8 * i)) & 15u), pg, bacc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sacc[hd * 128 + 4 * lane + i] += bacc[i];
+  }
+  int wbase = 0;
+#pragma unroll 1
+  for (int g = 0; g < 4; ++g) {
+    __syncwarp();  // the previous group's runs are done: desc may be rewritten
+    const SortedGroup sg = sort_group(m4[g], wbase, desc, dummy, [](int c) { return (uint32_t)c; }, lane);
+    uint32_t bA[2][NT], bB[2][NT];
+    pv_group_frags<NT>(tab, g, lane, bA, bB);
+    __syncwarp();  // desc of this group written
+#pragma unroll 1
+    for (int blk = 0; blk < sg.nblk; ++blk) {
+      switch (sg.width(blk)) {  // warp-uniform
+        case 4: pv_run<4, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
+        case 3: pv_run<3, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
+        case 2: pv_run<2, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
+        default: pv_run<1, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
+      }
+      __syncwarp();  // a run's sums are added before the next run (rows of one group differ, but
+                     // a lane adds rows it does not own across runs only through sacc)
+    }
+  }
+  return true;
 }
 
 // The fp16 tail of one (sequence, head), lane = channel sl*32 + lane; adds into the
 // warp's shared [G][128] channel sums.
 template <int G>
-__device__ __forceinline__ void pv_tail(const GemvArgs& a, long bh, float* sacc, int lane) {
+__device__ __forceinline__ void pv_tail(const GemvArgs& a, long bh, int nb, int tl, float* sacc, int lane) {
   const long b = bh / a.kv_heads, h = bh % a.kv_heads;
   const uint16_t* tail = a.tail + (size_t)bh * 128 * 128;
   float acc[4][G];
@@ -766,13 +1145,13 @@ __device__ __forceinline__ void pv_tail(const GemvArgs& a, long bh, float* sacc,
   for (int sl = 0; sl < 4; ++sl)
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) acc[sl][hd] = 0.f;
-  for (int t = 0; t < a.tail_len; ++t) {
+  for (int t = 0; t < tl; ++t) {
     float vv[4];
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
-      const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)a.n_blocks * 128 + t];
+      const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)nb * 128 + t];
 #pragma unroll
       for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = fmaf(pt, vv[sl], acc[sl][hd]);
     }

@@ -24,6 +24,8 @@
 // The encoder runs once per 128 tokens per head; it is not on the per-token path.
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -70,9 +72,44 @@ static_assert(sizeof(EncodeSmem) <= 113 * 1024, "two encoder CTAs per SM");
 
 __device__ __forceinline__ int bitlen(uint32_t x) { return x == 0 ? 0 : 32 - __clz(x); }
 
-__device__ __forceinline__ unsigned long long* entry64(uint32_t* index, const EncodeArgs& a, long blk_in_call) {
-  const long bh = blk_in_call / a.nb, i = blk_in_call % a.nb;
-  return reinterpret_cast<unsigned long long*>(index + ((size_t)bh * a.max_blocks + a.n_old + i) * 2);
+// Where block t of the call goes: the index entry (u32 pair index) of its (sequence,
+// head, logical block) -- through the block table if the cache has one -- and the row of
+// the input it is read from.  Uniform calls cover every sequence; ragged calls the
+// plan's sequences, each from its own first logical block.
+struct CallBlock {
+  size_t entry;  // u32 pair index into the index table
+  size_t row;    // input row: ((sequence * heads + head) * nb + i)
+};
+
+template <class Plan>
+__device__ __forceinline__ CallBlock call_block(const EncodeArgs& a, const Plan& plan, long t) {
+  const long i = t % a.nb, sh = t / a.nb;  // sh = (sequence of the call) * heads + head
+  const long h = sh % a.heads;
+  long b, j;
+  if constexpr (std::is_same<Plan, RaggedEncodePlan>::value) {
+    const long sidx = sh / a.heads;
+    b = plan.seq[sidx];
+    j = plan.first_block[sidx] + i;
+  } else {
+    b = sh / a.heads;
+    j = a.n_old + i;
+  }
+  long rb = b, jb = j;
+  if (a.block_table != nullptr) {
+    const int p = a.block_table[(size_t)b * a.max_blocks + j];
+    rb = p / a.max_blocks;
+    jb = p % a.max_blocks;
+  }
+  CallBlock c;
+  c.entry = ((size_t)rb * a.heads + h) * a.max_blocks + jb;
+  c.row = ((size_t)b * a.heads + h) * a.nb + i;
+  return c;
+}
+
+template <class Plan>
+__device__ __forceinline__ unsigned long long* entry64(uint32_t* index, const EncodeArgs& a, const Plan& plan,
+                                                       long blk_in_call) {
+  return reinterpret_cast<unsigned long long*>(index + call_block(a, plan, blk_in_call).entry * 2);
 }
 
 __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
@@ -88,7 +125,8 @@ __device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long lon
 // aggregates and moves down.  A window waits while any entry above its nearest
 // final entry is unpublished.  Returns false (and sets PACKKV_DEV_TIMEOUT) if a
 // predecessor did not publish within about a second.
-__device__ bool look_back(uint32_t* index, const EncodeArgs& a, long t, unsigned long long end0,
+template <class Plan>
+__device__ bool look_back(uint32_t* index, const EncodeArgs& a, const Plan& plan, long t, unsigned long long end0,
                           unsigned long long* excl, int lane) {
   unsigned long long sum = 0;
   long p = t - 1;  // top of the current window
@@ -97,7 +135,7 @@ __device__ bool look_back(uint32_t* index, const EncodeArgs& a, long t, unsigned
   while (p >= 0) {
     const long mine = p - lane;
     unsigned long long e = 0;
-    if (mine >= 0) e = ld_relaxed(entry64(index, a, mine));
+    if (mine >= 0) e = ld_relaxed(entry64(index, a, plan, mine));
     const uint32_t y = (uint32_t)(e >> 32);
     const bool unpublished = mine >= 0 && y == 0u;
     const bool fin = mine >= 0 && y != 0u && !(y & kFlagAggregate);
@@ -128,7 +166,8 @@ __device__ bool look_back(uint32_t* index, const EncodeArgs& a, long t, unsigned
   return true;
 }
 
-__global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
+template <class Plan>
+__global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs a, const __grid_constant__ Plan plan) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   EncodeSmem& s = *reinterpret_cast<EncodeSmem*>(smem_raw);
   const int tid = threadIdx.x;
@@ -147,10 +186,9 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
   }
   __syncthreads();
   const long t_call = s.ticket;                 // block index within the call
-  const int blk = (int)(t_call % a.nb);
-  const long bh = t_call / a.nb;                // b * heads + h
-  const size_t in_base = ((size_t)bh * a.nb + blk) * kBlockTokens * kHeadDim;
-  const size_t slot = (size_t)bh * a.max_blocks + a.n_old + blk;
+  const CallBlock where = call_block(a, plan, t_call);
+  const size_t in_base = where.row * kBlockTokens * kHeadDim;
+  const size_t slot = where.entry;  // the block's index entry (and its row of perm)
   if (tid == 0) {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     mbar_arrive_expect_tx(&s.bar, 2u * kBlockTokens * kHeadDim * 2u);
@@ -338,7 +376,7 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
     uint32_t* index = tensor ? a.v_index : a.k_index;
     const unsigned long long agg =
         (unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) | ((unsigned long long)kFlagAggregate << 32);
-    atomicExch(entry64(index, a, t_call), agg);
+    atomicExch(entry64(index, a, plan, t_call), agg);
   }
 
   // ---- unit word offsets ------------------------------------------------------
@@ -483,14 +521,14 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
     uint32_t* index = tensor ? a.v_index : a.k_index;
     const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
     unsigned long long excl = 0;
-    const bool ok = look_back(index, a, t_call, end0, &excl, lane);
+    const bool ok = look_back(index, a, plan, t_call, end0, &excl, lane);
     if (lane == 0) {
       if (!ok) s.failed = 1;
       s.prefix[tensor] = excl;
       // final entry {offset16, length16}; a failed call is invalidated by the last CTA
       const unsigned long long fin = (unsigned long long)(uint32_t)(end0 + excl) |
                                      ((unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) << 32);
-      atomicExch(entry64(index, a, t_call), fin);
+      atomicExch(entry64(index, a, plan, t_call), fin);
     }
   }
   __syncthreads();
@@ -529,15 +567,15 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(EncodeArgs a) {
   if (!s.last) return;
   if (s.failed) {
     for (long e = tid; e < n_call; e += blockDim.x) {
-      *entry64(a.k_index, a, e) = 0xFFFFFFFFull;  // {offset 0xFFFFFFFF, length 0}
-      *entry64(a.v_index, a, e) = 0xFFFFFFFFull;
+      *entry64(a.k_index, a, plan, e) = 0xFFFFFFFFull;  // {offset 0xFFFFFFFF, length 0}
+      *entry64(a.v_index, a, plan, e) = 0xFFFFFFFFull;
     }
     if (tid == 0) set_status(a.ctrl, PACKKV_DEV_CAPACITY);
   } else if (tid == 0 || tid == 32) {
     // prefix through the last block of the call = its final entry's offset - end + length
     const int tensor = tid >> 5;
     uint32_t* index = tensor ? a.v_index : a.k_index;
-    const unsigned long long e = atomicAdd(entry64(index, a, n_call - 1), 0ull);
+    const unsigned long long e = atomicAdd(entry64(index, a, plan, n_call - 1), 0ull);
     const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
     const unsigned long long total = (unsigned long long)(uint32_t)e - end0 + (uint32_t)(e >> 32);
     a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd] = end0 + total;
@@ -561,36 +599,87 @@ __global__ void append_tail_kernel(const uint16_t* __restrict__ k, const uint16_
   dst[ch] = src[ch];
 }
 
+// As append_tail_kernel, with each sequence's own position (plan.pos[b]; none if < 0).
+__global__ void append_tail_ragged_kernel(const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+                                          uint16_t* __restrict__ k_tail, uint16_t* __restrict__ v_tail, int batch,
+                                          int heads, const __grid_constant__ RaggedAppendPlan plan) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;  // 16-byte chunk
+  const int per_bh = kHeadDim * 2 / 16;
+  const int n_bh = batch * heads;
+  if (i >= 2 * n_bh * per_bh) return;
+  const int tensor = i / (n_bh * per_bh);
+  const int r = i % (n_bh * per_bh);
+  const int bh = r / per_bh, ch = r % per_bh;
+  const int pos = plan.pos[bh / heads];
+  if (pos < 0) return;
+  const uint4* src = reinterpret_cast<const uint4*>((tensor ? v : k) + (size_t)bh * kHeadDim);
+  uint4* dst = reinterpret_cast<uint4*>((tensor ? v_tail : k_tail) + ((size_t)bh * kBlockTokens + pos) * kHeadDim);
+  dst[ch] = src[ch];
+}
+
+// Zeroes the index entries a call will publish (the look-back reads 0 as "not yet
+// published"), wherever the plan and the block table put them.
+template <class Plan>
+__global__ void clear_entries_kernel(const EncodeArgs a, const __grid_constant__ Plan plan, long n_call) {
+  const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n_call) return;
+  const size_t e = call_block(a, plan, t).entry;
+  reinterpret_cast<unsigned long long*>(a.k_index)[e] = 0ull;
+  reinterpret_cast<unsigned long long*>(a.v_index)[e] = 0ull;
+}
+
+template <class Plan>
+cudaError_t launch_encode_t(const EncodeArgs& a, const Plan& plan, cudaStream_t stream) {
+  const size_t smem = sizeof(EncodeSmem);
+  static bool configured = false;  // per process; the attribute is per function, not per device
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(encode_kernel<Plan>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const long n_call = (long)a.batch * a.heads * a.nb;
+  // the look-back reads the new index entries as "not yet published" (0), and the
+  // ticket and done counters start from zero
+  cudaError_t e = cudaSuccess;
+  if (!a.ragged && a.block_table == nullptr) {
+    const size_t pitch = (size_t)a.max_blocks * 8;
+    const size_t width = (size_t)a.nb * 8;
+    const size_t height = (size_t)a.batch * a.heads;
+    e = cudaMemset2DAsync(a.k_index + (size_t)a.n_old * 2, pitch, 0, width, height, stream);
+    if (e == cudaSuccess) e = cudaMemset2DAsync(a.v_index + (size_t)a.n_old * 2, pitch, 0, width, height, stream);
+  } else {
+    clear_entries_kernel<Plan><<<(unsigned)((n_call + 255) / 256), 256, 0, stream>>>(a, plan, n_call);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.ctrl + kCtrlScratch, 0, sizeof(uint64_t), stream);
+  if (e != cudaSuccess) return e;
+  encode_kernel<Plan><<<(unsigned)n_call, kEncodeThreads, smem, stream>>>(a, plan);
+  return cudaGetLastError();
+}
+
+struct NoEncodePlan {};
+
 }  // namespace
 
 size_t encode_smem_bytes() { return sizeof(EncodeSmem); }
 
-cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t stream) {
-  const size_t smem = sizeof(EncodeSmem);
-  static bool configured = false;  // per process; the attribute is per function, not per device
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  // the look-back reads the new index entries as "not yet published" (0), and the
-  // ticket and done counters start from zero
-  const size_t pitch = (size_t)a.max_blocks * 8;
-  const size_t width = (size_t)a.nb * 8;
-  const size_t height = (size_t)a.batch * a.heads;
-  cudaError_t e = cudaMemset2DAsync(a.k_index + (size_t)a.n_old * 2, pitch, 0, width, height, stream);
-  if (e == cudaSuccess) e = cudaMemset2DAsync(a.v_index + (size_t)a.n_old * 2, pitch, 0, width, height, stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(a.ctrl + kCtrlScratch, 0, sizeof(uint64_t), stream);
-  if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)((long)a.batch * a.heads * a.nb);
-  encode_kernel<<<grid, kEncodeThreads, smem, stream>>>(a);
-  return cudaGetLastError();
+cudaError_t launch_encode(const EncodeArgs& a, const RaggedEncodePlan* plan, cudaStream_t stream) {
+  if (a.ragged) return launch_encode_t<RaggedEncodePlan>(a, *plan, stream);
+  return launch_encode_t<NoEncodePlan>(a, NoEncodePlan{}, stream);
 }
 
 cudaError_t launch_append(const uint16_t* k, const uint16_t* v, uint16_t* k_tail, uint16_t* v_tail, int n_bh,
                           int pos, cudaStream_t stream) {
   const int chunks = 2 * n_bh * (kHeadDim * 2 / 16);
   append_tail_kernel<<<(chunks + 255) / 256, 256, 0, stream>>>(k, v, k_tail, v_tail, n_bh, pos);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_ragged(const uint16_t* k, const uint16_t* v, uint16_t* k_tail, uint16_t* v_tail,
+                                 int batch, int heads, const RaggedAppendPlan& plan, cudaStream_t stream) {
+  const int chunks = 2 * batch * heads * (kHeadDim * 2 / 16);
+  append_tail_ragged_kernel<<<(chunks + 255) / 256, 256, 0, stream>>>(k, v, k_tail, v_tail, batch, heads, plan);
   return cudaGetLastError();
 }
 

@@ -24,8 +24,9 @@
 //    (u8 x s8 -> s32, exact) multiplies them by q' or p' written as three
 //    base-128 digits of q'*f (f = 127 / max|q'| per record and head; about 22
 //    significant bits, the digits in three B columns).
-//  * Compressed (frame-of-reference) records are decoded on the CUDA cores by
-//    per-unit field extraction.
+//  * Compressed (frame-of-reference) records also run on the int8 tensor cores: the
+//    units of each pack group are sorted by width so that every run of 16 units is
+//    decoded with one instruction sequence (decode.cuh, "Compressed records").
 //  * p·V: a warp sums its item range into per-channel fp32 partials and writes
 //    them to the workspace at every (sequence, head) boundary (split-K over the
 //    sequence); a second-pass kernel, launched as a programmatic dependent so
@@ -52,28 +53,32 @@ constexpr int pv_min_ctas(int bits, int g) {
   return kWarpsPerCta != 4 ? 0 : g == 1 ? 5 : g == 4 ? (bits == 3 ? 0 : 4) : 0;
 }
 
-template <int BITS, int G>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G)) qk_kernel(const GemvArgs a) {
+template <int BITS, int G, class Plan>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G))
+    qk_kernel(const GemvArgs a, const __grid_constant__ Plan plan) {
   using C = Cfg<BITS, G, false>;
   extern __shared__ __align__(128) unsigned char smem[];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (warp >= a.n_warps) return;
   const WarpMem<BITS, G, false> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
   const long lo = (long)((long long)a.n_items * warp / a.n_warps);
   const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
-  const int I = a.items_per_bh;
   if (lane == 0) {
     for (int s = 0; s < C::kStages; ++s) mbar_init(m.bar(s), 1);
     fence_mbar_init();
   }
+  // launched as a programmatic dependent: everything above overlapped the previous
+  // kernel's tail; its results are visible after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncwarp();
   long prod = lo;
-  Cursor pc{lo / I, (int)(lo % I)};
+  Cursor pc = cursor_at(a, plan, lo);
   Cursor cc = pc;
   EntryWindow win;
-  win.load(a, lo, hi, lane);
-  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, pc.next(I))
+  win.load(a, plan, lo, hi, lane);
+  for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, cursor_next(a, plan, pc))
     issue_item<BITS, G, false>(a, m, pc, win.get(prod), s, lane);
 
   const int q_heads = a.kv_heads * G;
@@ -81,7 +86,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G)) qk_ke
   float qr[G][4];
   uint32_t phases = 0;
   int s = 0;
-  for (long x = lo; x < hi; ++x, cc.next(I)) {
+  for (long x = lo; x < hi; ++x, cursor_next(a, plan, cc)) {
     const long bh = cc.bh;
     const int j = cc.j;
     const long b = bh / a.kv_heads, h = bh % a.kv_heads;
@@ -105,18 +110,19 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G)) qk_ke
       drain_stages<BITS, G, false>(m, phases, s, x, prod, a.ctrl);
       return;
     }
-    const int kind = *m.kind(s);
-    const unsigned char* st = m.stage(s);
+    const int kind_len = *m.kind(s);
+    const int kind = kind_len & 0xFF;
+    unsigned char* st = m.stage(s);
     if (kind == kKindTail) {
-      qk_tail<G>(a, bh, qr, srow0, lane);
+      qk_tail<G>(a, bh, cc.nb, cc.tl, qr, srow0, lane);
     } else if (kind == kKindInvalid) {
       if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
 #pragma unroll
       for (int hd = 0; hd < G; ++hd)
         for (int i = lane; i < 128; i += 32) srow0[hd * a.ld + (long)j * 128 + i] = __int_as_float(0x7fc00000);
     } else {
-      // per record: the min term sum_c q_c * mn_c, then q' = q * scale_c as the
-      // int8 tensor-core B table (raw records) or the CUDA-core q' table
+      // per record: the min term sum_c q_c * mn_c, then q' = q * scale_c as the int8
+      // tensor-core B table (raw and compressed records alike)
       const uint2 mnv = *reinterpret_cast<const uint2*>(st + kParamOffset + 8 * lane);
       const uint2 scv = *reinterpret_cast<const uint2*>(st + kParamOffset + 256 + 8 * lane);
       const float2 mn0 = __half22float2(*reinterpret_cast<const __half2*>(&mnv.x));
@@ -138,27 +144,26 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G)) qk_ke
         qv[hd][3] = qr[hd][3] * sc1.y;
       }
       float* sblk = srow0 + (long)j * 128;
+      uint32_t* tab = m.table();
+      float invf[G];
+      build_i8tab<G, C::kNT>(tab, qv, invf, lane);
+      __syncwarp();
       if (kind == kKindRaw) {
-        uint32_t* tab = m.table();
-        float invf[G];
-        build_i8tab<G, C::kNT>(tab, qv, invf, lane);
-        __syncwarp();
         qk_i8<BITS, G>(st, tab, cst, invf, sblk, a.ld, a.scale, lane);
-      } else {
-        float* qp = reinterpret_cast<float*>(m.table());
+      } else if (!qk_packed_tc<BITS, G>(st, (uint32_t)(kind_len >> 8) * 16u, tab, qv, cst, invf, sblk, a.ld,
+                                         a.scale, lane)) {
+        if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
 #pragma unroll
         for (int hd = 0; hd < G; ++hd)
-          *reinterpret_cast<float4*>(qp + hd * 128 + 4 * lane) = make_float4(qv[hd][0], qv[hd][1], qv[hd][2], qv[hd][3]);
-        __syncwarp();
-        qk_packed<G>(st, qp, cst, sblk, a.ld, a.scale, lane);
+          for (int i = lane; i < 128; i += 32) sblk[hd * a.ld + i] = __int_as_float(0x7fc00000);
       }
     }
     __syncwarp();
     if (prod < hi) {
-      if (prod - win.base >= 32) win.load(a, prod, hi, lane);
+      if (prod - win.base >= 32) win.load(a, plan, prod, hi, lane);
       issue_item<BITS, G, false>(a, m, pc, win.get(prod), s, lane);
       ++prod;
-      pc.next(I);
+      cursor_next(a, plan, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
@@ -225,17 +230,24 @@ __device__ __forceinline__ void add4(float4& s, const float4 x) {
   s.w += x.w;
 }
 
-template <int G>
-__global__ void __launch_bounds__(kReduceWarps * 32) pv_reduce_kernel(const GemvArgs a) {
+template <int G, class Plan>
+__global__ void __launch_bounds__(kReduceWarps * 32)
+    pv_reduce_kernel(const GemvArgs a, const __grid_constant__ Plan plan) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 warp_sum4[kReduceWarps][32];
   const long row = blockIdx.x;  // (b*kv_heads + h)*G + head
   const long bh = row / G;
   const int hd = (int)(row % G);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long I = a.items_per_bh;
-  const long w0 = warp_of_item(bh * I, a.n_items, a.n_warps) + bh;
-  const long w1 = warp_of_item((bh + 1) * I - 1, a.n_items, a.n_warps) + bh;
+  long first = 0, n = 0;
+  row_items(a, plan, bh, &first, &n);
+  if (n == 0) {  // a sequence without tokens (ragged batches): its output is zero
+    if (warp == 0) reinterpret_cast<float4*>(a.out + row * 128)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+    return;
+  }
+  const long w0 = warp_of_item(first, a.n_items, a.n_warps) + bh;
+  const long w1 = warp_of_item(first + n - 1, a.n_items, a.n_warps) + bh;
   const float4* base = reinterpret_cast<const float4*>(a.partials + hd * 128) + lane;
   const size_t slot_stride = (size_t)G * 128 / 4;  // float4 per partial slot
   constexpr long W = kReduceWarps;
@@ -265,8 +277,9 @@ __global__ void __launch_bounds__(kReduceWarps * 32) pv_reduce_kernel(const Gemv
   }
 }
 
-template <int BITS, int G>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_kernel(const GemvArgs a) {
+template <int BITS, int G, class Plan>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
+    pv_kernel(const GemvArgs a, const __grid_constant__ Plan plan) {
   using C = Cfg<BITS, G, true>;
   extern __shared__ __align__(128) unsigned char smem[];
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -276,21 +289,21 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_ke
   const WarpMem<BITS, G, true> m{smem + (threadIdx.x >> 5) * C::kWarpSmem};
   const long lo = (long)((long long)a.n_items * warp / a.n_warps);
   const long hi = (long)((long long)a.n_items * (warp + 1) / a.n_warps);
-  const int I = a.items_per_bh;
   if (lane == 0) {
     for (int s = 0; s < C::kStages; ++s) mbar_init(m.bar(s), 1);
     fence_mbar_init();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's results are visible
   __syncwarp();
   long prod = lo;
-  Cursor pc{lo / I, (int)(lo % I)};
+  Cursor pc = cursor_at(a, plan, lo);
   Cursor cc = pc;
   EntryWindow win;
-  win.load(a, lo, hi, lane);
+  win.load(a, plan, lo, hi, lane);
   // p of the record in flight (this lane's slots 4*lane .. +3), loaded with its copy
   float4 pn[G];
-  auto load_p = [&](Cursor c) {
-    if (c.j < a.n_blocks) {
+  auto load_p = [&](const Cursor& c) {
+    if (c.j < c.nb) {
       const long b = c.bh / a.kv_heads, h = c.bh % a.kv_heads;
       const float* prow = a.p + ((size_t)b * a.kv_heads * G + h * G) * a.ld + (size_t)c.j * 128;
 #pragma unroll
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_ke
     issue_item<BITS, G, true>(a, m, pc, win.get(prod), 0, lane);
     load_p(pc);
     ++prod;
-    pc.next(I);
+    cursor_next(a, plan, pc);
   }
 
   float mp[G];  // sum over the warp's records of p * mn (lane: slots 4*lane .. +3)
@@ -314,13 +327,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_ke
 #pragma unroll
     for (int T = 0; T < 8; ++T) acc_lo[jn][T] = acc_hi[jn][T] = 0.f;
   float* sacc = m.sums();
-  float* pp = reinterpret_cast<float*>(m.table());  // p'' [G][128] then group sums [G][4]
   zero_sums<G>(sacc, lane);
   __syncwarp();
   long cur_bh = cc.bh;
   uint32_t phases = 0;
   int s = 0;
-  for (long x = lo; x < hi; ++x, cc.next(I)) {
+  for (long x = lo; x < hi; ++x, cursor_next(a, plan, cc)) {
     const long bh = cc.bh;
     if (bh != cur_bh) {
       pv_flush<G>(a, cur_bh, warp, sacc, acc_lo, acc_hi, mp, lane);
@@ -332,10 +344,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_ke
       drain_stages<BITS, G, true>(m, phases, s, x, prod, a.ctrl);
       return;
     }
-    const int kind = *m.kind(s);
-    const unsigned char* st = m.stage(s);
+    const int kind_len = *m.kind(s);
+    const int kind = kind_len & 0xFF;
+    unsigned char* st = m.stage(s);
     if (kind == kKindTail) {
-      pv_tail<G>(a, bh, sacc, lane);
+      pv_tail<G>(a, bh, cc.nb, cc.tl, sacc, lane);
     } else if (kind == kKindInvalid) {
       if (lane == 0) set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
     } else {
@@ -349,48 +362,41 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G)) pv_ke
       const float mnr[4] = {mn0.x, mn0.y, mn1.x, mn1.y};
       const float scr[4] = {sc0.x, sc0.y, sc1.x, sc1.y};
       float pv4[G][4];
+      float mpr[G];
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
         const float4 p4 = pn[hd];
         const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
+        mpr[hd] = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          mp[hd] = fmaf(pr[i], mnr[i], mp[hd]);
+          mpr[hd] = fmaf(pr[i], mnr[i], mpr[hd]);
           pv4[hd][i] = pr[i] * scr[i];
         }
       }
-      if (kind == kKindRaw) {
-        uint32_t* tab = m.table();
-        float invf[G];
-        build_i8tab<G, C::kNT>(tab, pv4, invf, lane);
-        __syncwarp();
+      uint32_t* tab = m.table();
+      float invf[G];
+      build_i8tab<G, C::kNT>(tab, pv4, invf, lane);
+      __syncwarp();
+      bool ok = true;
+      if (kind == kKindRaw)
         pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
-      } else {
-        // compressed record: p' by storage slot and the per-group sums of p'
+      else
+        ok = pv_packed_tc<BITS, G>(st, (uint32_t)(kind_len >> 8) * 16u, tab, pv4, invf, sacc, lane);
+      if (ok) {
 #pragma unroll
-        for (int hd = 0; hd < G; ++hd) {
-          float ps = 0.f;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ps += pv4[hd][i];
-          *reinterpret_cast<float4*>(pp + hd * 128 + 4 * lane) =
-              make_float4(pv4[hd][0], pv4[hd][1], pv4[hd][2], pv4[hd][3]);
-          // lanes 8g .. 8g+7 hold group g
-          ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-          ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-          ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-          if ((lane & 7) == 0) pp[G * 128 + hd * 4 + (lane >> 3)] = ps;
-        }
-        __syncwarp();
-        pv_packed<G>(st, pp, pp + G * 128, sacc, lane);
+        for (int hd = 0; hd < G; ++hd) mp[hd] += mpr[hd];
+      } else if (lane == 0) {
+        set_status(a.ctrl, PACKKV_DEV_BAD_RECORD);
       }
     }
     __syncwarp();
     if (prod < hi) {
-      if (prod - win.base >= 32) win.load(a, prod, hi, lane);
+      if (prod - win.base >= 32) win.load(a, plan, prod, hi, lane);
       issue_item<BITS, G, true>(a, m, pc, win.get(prod), s, lane);
       load_p(pc);
       ++prod;
-      pc.next(I);
+      cursor_next(a, plan, pc);
     }
     s = (s + 1 == C::kStages) ? 0 : s + 1;
   }
@@ -405,20 +411,20 @@ struct KernelInfo {
   int smem;
 };
 
-template <int BITS, int G, bool PV>
+template <int BITS, int G, bool PV, class Plan>
 KernelInfo kernel_info() {
   using C = Cfg<BITS, G, PV>;
   if constexpr (PV)
-    return {reinterpret_cast<const void*>(&pv_kernel<BITS, G>), kWarpsPerCta * C::kWarpSmem};
+    return {reinterpret_cast<const void*>(&pv_kernel<BITS, G, Plan>), kWarpsPerCta * C::kWarpSmem};
   else
-    return {reinterpret_cast<const void*>(&qk_kernel<BITS, G>), kWarpsPerCta * C::kWarpSmem};
+    return {reinterpret_cast<const void*>(&qk_kernel<BITS, G, Plan>), kWarpsPerCta * C::kWarpSmem};
 }
 
-template <bool PV>
+template <bool PV, class Plan>
 bool select(int bits, int group, KernelInfo* out) {
 #define PACKKV_CASE(B, GG)                  \
   if (bits == B && group == GG) {           \
-    *out = kernel_info<B, GG, PV>();        \
+    *out = kernel_info<B, GG, PV, Plan>();  \
     return true;                            \
   }
   PACKKV_CASE(4, 1) PACKKV_CASE(4, 2) PACKKV_CASE(4, 4) PACKKV_CASE(4, 8)
@@ -464,28 +470,45 @@ cudaError_t resident_warps(const KernelInfo& info, int* warps) {
   return cudaSuccess;
 }
 
-template <bool PV>
-cudaError_t launch(GemvArgs a, cudaStream_t stream) {
+template <int G, class Plan>
+const void* reduce_fn() {
+  return reinterpret_cast<const void*>(&pv_reduce_kernel<G, Plan>);
+}
+
+template <bool PV, class Plan>
+cudaError_t launch(GemvArgs a, const Plan* plan, cudaStream_t stream) {
   KernelInfo info{};
-  if (!select<PV>(a.bits, a.group, &info)) return cudaErrorInvalidValue;
+  if (!select<PV, Plan>(a.bits, a.group, &info)) return cudaErrorInvalidValue;
   int w = 0;
   cudaError_t e = resident_warps(info, &w);
   if (e != cudaSuccess) return e;
   if (w > gemv_max_warps()) w = gemv_max_warps();
   a.n_warps = (int)(a.n_items < w ? a.n_items : w);
+  if (a.n_warps < 1) a.n_warps = 1;
   const unsigned grid = (unsigned)((a.n_warps + kWarpsPerCta - 1) / kWarpsPerCta);
-  void* args[] = {&a};
-  e = cudaLaunchKernel(info.fn, dim3(grid), dim3(kWarpsPerCta * 32), args, info.smem, stream);
-  if (e != cudaSuccess || !PV) return e;
+  void* args[] = {&a, const_cast<Plan*>(plan)};
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  if (a.n_items > 0) {
+    // a programmatic dependent of whatever precedes it: the kernel waits for that
+    // kernel's results before its first global access (griddepcontrol.wait)
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(grid);
+    lc.blockDim = dim3(kWarpsPerCta * 32);
+    lc.dynamicSmemBytes = (size_t)info.smem;
+    lc.stream = stream;
+    lc.attrs = pdl;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelExC(&lc, info.fn, args);
+    if (e != cudaSuccess || !PV) return e;
+  } else if (!PV) {
+    return cudaSuccess;
+  }
   // second pass of p·V, launched early (programmatic dependent launch); it waits for pv_kernel
   const long rows = (long)a.batch * a.kv_heads * a.group;
-  const void* red = nullptr;
-  switch (a.group) {
-    case 1: red = reinterpret_cast<const void*>(&pv_reduce_kernel<1>); break;
-    case 2: red = reinterpret_cast<const void*>(&pv_reduce_kernel<2>); break;
-    case 4: red = reinterpret_cast<const void*>(&pv_reduce_kernel<4>); break;
-    default: red = reinterpret_cast<const void*>(&pv_reduce_kernel<8>); break;
-  }
+  const void* red = a.group == 1 ? reduce_fn<1, Plan>() : a.group == 2 ? reduce_fn<2, Plan>()
+                  : a.group == 4 ? reduce_fn<4, Plan>() : reduce_fn<8, Plan>();
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)rows);
   cfg.blockDim = dim3(kReduceWarps * 32);
@@ -495,7 +518,7 @@ cudaError_t launch(GemvArgs a, cudaStream_t stream) {
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.n_items > 0 ? 1 : 0;
   return cudaLaunchKernelExC(&cfg, red, args);
 }
 
@@ -514,7 +537,7 @@ size_t pv_workspace_bytes(int batch, int kv_heads, int group) {
 
 cudaError_t pv_launch_workspace_bytes(const GemvArgs& a, size_t* bytes) {
   KernelInfo info{};
-  if (!select<true>(a.bits, a.group, &info)) return cudaErrorInvalidValue;
+  if (!select<true, NoPlan>(a.bits, a.group, &info)) return cudaErrorInvalidValue;
   int w = 0;
   const cudaError_t e = resident_warps(info, &w);
   if (e != cudaSuccess) return e;
@@ -524,7 +547,13 @@ cudaError_t pv_launch_workspace_bytes(const GemvArgs& a, size_t* bytes) {
   return cudaSuccess;
 }
 
-cudaError_t launch_qk(GemvArgs a, cudaStream_t stream) { return launch<false>(a, stream); }
-cudaError_t launch_pv(GemvArgs a, cudaStream_t stream) { return launch<true>(a, stream); }
+cudaError_t launch_qk(GemvArgs a, const RaggedPlan* plan, cudaStream_t stream) {
+  static const NoPlan none{};
+  return plan ? launch<false, RaggedPlan>(a, plan, stream) : launch<false, NoPlan>(a, &none, stream);
+}
+cudaError_t launch_pv(GemvArgs a, const RaggedPlan* plan, cudaStream_t stream) {
+  static const NoPlan none{};
+  return plan ? launch<true, RaggedPlan>(a, plan, stream) : launch<true, NoPlan>(a, &none, stream);
+}
 
 }  // namespace packkv

@@ -5,7 +5,28 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "packkv.h"
+
 namespace packkv {
+
+// Ragged batches (sequences of their own lengths) are described to the kernels by value,
+// in the launch's parameter space: per sequence b, base[b] = its first item in the flat
+// (sequence, head, item) list and tail[b] = its tail tokens (items of b: base[b+1] -
+// base[b] = kv_heads * (blocks + (tail > 0))).  At most kMaxRaggedBatch sequences.
+constexpr int kMaxRaggedBatch = PACKKV_RAGGED_MAX_BATCH;
+struct RaggedPlan {
+  int32_t base[kMaxRaggedBatch + 1];
+  int32_t tail[kMaxRaggedBatch];
+};
+// The sequences an encode call touches, in order, and the logical block each starts at.
+struct RaggedEncodePlan {
+  int32_t seq[kMaxRaggedBatch];
+  int32_t first_block[kMaxRaggedBatch];
+};
+// The tail position each sequence appends at (-1: the sequence takes no token).
+struct RaggedAppendPlan {
+  int32_t pos[kMaxRaggedBatch];
+};
 
 struct EncodeArgs {
   const uint16_t* k;  // [batch][heads][nb*128][128] fp16
@@ -18,11 +39,18 @@ struct EncodeArgs {
   uint64_t arena_bytes;
   uint8_t* perm;  // optional
   uint64_t* ctrl;
+  // ragged calls: `batch` sequences of the plan (seq[s], first_block[s]); k, v rows are
+  // (seq[s] * heads + h) * nb + i; block_table (optional, device) maps logical blocks
+  const int32_t* block_table;
+  bool ragged;
 };
 
-cudaError_t launch_encode(const EncodeArgs& a, cudaStream_t stream);
+cudaError_t launch_encode(const EncodeArgs& a, const RaggedEncodePlan* plan, cudaStream_t stream);
 cudaError_t launch_append(const uint16_t* k, const uint16_t* v, uint16_t* k_tail, uint16_t* v_tail, int n_bh,
                           int pos, cudaStream_t stream);
+// Ragged append: sequence b's token goes to tail position plan.pos[b] (none if negative).
+cudaError_t launch_append_ragged(const uint16_t* k, const uint16_t* v, uint16_t* k_tail, uint16_t* v_tail,
+                                 int batch, int heads, const RaggedAppendPlan& plan, cudaStream_t stream);
 size_t encode_smem_bytes();
 
 // One decode GEMV over the packed cache (q·Kᵀ or p·V).
@@ -36,6 +64,8 @@ struct GemvArgs {
   long n_items;           // batch*kv_heads*items_per_bh
   int items_per_bh;       // n_blocks + (tail_len > 0)
   int n_warps;            // logical warps sharing the items
+  const int32_t* block_table;  // optional: physical block of (sequence, logical block)
+  bool ragged;            // sequences of their own lengths (RaggedPlan passed with the launch)
   // q·Kᵀ
   const uint16_t* q;      // [batch][q_heads][128]
   float* scores;          // row (b, hq) at (b*q_heads + hq) * ld
@@ -47,8 +77,8 @@ struct GemvArgs {
   float* partials;        // [n_warps + batch*kv_heads][group][128]
 };
 
-cudaError_t launch_qk(GemvArgs a, cudaStream_t stream);
-cudaError_t launch_pv(GemvArgs a, cudaStream_t stream);
+cudaError_t launch_qk(GemvArgs a, const RaggedPlan* plan, cudaStream_t stream);
+cudaError_t launch_pv(GemvArgs a, const RaggedPlan* plan, cudaStream_t stream);
 
 // Logical warps used by the GEMVs on the current device (an upper bound used
 // for workspace sizing), and the workspace layout of p·V.
@@ -71,13 +101,15 @@ struct AttnArgs {
   long n_items;             // batch*kv_heads*items_per_bh
   int items_per_bh;         // n_blocks + (tail_len > 0)
   int n_warps;              // logical warps sharing the items
+  const int32_t* block_table;  // optional: physical block of (sequence, logical block)
+  bool ragged;              // sequences of their own lengths (RaggedPlan passed with the launch)
   const uint16_t* q;        // [batch][q_heads][128]
   float scale;
   float* out;               // [batch][q_heads][128]
   float* partials;          // [n_warps + batch*kv_heads][group][132]: sums [128], max, sum of exp
 };
 
-cudaError_t launch_attention(AttnArgs a, cudaStream_t stream);
+cudaError_t launch_attention(AttnArgs a, const RaggedPlan* plan, cudaStream_t stream);
 size_t attention_workspace_bytes(int batch, int kv_heads, int group);
 
 }  // namespace packkv

@@ -55,6 +55,7 @@ packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, 
                                      float* out, void* stream) {
   const packkv_status st = packkv_cache_check(cache);
   if (st != PACKKV_OK) return st;
+  if (cache->seq_blocks != nullptr || cache->block_table != nullptr) return PACKKV_ERR_UNSUPPORTED;
   if (q_heads < 1 || q_heads % cache->kv_heads != 0) return PACKKV_ERR_INVALID_ARG;
   const int g = q_heads / cache->kv_heads;
   if (g != 1 && g != 2 && g != 4 && g != 8) return PACKKV_ERR_UNSUPPORTED;
@@ -89,7 +90,7 @@ packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, 
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return PACKKV_ERR_CUDA;
   a.partials = reinterpret_cast<float*>(scratch);
-  return packkv::launch_pv(a, s) == cudaSuccess ? PACKKV_OK : PACKKV_ERR_CUDA;
+  return packkv::launch_pv(a, nullptr, s) == cudaSuccess ? PACKKV_OK : PACKKV_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -31,8 +31,10 @@ EXPORTED = [
     "packkv_workspace_bytes", "packkv_cache_check", "packkv_cache_reset", "packkv_encode_block",
     "packkv_append_token", "packkv_qk_gemv", "packkv_pv_gemv", "packkv_get_status",
     "packkv_pv_gemv_noalloc", "packkv_attention_workspace_bytes",
-    "packkv_attention_decode",
+    "packkv_attention_decode", "packkv_append_token_masked",
 ]
+
+RAGGED_MAX_BATCH = 2048
 
 
 class PackKVError(RuntimeError):
@@ -52,7 +54,8 @@ class CacheStruct(ctypes.Structure):
                 ("reserved0", ctypes.c_int32), ("k_arena", ctypes.c_void_p), ("v_arena", ctypes.c_void_p),
                 ("arena_bytes", ctypes.c_uint64), ("k_index", ctypes.c_void_p), ("v_index", ctypes.c_void_p),
                 ("k_tail", ctypes.c_void_p), ("v_tail", ctypes.c_void_p), ("ctrl", ctypes.c_void_p),
-                ("perm", ctypes.c_void_p)]
+                ("perm", ctypes.c_void_p), ("seq_blocks", ctypes.POINTER(ctypes.c_int32)),
+                ("seq_tail", ctypes.POINTER(ctypes.c_int32)), ("block_table", ctypes.c_void_p)]
 
 
 def _load():
@@ -78,6 +81,7 @@ def _load():
         "packkv_pv_gemv_noalloc": (ctypes.c_int, [P, vp, i64, i32, vp, vp]),
         "packkv_attention_workspace_bytes": (sz, [P, i32]),
         "packkv_attention_decode": (ctypes.c_int, [P, vp, i32, f32, vp, vp, sz, vp]),
+        "packkv_append_token_masked": (ctypes.c_int, [P, vp, vp, ctypes.POINTER(ctypes.c_uint8), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -114,10 +118,15 @@ def record_bytes_max(bits: int) -> int:
 
 
 class PackKVCache:
-    """Device buffers + the packkv_cache struct of one layer's packed cache."""
+    """Device buffers + the packkv_cache struct of one layer's packed cache.
+
+    ragged=True gives every sequence its own length (host counters seq_blocks /
+    seq_tail in the struct); block_table (int32 [batch, max_blocks], on the device)
+    maps each sequence's logical blocks to physical blocks of the index."""
 
     def __init__(self, batch: int, kv_heads: int, max_blocks: int, bits: int, reorder_key: int = KEY_K_SUM,
-                 arena_bytes: int | None = None, keep_perm: bool = False, device="cuda"):
+                 arena_bytes: int | None = None, keep_perm: bool = False, device="cuda", ragged: bool = False,
+                 block_table: torch.Tensor | None = None):
         dev = torch.device(device)
         if arena_bytes is None:
             arena_bytes = batch * kv_heads * max_blocks * record_bytes_max(bits)
@@ -141,6 +150,19 @@ class PackKVCache:
         self.s.k_tail, self.s.v_tail = self.k_tail.data_ptr(), self.v_tail.data_ptr()
         self.s.ctrl = self.ctrl.data_ptr()
         self.s.perm = self.perm.data_ptr() if self.perm is not None else None
+        self.ragged = ragged
+        if ragged:
+            self._seq_blocks = (ctypes.c_int32 * batch)()
+            self._seq_tail = (ctypes.c_int32 * batch)()
+            self.s.seq_blocks = ctypes.cast(self._seq_blocks, ctypes.POINTER(ctypes.c_int32))
+            self.s.seq_tail = ctypes.cast(self._seq_tail, ctypes.POINTER(ctypes.c_int32))
+        self.block_table = None
+        if block_table is not None:
+            bt = block_table.to(device=dev, dtype=torch.int32).contiguous()
+            if tuple(bt.shape) != (batch, max_blocks):
+                raise ValueError("block_table must be int32 [batch, max_blocks]")
+            self.block_table = bt
+            self.s.block_table = bt.data_ptr()
         _check("packkv_cache_check", _lib.packkv_cache_check(ctypes.byref(self.s)))
         self._ws = {}
 
@@ -155,7 +177,23 @@ class PackKVCache:
 
     @property
     def tokens(self) -> int:
+        """Tokens of the longest sequence (every sequence, for a uniform batch)."""
+        if self.ragged:
+            return max((self.seq_tokens(b) for b in range(self.batch)), default=0)
         return self.s.n_blocks * BLOCK_TOKENS + self.s.tail_len
+
+    def seq_tokens(self, b: int) -> int:
+        if not self.ragged:
+            return self.tokens
+        return self._seq_blocks[b] * BLOCK_TOKENS + self._seq_tail[b]
+
+    @property
+    def seq_blocks(self):
+        return list(self._seq_blocks) if self.ragged else [self.s.n_blocks] * self.batch
+
+    @property
+    def seq_tail(self):
+        return list(self._seq_tail) if self.ragged else [self.s.tail_len] * self.batch
 
     @property
     def bits(self) -> int:
@@ -213,6 +251,16 @@ def packkv_append_token(cache: PackKVCache, k: torch.Tensor, v: torch.Tensor, st
         raise ValueError("k, v must be fp16 [batch, kv_heads, 128]")
     _check("packkv_append_token", _lib.packkv_append_token(ctypes.byref(cache.s), _ptr(k), _ptr(v),
                                                            _stream(stream)))
+
+
+def packkv_append_token_masked(cache: PackKVCache, k: torch.Tensor, v: torch.Tensor, active, stream=None):
+    """Ragged caches: one token for the sequences with active[b] (k, v fp16 [batch, kv_heads, 128])."""
+    if k.dtype != torch.float16 or v.dtype != torch.float16 or tuple(k.shape) != (cache.batch, cache.kv_heads,
+                                                                                   HEAD_DIM) or k.shape != v.shape:
+        raise ValueError("k, v must be fp16 [batch, kv_heads, 128]")
+    act = (ctypes.c_uint8 * cache.batch)(*[1 if a else 0 for a in active])
+    _check("packkv_append_token_masked", _lib.packkv_append_token_masked(ctypes.byref(cache.s), _ptr(k), _ptr(v),
+                                                                         act, _stream(stream)))
 
 
 def packkv_qk_gemv(cache: PackKVCache, q: torch.Tensor, scale: float, scores: torch.Tensor, stream=None):

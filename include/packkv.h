@@ -38,11 +38,12 @@
 extern "C" {
 #endif
 
-#define PACKKV_ABI_VERSION 1u
+#define PACKKV_ABI_VERSION 2u
 #define PACKKV_FORMAT_VERSION 1u
 #define PACKKV_BLOCK_TOKENS 128
 #define PACKKV_GROUP_TOKENS 32
 #define PACKKV_HEAD_DIM 128
+#define PACKKV_RAGGED_MAX_BATCH 2048  /* sequences of a ragged batch (see packkv_cache) */
 
 typedef enum {
   PACKKV_OK = 0,
@@ -77,6 +78,20 @@ typedef struct {
  * The packed cache of one attention layer: plain data, every pointer owned by
  * the caller.  Zero ctrl[0..3] and set n_blocks = tail_len = 0 before first
  * use (packkv_cache_reset does both).
+ *
+ * Ragged batches and paged blocks (the visualisation page, "Read the caveat":
+ * paging and multi-request scheduling).  With seq_blocks and seq_tail set, each
+ * sequence b has its own length: seq_blocks[b] packed blocks and seq_tail[b]
+ * (0..127) tail tokens.  Both are HOST arrays of `batch` int32 that the calls
+ * read and advance at enqueue time, as they do n_blocks and tail_len for a
+ * uniform batch (which must then stay 0); batch <= PACKKV_RAGGED_MAX_BATCH.
+ * Scores and probabilities of sequence b are its first seq_blocks[b]*128 +
+ * seq_tail[b] row entries; a sequence without tokens gets zero outputs.
+ * With block_table set (uniform or ragged), logical block j of sequence b is the
+ * physical block p = block_table[b*max_blocks + j] (device int32), whose records
+ * the index entries at (p / max_blocks, head, p % max_blocks) name: sequences may
+ * share blocks (a common prompt) and need not own contiguous index rows.  The
+ * blocks an encode or append call creates must map to distinct physical blocks.
  */
 typedef struct {
   packkv_format fmt;
@@ -95,7 +110,10 @@ typedef struct {
   uint16_t* v_tail;    /* device fp16, same shape */
   uint64_t* ctrl;      /* device u64[4]: K arena end (16-B units), V arena end, status bits, scratch */
   uint8_t* perm;       /* device, optional (NULL): u8 [batch][kv_heads][max_blocks][128],
-                          perm[slot] = token index within the block */
+                          perm[slot] = token index within the block (at the physical block) */
+  int32_t* seq_blocks; /* host, optional (NULL = uniform batch): [batch] packed blocks per sequence */
+  int32_t* seq_tail;   /* host, with seq_blocks: [batch] tail tokens per sequence */
+  const int32_t* block_table; /* device, optional (NULL): [batch][max_blocks] physical blocks */
 } packkv_cache;
 
 /* ABI version and sizeof(packkv_cache), for bindings to check their mirror. */
@@ -132,6 +150,8 @@ packkv_status packkv_cache_reset(packkv_cache* cache, void* stream);
  * arena offsets come from a decoupled look-back over the new index entries
  * (which the call clears first) and ctrl[3] counts the call's blocks.
  * n_blocks == 0 is a no-op.
+ * Ragged batch: every sequence gets n_blocks blocks after its own seq_blocks[b]
+ * (every seq_tail[b] must be 0); seq_blocks[b] += n_blocks.
  */
 packkv_status packkv_encode_block(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
                                   int32_t n_blocks, void* stream);
@@ -142,9 +162,21 @@ packkv_status packkv_encode_block(packkv_cache* cache, const uint16_t* k, const 
  * When the tail reaches 128 tokens it is encoded as one block (as
  * packkv_encode_block) and tail_len returns to 0.
  * PACKKV_ERR_CAPACITY if the tail is full-to-be and the block table is full.
+ * Ragged batch: every sequence appends at its own seq_tail[b]; the sequences whose
+ * tail completes are encoded (in ascending order) into their next block.
  */
 packkv_status packkv_append_token(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
                                   void* stream);
+
+/*
+ * Ragged batch only: as packkv_append_token for the sequences with active[b] != 0
+ * (host uint8 [batch]); the others take no token (k, v rows of those are not read).
+ * This is how sequences of one batch come to differ in length (a request that
+ * joins later, or one that has finished).  PACKKV_ERR_UNSUPPORTED for a uniform
+ * batch.
+ */
+packkv_status packkv_append_token_masked(packkv_cache* cache, const uint16_t* k, const uint16_t* v,
+                                         const uint8_t* active, void* stream);
 
 /*
  * scores[b][hq][i] = scale * sum_c q[b][hq][c] * k_hat[b][hq/G][i][c]  (fp32 accumulate)
@@ -152,7 +184,8 @@ packkv_status packkv_append_token(packkv_cache* cache, const uint16_t* k, const 
  * (packed-cache format v1, sections 6-7; paper page Figure 1, Figure 2 fused decompression).
  *   q:      device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8}.
  *   scores: device fp32, row (b, hq) starts at (b*q_heads + hq) * ld_scores;
- *           ld_scores >= T = n_blocks*128 + tail_len, multiple of 4.
+ *           ld_scores >= T = n_blocks*128 + tail_len (ragged: the longest sequence),
+ *           multiple of 4.
  *   ws, ws_bytes: unused (may be NULL / 0).
  * The decompressed K is never written to memory.  T == 0 is a no-op.
  */
@@ -198,6 +231,7 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
  * All calls share the one array, and it keeps the last call's partials: calls
  * that overlap in time on the GPU race.  Nothing in it needs clearing (every
  * partial is written before it is read).  With T == 0, out is set to zero.
+ * A ragged cache or one with a block table: PACKKV_ERR_UNSUPPORTED.
  */
 #define PACKKV_PV_NOALLOC_SCRATCH_BYTES (8u << 20)
 packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, int64_t ld_p,
@@ -216,7 +250,8 @@ packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, 
  *   out: device fp32 [batch][q_heads][128].
  *   ws:  device, ws_bytes >= packkv_attention_workspace_bytes(cache, q_heads)
  *        (no initialisation needed; two calls sharing ws must not overlap in time).
- * T == 0 (nothing to attend to) is PACKKV_ERR_INVALID_ARG.  A record with an
+ * T == 0 (nothing to attend to) is PACKKV_ERR_INVALID_ARG for a uniform batch; in a
+ * ragged batch a sequence without tokens gets zero outputs.  A record with an
  * invalid index entry sets PACKKV_DEV_BAD_RECORD and its tokens are left out.
  */
 size_t packkv_attention_workspace_bytes(const packkv_cache* cache, int32_t q_heads);

@@ -494,6 +494,143 @@ class OracleCache:
 
 
 # ----------------------------------------------------------------------------
+# Ragged batches and paged blocks (the visualisation page, "Read the caveat":
+# paging and multi-request scheduling are what deployment adds)
+# ----------------------------------------------------------------------------
+class RaggedOracleCache(OracleCache):
+    """A batch whose sequences have their own lengths, over the same record format.
+
+    Sequence b holds seq_blocks[b] packed blocks and seq_tail[b] tail tokens.  Logical
+    block j of sequence b lives at physical block p = table[b, j] (default
+    b * max_blocks + j), i.e. at index entry (p // max_blocks, head, p % max_blocks):
+    sequences may share a physical block (a common prefix) and a sequence's blocks need
+    not be contiguous.  Calls append records to the arenas in ascending (sequence, head,
+    block) order of the sequences they touch, as the uniform cache does.
+    """
+
+    def __init__(self, batch, kv_heads, max_blocks, bits, key_kind=KEY_K_SUM, table=None):
+        super().__init__(batch, kv_heads, max_blocks, bits, key_kind)
+        self.seq_blocks = [0] * batch
+        self.seq_tail = [0] * batch
+        ids = np.arange(batch * max_blocks, dtype=np.int64).reshape(batch, max_blocks)
+        self.table = ids if table is None else np.asarray(table, np.int64).reshape(batch, max_blocks)
+
+    def physical(self, b: int, j: int):
+        """(index row, block slot) of logical block j of sequence b."""
+        return divmod(int(self.table[b, j]), self.max_blocks)
+
+    def _encode_one(self, b, h, j, k_blk, v_blk):
+        k_rec, v_rec, perm = encode_block(k_blk, v_blk, self.bits, self.key_kind)
+        rb, jb = self.physical(b, j)
+        self.k_index[rb, h, jb] = (len(self.k_arena) // 16, len(k_rec) // 16)
+        self.v_index[rb, h, jb] = (len(self.v_arena) // 16, len(v_rec) // 16)
+        self.k_arena += k_rec
+        self.v_arena += v_rec
+        self.perm[rb, h, jb] = perm
+        for key in [key for key in self._decoded if key[1:] == (rb, h, jb)]:
+            del self._decoded[key]
+
+    def encode_blocks_ragged(self, k: np.ndarray, v: np.ndarray, n_blocks: int):
+        """Append n_blocks blocks to every sequence (after its own blocks; its tail must
+        be empty); k, v: [B, Hkv, n_blocks*128, D] fp16."""
+        for b in range(self.batch):
+            if self.seq_tail[b] != 0 or self.seq_blocks[b] + n_blocks > self.max_blocks:
+                raise ValueError("tail not empty or capacity")
+        for b in range(self.batch):
+            for h in range(self.kv_heads):
+                for i in range(n_blocks):
+                    sl = slice(i * BLOCK_TOKENS, (i + 1) * BLOCK_TOKENS)
+                    self._encode_one(b, h, self.seq_blocks[b] + i, k[b, h, sl], v[b, h, sl])
+            self.seq_blocks[b] += n_blocks
+
+    def append_token_ragged(self, k_tok: np.ndarray, v_tok: np.ndarray, active=None):
+        """One token for every sequence in `active` (default: all), at its own tail
+        position; a tail that reaches 128 tokens is encoded as the sequence's next block
+        (sequences in ascending order)."""
+        seqs = range(self.batch) if active is None else sorted(active)
+        done = []
+        for b in seqs:
+            self.k_tail[b, :, self.seq_tail[b]] = k_tok[b]
+            self.v_tail[b, :, self.seq_tail[b]] = v_tok[b]
+            self.seq_tail[b] += 1
+            if self.seq_tail[b] == BLOCK_TOKENS:
+                done.append(b)
+        for b in done:
+            if self.seq_blocks[b] >= self.max_blocks:
+                raise ValueError("capacity")
+            for h in range(self.kv_heads):
+                self._encode_one(b, h, self.seq_blocks[b], self.k_tail[b, h].copy(), self.v_tail[b, h].copy())
+            self.seq_blocks[b] += 1
+            self.seq_tail[b] = 0
+
+    def seq_tokens(self, b: int) -> int:
+        return self.seq_blocks[b] * BLOCK_TOKENS + self.seq_tail[b]
+
+    def decoded(self, which: str, b: int, h: int) -> np.ndarray:
+        """Sequence b, head h in storage order, fp64 [T_b, D]: its blocks through the
+        table, then its tail."""
+        parts = []
+        for j in range(self.seq_blocks[b]):
+            rb, jb = self.physical(b, j)
+            key = (which, rb, h, jb)
+            if key not in self._decoded:
+                rec = parse_record(self.record(which, rb, h, jb))
+                self._decoded[key] = dequant_k(rec) if which == "k" else dequant_v(rec)
+            parts.append(self._decoded[key])
+        tail = (self.k_tail if which == "k" else self.v_tail)[b, h, :self.seq_tail[b]]
+        parts.append(tail.astype(np.float64))
+        return np.concatenate(parts, axis=0)
+
+    @property
+    def tokens(self) -> int:
+        return max(self.seq_tokens(b) for b in range(self.batch))
+
+
+def ragged_qk(cache: RaggedOracleCache, q: np.ndarray, scale: float):
+    """Scores of a ragged batch: [B, Hq, T_max] with row (b, hq) defined on [0, T_b)
+    (NaN past it), and the sums of |terms|."""
+    B, Hq, _ = q.shape
+    G = Hq // cache.kv_heads
+    T = cache.tokens
+    scores = np.full((B, Hq, T), np.nan)
+    sums = np.full((B, Hq, T), np.nan)
+    for b in range(B):
+        Tb = cache.seq_tokens(b)
+        for h in range(cache.kv_heads):
+            s_, a_ = qk_scores(q[b, h * G:(h + 1) * G], cache.decoded("k", b, h), scale)
+            scores[b, h * G:(h + 1) * G, :Tb] = s_
+            sums[b, h * G:(h + 1) * G, :Tb] = a_
+    return scores, sums
+
+
+def ragged_pv(cache: RaggedOracleCache, p: np.ndarray):
+    """Outputs of a ragged batch: p [B, Hq, >= T_b] (only [:T_b] of row b is read)."""
+    B, Hq, _ = p.shape
+    G = Hq // cache.kv_heads
+    out = np.zeros((B, Hq, HEAD_DIM))
+    sums = np.zeros((B, Hq, HEAD_DIM))
+    for b in range(B):
+        Tb = cache.seq_tokens(b)
+        for h in range(cache.kv_heads):
+            o, a_ = pv_out(p[b, h * G:(h + 1) * G, :Tb], cache.decoded("v", b, h))
+            out[b, h * G:(h + 1) * G] = o
+            sums[b, h * G:(h + 1) * G] = a_
+    return out, sums
+
+
+def ragged_attention(cache: RaggedOracleCache, q: np.ndarray, scale: float):
+    """Decode attention of a ragged batch: each sequence's softmax runs over its own
+    T_b tokens ([Fig. 1])."""
+    B, Hq, _ = q.shape
+    scores, _ = ragged_qk(cache, q, scale)
+    p = np.zeros_like(scores)
+    for b in range(B):
+        Tb = cache.seq_tokens(b)
+        p[b, :, :Tb] = softmax(scores[b, :, :Tb])
+    return ragged_pv(cache, p)
+
+
+# ----------------------------------------------------------------------------
 # The two decode products ([Fig. 1], [Fig. 2] fused decompression + GEMV), fp64
 # ----------------------------------------------------------------------------
 def qk_scores(q: np.ndarray, k_dec: np.ndarray, scale: float):

@@ -58,7 +58,7 @@ def test_library_exports_every_declared_symbol(pk):
 
 def test_abi_constants(pk):
     lib = pk._lib
-    assert lib.packkv_abi_version() == 1
+    assert lib.packkv_abi_version() == 2
     assert lib.packkv_cache_struct_size() == ctypes.sizeof(pk.CacheStruct)
     assert [lib.packkv_record_bytes_max(b) for b in (1, 2, 3, 4, 5)] == [0, 4624, 6672, 8720, 0]
     assert lib.packkv_status_string(3) == b"capacity exceeded"
@@ -130,3 +130,46 @@ def test_host_checks_reject_before_launch(pk):
     need = lib.packkv_attention_workspace_bytes(ctypes.byref(s), 2)
     assert need > 0
     assert att(ctypes.byref(s), k, 2, 1.0, k, k, need - 16, None) == pk.ERR_INVALID_ARG
+
+
+def test_ragged_host_checks(pk):
+    """Ragged caches (host counters per sequence): malformed counters, appends that
+    would overflow a sequence's blocks, calls that need an empty tail, and calls that
+    do not take ragged caches are refused on the host, before any launch."""
+    lib = pk._lib
+    B = 2
+    blocks = (ctypes.c_int32 * B)(1, 3)
+    tail = (ctypes.c_int32 * B)(0, 127)
+    P = ctypes.POINTER(ctypes.c_int32)
+
+    def ragged(**over):
+        s = _fake_cache(pk, **over)
+        s.seq_blocks, s.seq_tail = ctypes.cast(blocks, P), ctypes.cast(tail, P)
+        return s
+
+    assert lib.packkv_cache_check(ctypes.byref(ragged())) == pk.OK
+    assert lib.packkv_cache_check(ctypes.byref(ragged(n_blocks=1))) == pk.ERR_INVALID_ARG
+    half = _fake_cache(pk)
+    half.seq_blocks = ctypes.cast(blocks, P)
+    assert lib.packkv_cache_check(ctypes.byref(half)) == pk.ERR_INVALID_ARG      # seq_tail missing
+    tail[1] = 128
+    assert lib.packkv_cache_check(ctypes.byref(ragged())) == pk.ERR_INVALID_ARG  # tail out of range
+    tail[1] = 127
+    blocks[0] = 5
+    assert lib.packkv_cache_check(ctypes.byref(ragged())) == pk.ERR_INVALID_ARG  # beyond max_blocks
+    blocks[0] = 1
+    big = ragged(batch=pk.RAGGED_MAX_BATCH + 1)
+    assert lib.packkv_cache_check(ctypes.byref(big)) == pk.ERR_UNSUPPORTED
+    k = ctypes.c_void_p(0x20000000)
+    s = ragged()
+    assert lib.packkv_encode_block(ctypes.byref(s), k, k, 1, None) == pk.ERR_INVALID_ARG  # a tail is not empty
+    blocks[1], tail[1] = 4, 127                         # sequence 1 completes a block it has no room for
+    act = (ctypes.c_uint8 * B)(0, 1)
+    assert lib.packkv_append_token_masked(ctypes.byref(ragged()), k, k, act, None) == pk.ERR_CAPACITY
+    assert list(blocks) == [1, 4] and list(tail) == [0, 127]   # nothing advanced
+    u = _fake_cache(pk)
+    assert lib.packkv_append_token_masked(ctypes.byref(u), k, k, act, None) == pk.ERR_UNSUPPORTED
+    assert lib.packkv_pv_gemv_noalloc(ctypes.byref(ragged()), k, 1024, 2, k, None) == pk.ERR_UNSUPPORTED
+    s = _fake_cache(pk, n_blocks=1)
+    s.block_table = 0x30000002                          # misaligned table
+    assert lib.packkv_cache_check(ctypes.byref(s)) == pk.ERR_INVALID_ARG
