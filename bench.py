@@ -321,10 +321,10 @@ def compression_entry(cs, bits):
             "k_record_bytes": int(cs.k_used), "v_record_bytes": int(cs.v_used)}
 
 
-def workload_record(pk, dev, wid, bits, peak, structured=False, kd=None, vd=None, attention=True):
+def workload_record(pk, dev, wid, bits, peak, structured=False, kd=None, vd=None, attention=True, w_override=None):
     """Per-kernel figures of one workload: q·Kᵀ, p·V and the fused attention, each
     timed alone over whole rotations of enough cache copies; compression; cuBLAS."""
-    w = synth.WORKLOADS[wid]
+    w = synth.WORKLOADS[wid] if w_override is None else w_override
     if kd is None:
         kd, vd = upload(w, w.seq, dev, structured)
     probe_bytes = w.batch * w.kv_heads * (w.seq // 128) * (528 + 2048 * bits)
@@ -439,6 +439,81 @@ def streaming_record(pk, dev, bits, layers=3):
                       "CUDA events, after a warm-up replay of an identical graph"}
 
 
+def ragged_record(pk, dev, peak, bits=3):
+    """Ragged batched decode: the batched shape (16 sequences x 32 heads, 3-bit) with
+    each sequence's own length, a seeded multiple of 128 in [4096, 16384].  The cache
+    is prefilled to 16384 tokens and each sequence's host counters are then set to
+    its length (the records past it are not read).  q·Kᵀ, p·V and the fused attention
+    are timed per launch; tokens/s counts every sequence's own tokens."""
+    import torch
+    w = synth.WORKLOADS[3]
+    B, H, T = w.batch, w.kv_heads, w.seq
+    nb = T // 128
+    kd, vd = upload(w, T, dev)
+    lens_blocks = np.random.default_rng(w.seed + 5).integers(32, nb + 1, B)
+    probe = pk.PackKVCache(B, H, nb, bits, ragged=True)
+    pk.packkv_encode_block(probe, kd, vd, nb)
+    k_lens = probe.k_index[..., 1].cpu().numpy().astype(np.int64)
+    v_lens = probe.v_index[..., 1].cpu().numpy().astype(np.int64)
+    used_k = sum(int(k_lens[b, :, :lens_blocks[b]].sum()) * 16 for b in range(B))
+    used_v = sum(int(v_lens[b, :, :lens_blocks[b]].sum()) * 16 for b in range(B))
+    del probe
+    R = copies_for(used_k)
+    caches = []
+    for _ in range(R):
+        c = pk.PackKVCache(B, H, nb, bits, ragged=True)
+        pk.packkv_encode_block(c, kd, vd, nb)
+        for b in range(B):
+            c._seq_blocks[b] = int(lens_blocks[b])
+        caches.append(c)
+    assert all(pk.packkv_get_status(c) == 0 for c in caches)
+    del kd, vd
+    Hq = w.q_heads
+    ld = T
+    q = [torch.from_numpy(synth.queries(w, i)).to(dev) for i in range(R)]
+    p = torch.from_numpy(synth.timing_probs(w, T)).to(dev)
+    scores = torch.empty((B, Hq, ld), dtype=torch.float32, device=dev)
+    out = torch.empty((B, Hq, 128), dtype=torch.float32, device=dev)
+    ws, wsa = caches[0].workspace(Hq), caches[0].attention_workspace(Hq)
+
+    def per_launch(fn):
+        g = capture(dev, lambda: [fn(i) for i in range(R)])
+        g.replay()
+        reps = max(1, int(np.ceil(60 / R)))
+        return timed_ms(dev, lambda: [g.replay() for _ in range(reps)]) / (reps * R)
+    qk_ms = per_launch(lambda i: pk.packkv_qk_gemv(caches[i], q[i], SCALE, scores))
+    pv_ms = per_launch(lambda i: pk.packkv_pv_gemv(caches[i], p, out, ws))
+    at_ms = per_launch(lambda i: pk.packkv_attention_decode(caches[i], q[i], SCALE, out, wsa))
+    tokens = int(lens_blocks.sum()) * 128
+    index_bytes = int(lens_blocks.sum()) * H * 8
+    fp16 = tokens * H * 128 * 2
+    qk_alg = used_k + index_bytes + B * Hq * 256 + int(lens_blocks.sum()) * 128 * Hq * 4
+    pv_alg = used_v + index_bytes + int(lens_blocks.sum()) * 128 * Hq * 4 + B * Hq * 512
+    del caches
+    return {"workload": "ragged batched b16 h32 d128 seq 4096..16384 per sequence 3-bit", "bits": bits,
+            "inputs": "i.i.d. (the workload's distributions)", "batch": B, "q_heads": Hq, "kv_heads": H,
+            "tokens": tokens, "seq_lengths": [int(x) * 128 for x in lens_blocks], "copies": R,
+            "qk": gemv_entry(qk_ms, used_k + index_bytes, qk_alg, fp16, tokens, peak),
+            "pv": gemv_entry(pv_ms, used_v + index_bytes, pv_alg, fp16, tokens, peak),
+            "attention": {"ms": at_ms, "tokens_per_s": tokens / (at_ms * 1e-3)},
+            "step_tokens_per_s": tokens / ((qk_ms + pv_ms) * 1e-3)}
+
+
+def speculative_record(pk, dev, peak, bits=4, S=4):
+    """Several queries per KV head: the GQA shape (32 query / 8 KV heads, 131k tokens)
+    decoding S = 4 draft positions at once, i.e. 16 query rows per KV head (two
+    launches of 8).  Per-launch-call times of q·Kᵀ, p·V and the fused attention over
+    the whole cache; tokens/s counts cache tokens x draft positions."""
+    import torch
+    w0 = synth.WORKLOADS[2]
+    w = synth.Workload(w0.name + " x4 draft positions", w0.batch, w0.q_heads * S, w0.kv_heads, w0.seq,
+                       (bits,), w0.seed)
+    rec = workload_record(pk, dev, 2, bits, peak, w_override=w)
+    rec["workload"] = f"speculative: gqa8b b1 hkv8 d128 seq131072, {S} draft positions x G=4 (16 rows per kv head)"
+    rec["tokens_per_s_x_positions"] = rec["step_tokens_per_s"] * S
+    return rec
+
+
 # ------------------------------------------------------------------ the CUDA path: the run
 def run_ours(args):
     import torch
@@ -457,8 +532,7 @@ def run_ours(args):
     bits = args.bits or w.bits[0]
     B, Hq, Hkv, T = w.batch, w.q_heads, w.kv_heads, w.seq
     nb = T // 128
-    kd, vd = upload(w, T, dev)
-    stream = torch.cuda.current_stream(dev)
+    kd, vd = upload(w, T, dev, structured=args.structured)
 
     # encoder throughput (prefill of the whole cache; fp16 bytes in)
     enc_cache = pk.PackKVCache(B, Hkv, nb, bits)
@@ -567,7 +641,8 @@ def run_ours(args):
         "metric": METRIC, "value": job_value(world, B * T, ms_per_step), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8xs8->s32 (tensor cores) + f32",
-        "data": "synthetic (seeded; K per-channel N(mu,sigma) with outlier channels, V N(0,1)); no weights needed",
+        "data": ("synthetic, run-structured (few levels per channel held for random runs)" if args.structured else
+                 "synthetic (seeded; K per-channel N(mu,sigma) with outlier channels, V N(0,1)); no weights needed"),
         "config": {"workload": w0.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": 128, "seq": T,
                    "bits": bits, "block_tokens": 128, "group_tokens": 32, "reorder_key": "k-code-sum",
                    "l2": f"inputs larger than L2: steps rotate over {R} packed-cache copies "
@@ -623,6 +698,10 @@ def run_ours(args):
         del kd2, vd2
         torch.cuda.empty_cache()
         subs.append(workload_record(pk, dev, 3, 3, hbm_peak))
+        torch.cuda.empty_cache()
+        subs.append(ragged_record(pk, dev, hbm_peak))
+        torch.cuda.empty_cache()
+        subs.append(speculative_record(pk, dev, hbm_peak))
         torch.cuda.empty_cache()
         for b in (2, 3, 4):
             subs.append(streaming_record(pk, dev, b))
@@ -745,6 +824,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true", help="headline workload only (no per-workload sub-records)")
+    ap.add_argument("--structured", action="store_true",
+                    help="run-structured inputs for the headline workload (compressed records; profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -128,12 +128,17 @@ EncodeArgs encode_args(const packkv_cache* c, const uint16_t* k, const uint16_t*
   return a;
 }
 
+// Query heads per kv head: 1, 2, 4 or 8 in one launch; 16, 32 or 64 (a wide group, or
+// several queries per kv head, e.g. speculative decoding) in launches of 8 heads each.
 bool group_ok(const packkv_cache* c, int32_t q_heads, int* group) {
   if (q_heads < 1 || q_heads % c->kv_heads != 0) return false;
   const int g = q_heads / c->kv_heads;
   *group = g;
-  return g == 1 || g == 2 || g == 4 || g == 8;
+  return g == 1 || g == 2 || g == 4 || g == 8 || g == 16 || g == 32 || g == 64;
 }
+
+constexpr int kMaxLaunchGroup = 8;  // query heads one launch serves
+int launch_group(int g) { return g < kMaxLaunchGroup ? g : kMaxLaunchGroup; }
 
 GemvArgs gemv_args(const packkv_cache* c, int group, const uint8_t* arena, const uint32_t* index,
                    const uint16_t* tail) {
@@ -143,7 +148,9 @@ GemvArgs gemv_args(const packkv_cache* c, int group, const uint8_t* arena, const
   a.tail = tail;
   a.batch = c->batch;
   a.kv_heads = c->kv_heads;
-  a.group = group;
+  a.group = launch_group(group);
+  a.g_total = group;
+  a.g_off = 0;
   a.max_blocks = c->max_blocks;
   a.n_blocks = c->n_blocks;
   a.tail_len = c->tail_len;
@@ -196,7 +203,7 @@ size_t packkv_workspace_bytes(const packkv_cache* cache, int32_t q_heads) {
   if (check_cache(cache) != PACKKV_OK) return 0;
   int g = 0;
   if (!group_ok(cache, q_heads, &g)) return 0;
-  return packkv::pv_workspace_bytes(cache->batch, cache->kv_heads, g);
+  return packkv::pv_workspace_bytes(cache->batch, cache->kv_heads, launch_group(g));
 }
 
 packkv_status packkv_cache_check(const packkv_cache* cache) { return check_cache(cache); }
@@ -332,7 +339,11 @@ packkv_status packkv_qk_gemv(const packkv_cache* cache, const uint16_t* q, int32
   a.scores = scores;
   a.ld = ld_scores;
   a.scale = scale;
-  return cuda_status(packkv::launch_qk(a, plan, as_stream(stream)));
+  for (a.g_off = 0; a.g_off < g; a.g_off += a.group) {
+    const cudaError_t e = packkv::launch_qk(a, plan, as_stream(stream));
+    if (e != cudaSuccess) return PACKKV_ERR_CUDA;
+  }
+  return PACKKV_OK;
 }
 
 packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t ld_p, int32_t q_heads, float* out,
@@ -348,7 +359,7 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
     const size_t bytes = (size_t)cache->batch * q_heads * PACKKV_HEAD_DIM * sizeof(float);
     return cuda_status(cudaMemsetAsync(out, 0, bytes, as_stream(stream)));
   }
-  const size_t need = packkv::pv_workspace_bytes(cache->batch, cache->kv_heads, g);
+  const size_t need = packkv::pv_workspace_bytes(cache->batch, cache->kv_heads, launch_group(g));
   if (!aligned16(ws) || ws_bytes < need) return PACKKV_ERR_INVALID_ARG;
   GemvArgs a = gemv_args(cache, g, cache->v_arena, cache->v_index, cache->v_tail);
   const RaggedPlan* plan = launch_plan(cache, a);
@@ -356,14 +367,18 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
   a.ld = ld_p;
   a.out = out;
   a.partials = reinterpret_cast<float*>(ws);
-  return cuda_status(packkv::launch_pv(a, plan, as_stream(stream)));
+  for (a.g_off = 0; a.g_off < g; a.g_off += a.group) {  // launches of one stream: ws is reused in turn
+    const cudaError_t e = packkv::launch_pv(a, plan, as_stream(stream));
+    if (e != cudaSuccess) return PACKKV_ERR_CUDA;
+  }
+  return PACKKV_OK;
 }
 
 size_t packkv_attention_workspace_bytes(const packkv_cache* cache, int32_t q_heads) {
   if (check_cache(cache) != PACKKV_OK) return 0;
   int g = 0;
   if (!group_ok(cache, q_heads, &g)) return 0;
-  return packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, g);
+  return packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, launch_group(g));
 }
 
 packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t* q, int32_t q_heads, float scale,
@@ -375,7 +390,7 @@ packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t*
   if (!group_ok(cache, q_heads, &g)) return PACKKV_ERR_UNSUPPORTED;
   const int64_t T = max_tokens(cache);
   if ((T == 0 && !is_ragged(cache)) || !aligned16(q) || !aligned16(out)) return PACKKV_ERR_INVALID_ARG;
-  const size_t need = packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, g);
+  const size_t need = packkv::attention_workspace_bytes(cache->batch, cache->kv_heads, launch_group(g));
   if (!aligned16(ws) || ws_bytes < need) return PACKKV_ERR_INVALID_ARG;
   AttnArgs a{};
   a.k_arena = cache->k_arena;
@@ -386,7 +401,8 @@ packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t*
   a.v_tail = cache->v_tail;
   a.batch = cache->batch;
   a.kv_heads = cache->kv_heads;
-  a.group = g;
+  a.group = launch_group(g);
+  a.g_total = g;
   a.max_blocks = cache->max_blocks;
   a.n_blocks = cache->n_blocks;
   a.tail_len = cache->tail_len;
@@ -402,7 +418,11 @@ packkv_status packkv_attention_decode(const packkv_cache* cache, const uint16_t*
   a.scale = scale;
   a.out = out;
   a.partials = reinterpret_cast<float*>(ws);
-  return cuda_status(packkv::launch_attention(a, plan, as_stream(stream)));
+  for (a.g_off = 0; a.g_off < g; a.g_off += a.group) {
+    const cudaError_t e = packkv::launch_attention(a, plan, as_stream(stream));
+    if (e != cudaSuccess) return PACKKV_ERR_CUDA;
+  }
+  return PACKKV_OK;
 }
 
 packkv_status packkv_get_status(const packkv_cache* cache, void* stream, uint32_t* bits_out) {

@@ -82,6 +82,8 @@ __device__ __forceinline__ GemvArgs tensor_view(const AttnArgs& a, bool v) {
   g.batch = a.batch;
   g.kv_heads = a.kv_heads;
   g.group = a.group;
+  g.g_total = a.g_total;
+  g.g_off = a.g_off;
   g.max_blocks = a.max_blocks;
   g.n_blocks = a.n_blocks;
   g.tail_len = a.tail_len;
@@ -226,7 +228,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, attn_min_ctas(BITS, G))
     mbar_init(m.bar(1), 1);
     fence_mbar_init();
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's results are visible
   __syncwarp();
   Cursor cc = cursor_at(a, plan, lo);
   EntryWindow wk, wv;
@@ -235,7 +236,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, attn_min_ctas(BITS, G))
   issue_item<BITS, G, false>(ka, m, cc, wk.get(lo), 0, lane);
   if (!kOneStage) issue_item<BITS, G, false>(va, m, cc, wv.get(lo), 1, lane);
 
-  const int q_heads = a.kv_heads * G;
   float qr[G][4];
   float mrun[G], lrun[G], mp[G];
   float acc_lo[NH][8], acc_hi[NH][8];
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, attn_min_ctas(BITS, G))
       cur_bh = bh;
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
-        const uint2 hv = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * q_heads + h * G + hd) * 128 + 4 * lane);
+        const uint2 hv = *reinterpret_cast<const uint2*>(a.q + head_row(a, b, h, hd) * 128 + 4 * lane);
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
         qr[hd][0] = f0.x;
@@ -463,14 +463,13 @@ constexpr int kMergeWarps = 32;
 template <int G, class Plan>
 __global__ void __launch_bounds__(kMergeWarps * 32)
     attn_merge_kernel(const AttnArgs a, const __grid_constant__ Plan plan) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 wsum[kMergeWarps][32];
   __shared__ float wl[kMergeWarps];
   __shared__ float wmax[kMergeWarps];
-  const long row = blockIdx.x;  // (b*kv_heads + h)*G + head
-  const long bh = row / G;
-  const int hd = (int)(row % G);
+  const long bh = blockIdx.x / G;  // block: (b*kv_heads + h)*G + head
+  const int hd = (int)(blockIdx.x % G);
+  const long row = (long)(head_row(a, bh / a.kv_heads, bh % a.kv_heads, hd));  // row of out
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   long first = 0, n = 0;
   row_items(a, plan, bh, &first, &n);
@@ -608,19 +607,8 @@ cudaError_t launch_attention_t(AttnArgs a, const Plan* plan, cudaStream_t stream
   if (a.n_warps < 1) a.n_warps = 1;
   const unsigned grid = (unsigned)((a.n_warps + kAttnWarps - 1) / kAttnWarps);
   void* args[] = {&a, const_cast<Plan*>(plan)};
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   if (a.n_items > 0) {
-    // a programmatic dependent of whatever precedes it (griddepcontrol.wait in the kernel)
-    cudaLaunchConfig_t lc{};
-    lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(kAttnWarps * 32);
-    lc.dynamicSmemBytes = (size_t)k.smem;
-    lc.stream = stream;
-    lc.attrs = pdl;
-    lc.numAttrs = 1;
-    e = cudaLaunchKernelExC(&lc, k.fn, args);
+    e = cudaLaunchKernel(k.fn, dim3(grid), dim3(kAttnWarps * 32), args, k.smem, stream);
     if (e != cudaSuccess) return e;
   }
   const void* merge = a.group == 1 ? merge_fn<1, Plan>() : a.group == 2 ? merge_fn<2, Plan>()

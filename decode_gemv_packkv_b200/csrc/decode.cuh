@@ -196,6 +196,13 @@ __device__ __forceinline__ void row_items(const A& a, const RaggedPlan& p, long 
   *first = p.base[b] + h * *n;
 }
 
+// Row of query head hd of (sequence b, kv head h) in q, scores, p and out: a launch
+// serves `group` of the g_total query heads of each kv head, from g_off on.
+template <class A>
+__device__ __forceinline__ size_t head_row(const A& a, long b, long h, int hd) {
+  return ((size_t)b * a.kv_heads + h) * a.g_total + a.g_off + hd;
+}
+
 // Index entry {offset16, length16} of block j of row bh: through the block table if the
 // cache has one (a physical block outside the index reads as an invalid entry).
 template <class A>
@@ -1151,7 +1158,7 @@ __device__ __forceinline__ void pv_tail(const GemvArgs& a, long bh, int nb, int 
     for (int sl = 0; sl < 4; ++sl) vv[sl] = half_bits_to_float(tail[(size_t)t * 128 + sl * 32 + lane]);
 #pragma unroll
     for (int hd = 0; hd < G; ++hd) {
-      const float pt = a.p[((size_t)b * a.kv_heads * G + h * G + hd) * a.ld + (long)nb * 128 + t];
+      const float pt = a.p[head_row(a, b, h, hd) * a.ld + (long)nb * 128 + t];
 #pragma unroll
       for (int sl = 0; sl < 4; ++sl) acc[sl][hd] = fmaf(pt, vv[sl], acc[sl][hd]);
     }

@@ -51,6 +51,7 @@ struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
   uint8_t cv[kBlockTokens][kHeadDim];  // V codes [token][channel]
   uint16_t kmin[kHeadDim], kscale[kHeadDim];     // per channel
   uint16_t vmin[kBlockTokens], vscale[kBlockTokens];  // per token (original order)
+  float krcp[kHeadDim], vrcp[kBlockTokens];      // 1 / scale (rounded), 0 for a zero scale
   float red[4][kEncodeThreads];        // min / max partials
   int key[kBlockTokens];
   int rank_part[kParts][kBlockTokens];
@@ -71,6 +72,17 @@ struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
 static_assert(sizeof(EncodeSmem) <= 113 * 1024, "two encoder CTAs per SM");
 
 __device__ __forceinline__ int bitlen(uint32_t x) { return x == 0 ? 0 : 32 - __clz(x); }
+
+// code = clamp(rint(fl(d / s)), 0, qmax) for d = fl(x - mn) >= 0 and scale s > 0, with
+// r = 1/s rounded to nearest.  q1 = fl(d * r) lies within 2^-18 of fl(d / s) (both are
+// within 2^-19 of d / s, which is below 16), so the two round to the same integer unless
+// fl(d / s) is within 2^-18 of a half-integer; then the correctly rounded quotient decides.
+__device__ __forceinline__ int quant_code(float d, float s, float r, int qmax) {
+  const float q1 = __fmul_rn(d, r);
+  const float h = __fsub_rn(__fsub_rn(q1, floorf(q1)), 0.5f);  // exact
+  const float y = fabsf(h) > 7.62939453125e-06f ? q1 : __fdiv_rn(d, s);  // 2^-17
+  return (int)fminf(fmaxf(rintf(y), 0.0f), (float)qmax);
+}
 
 // Where block t of the call goes: the index entry (u32 pair index) of its (sequence,
 // head, logical block) -- through the block table if the cache has one -- and the row of
@@ -251,35 +263,33 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     uint16_t sc = 0;
     if (range > 0.0f) sc = __half_as_ushort(__float2half_ru(__fdiv_rn(range, (float)qmax)));
     const uint16_t mnb = __half_as_ushort(__float2half_rn(lo));  // exact: lo is an fp16 value
+    const float rcp = sc ? __frcp_rn(half_bits_to_float(sc)) : 0.0f;
     if (is_k) {
       s.kmin[i] = mnb;
       s.kscale[i] = sc;
+      s.krcp[i] = rcp;
     } else {
       s.vmin[i] = mnb;
       s.vscale[i] = sc;
+      s.vrcp[i] = rcp;
     }
   }
   __syncthreads();
 
   // ---- codes -----------------------------------------------------------------
-  for (int e = tid; e < kBlockTokens * kHeadDim; e += blockDim.x) {
-    const int t = e >> 7, c = e & 127;
-    {
-      const float sc = half_bits_to_float(s.kscale[c]);
+  // A thread keeps one channel (its K parameters in registers) and walks tokens.
+  {
+    static_assert(kEncodeThreads % kHeadDim == 0, "a thread keeps its channel");
+    const int c = tid & (kHeadDim - 1);
+    const float kmn = half_bits_to_float(s.kmin[c]), ksc = half_bits_to_float(s.kscale[c]), kr = s.krcp[c];
+    for (int t = tid >> 7; t < kBlockTokens; t += kEncodeThreads / kHeadDim) {
       int code = 0;
-      if (sc > 0.0f) {
-        const float y = __fdiv_rn(__fsub_rn(__half2float(s.kx[t][c]), half_bits_to_float(s.kmin[c])), sc);
-        code = (int)fminf(fmaxf(rintf(y), 0.0f), (float)qmax);
-      }
+      if (ksc > 0.0f) code = quant_code(__fsub_rn(__half2float(s.kx[t][c]), kmn), ksc, kr, qmax);
       s.ck[t][c] = (uint8_t)code;
-    }
-    {
-      const float sc = half_bits_to_float(s.vscale[t]);
-      int code = 0;
-      if (sc > 0.0f) {
-        const float y = __fdiv_rn(__fsub_rn(__half2float(s.vx[t][c]), half_bits_to_float(s.vmin[t])), sc);
-        code = (int)fminf(fmaxf(rintf(y), 0.0f), (float)qmax);
-      }
+      const float vsc = half_bits_to_float(s.vscale[t]);
+      code = 0;
+      if (vsc > 0.0f)
+        code = quant_code(__fsub_rn(__half2float(s.vx[t][c]), half_bits_to_float(s.vmin[t])), vsc, s.vrcp[t], qmax);
       s.cv[t][c] = (uint8_t)code;
     }
   }

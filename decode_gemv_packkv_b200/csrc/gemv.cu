@@ -58,7 +58,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G))
     qk_kernel(const GemvArgs a, const __grid_constant__ Plan plan) {
   using C = Cfg<BITS, G, false>;
   extern __shared__ __align__(128) unsigned char smem[];
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int warp = blockIdx.x * kWarpsPerCta + (threadIdx.x >> 5);
   if (warp >= a.n_warps) return;
@@ -69,9 +68,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G))
     for (int s = 0; s < C::kStages; ++s) mbar_init(m.bar(s), 1);
     fence_mbar_init();
   }
-  // launched as a programmatic dependent: everything above overlapped the previous
-  // kernel's tail; its results are visible after this wait
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncwarp();
   long prod = lo;
   Cursor pc = cursor_at(a, plan, lo);
@@ -81,7 +77,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G))
   for (int s = 0; s < C::kStages && prod < hi; ++s, ++prod, cursor_next(a, plan, pc))
     issue_item<BITS, G, false>(a, m, pc, win.get(prod), s, lane);
 
-  const int q_heads = a.kv_heads * G;
   long cur_bh = -1;
   float qr[G][4];
   uint32_t phases = 0;
@@ -90,12 +85,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, qk_min_ctas(BITS, G))
     const long bh = cc.bh;
     const int j = cc.j;
     const long b = bh / a.kv_heads, h = bh % a.kv_heads;
-    float* srow0 = a.scores + ((size_t)b * q_heads + h * G) * a.ld;
+    float* srow0 = a.scores + head_row(a, b, h, 0) * a.ld;
     if (bh != cur_bh) {
       cur_bh = bh;
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
-        const uint2 hv = *reinterpret_cast<const uint2*>(a.q + ((size_t)b * q_heads + h * G + hd) * 128 + 4 * lane);
+        const uint2 hv = *reinterpret_cast<const uint2*>(a.q + head_row(a, b, h, hd) * 128 + 4 * lane);
         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
         qr[hd][0] = f0.x;
@@ -233,12 +228,11 @@ __device__ __forceinline__ void add4(float4& s, const float4 x) {
 template <int G, class Plan>
 __global__ void __launch_bounds__(kReduceWarps * 32)
     pv_reduce_kernel(const GemvArgs a, const __grid_constant__ Plan plan) {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float4 warp_sum4[kReduceWarps][32];
-  const long row = blockIdx.x;  // (b*kv_heads + h)*G + head
-  const long bh = row / G;
-  const int hd = (int)(row % G);
+  const long bh = blockIdx.x / G;  // block: (b*kv_heads + h)*G + head
+  const int hd = (int)(blockIdx.x % G);
+  const long row = (long)(head_row(a, bh / a.kv_heads, bh % a.kv_heads, hd));  // row of out
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   long first = 0, n = 0;
   row_items(a, plan, bh, &first, &n);
@@ -293,7 +287,6 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
     for (int s = 0; s < C::kStages; ++s) mbar_init(m.bar(s), 1);
     fence_mbar_init();
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's results are visible
   __syncwarp();
   long prod = lo;
   Cursor pc = cursor_at(a, plan, lo);
@@ -305,7 +298,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
   auto load_p = [&](const Cursor& c) {
     if (c.j < c.nb) {
       const long b = c.bh / a.kv_heads, h = c.bh % a.kv_heads;
-      const float* prow = a.p + ((size_t)b * a.kv_heads * G + h * G) * a.ld + (size_t)c.j * 128;
+      const float* prow = a.p + head_row(a, b, h, 0) * a.ld + (size_t)c.j * 128;
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) pn[hd] = __ldcs(reinterpret_cast<const float4*>(prow + hd * a.ld) + lane);
     }
@@ -487,20 +480,8 @@ cudaError_t launch(GemvArgs a, const Plan* plan, cudaStream_t stream) {
   if (a.n_warps < 1) a.n_warps = 1;
   const unsigned grid = (unsigned)((a.n_warps + kWarpsPerCta - 1) / kWarpsPerCta);
   void* args[] = {&a, const_cast<Plan*>(plan)};
-  cudaLaunchAttribute pdl[1];
-  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  pdl[0].val.programmaticStreamSerializationAllowed = 1;
   if (a.n_items > 0) {
-    // a programmatic dependent of whatever precedes it: the kernel waits for that
-    // kernel's results before its first global access (griddepcontrol.wait)
-    cudaLaunchConfig_t lc{};
-    lc.gridDim = dim3(grid);
-    lc.blockDim = dim3(kWarpsPerCta * 32);
-    lc.dynamicSmemBytes = (size_t)info.smem;
-    lc.stream = stream;
-    lc.attrs = pdl;
-    lc.numAttrs = 1;
-    e = cudaLaunchKernelExC(&lc, info.fn, args);
+    e = cudaLaunchKernel(info.fn, dim3(grid), dim3(kWarpsPerCta * 32), args, info.smem, stream);
     if (e != cudaSuccess || !PV) return e;
   } else if (!PV) {
     return cudaSuccess;

@@ -59,6 +59,7 @@ struct GemvArgs {
   const uint32_t* index;  // [batch][kv_heads][max_blocks][2]
   const uint16_t* tail;   // [batch][kv_heads][128][128] fp16
   int batch, kv_heads, group, max_blocks, n_blocks, tail_len, bits;
+  int g_total, g_off;     // query heads per kv head, and the first one this launch serves
   uint64_t arena16;       // arena_bytes / 16
   uint64_t* ctrl;
   long n_items;           // batch*kv_heads*items_per_bh
@@ -96,6 +97,7 @@ struct AttnArgs {
   const uint16_t* k_tail;   // [batch][kv_heads][128][128] fp16
   const uint16_t* v_tail;
   int batch, kv_heads, group, max_blocks, n_blocks, tail_len, bits;
+  int g_total, g_off;       // query heads per kv head, and the first one this launch serves
   uint64_t arena16;         // arena_bytes / 16
   uint64_t* ctrl;
   long n_items;             // batch*kv_heads*items_per_bh

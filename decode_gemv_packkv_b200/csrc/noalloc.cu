@@ -73,6 +73,8 @@ packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, 
   a.batch = cache->batch;
   a.kv_heads = cache->kv_heads;
   a.group = g;
+  a.g_total = g;
+  a.g_off = 0;
   a.max_blocks = cache->max_blocks;
   a.n_blocks = cache->n_blocks;
   a.tail_len = cache->tail_len;

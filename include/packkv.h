@@ -182,7 +182,10 @@ packkv_status packkv_append_token_masked(packkv_cache* cache, const uint16_t* k,
  * scores[b][hq][i] = scale * sum_c q[b][hq][c] * k_hat[b][hq/G][i][c]  (fp32 accumulate)
  * over the packed blocks in storage order, then the tail in arrival order
  * (packed-cache format v1, sections 6-7; paper page Figure 1, Figure 2 fused decompression).
- *   q:      device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8}.
+ *   q:      device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8,16,32,64}.
+ *           G > 8 runs as G/8 launches of 8 query heads (the cache is read G/8 times).
+ *           Several queries per kv head in one step (speculative decoding) are such a
+ *           group: the S queries of the G heads of kv head h are rows h*S*G .. +S*G-1.
  *   scores: device fp32, row (b, hq) starts at (b*q_heads + hq) * ld_scores;
  *           ld_scores >= T = n_blocks*128 + tail_len (ragged: the longest sequence),
  *           multiple of 4.
@@ -231,7 +234,7 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
  * All calls share the one array, and it keeps the last call's partials: calls
  * that overlap in time on the GPU race.  Nothing in it needs clearing (every
  * partial is written before it is read).  With T == 0, out is set to zero.
- * A ragged cache or one with a block table: PACKKV_ERR_UNSUPPORTED.
+ * A ragged cache, one with a block table, or G above 8: PACKKV_ERR_UNSUPPORTED.
  */
 #define PACKKV_PV_NOALLOC_SCRATCH_BYTES (8u << 20)
 packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, int64_t ld_p,
@@ -246,7 +249,8 @@ packkv_status packkv_pv_gemv_noalloc(const packkv_cache* cache, const float* p, 
  * reach global memory; the softmax is computed online (a running maximum and
  * sum of exponentials per warp), split over the sequence and merged with the
  * log-sum-exp rule by a second kernel in a fixed order (deterministic).
- *   q:   device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8}.
+ *   q:   device fp16 [batch][q_heads][128]; q_heads = G * kv_heads, G in {1,2,4,8,16,32,64}
+ *        (as for packkv_qk_gemv).
  *   out: device fp32 [batch][q_heads][128].
  *   ws:  device, ws_bytes >= packkv_attention_workspace_bytes(cache, q_heads)
  *        (no initialisation needed; two calls sharing ws must not overlap in time).

@@ -26,6 +26,8 @@ def assert_within_terms(gpu: np.ndarray, ref: np.ndarray, abs_terms: np.ndarray,
         raise AssertionError(f"{what}: {int(bad.sum())} elements out of tolerance, e.g. "
                              + ", ".join(f"{tuple(i)}: gpu={gpu[tuple(i)]:.9g} ref={ref[tuple(i)]:.9g} "
                                          f"bound={bound[tuple(i)]:.3g}" for i in idx))
+    if err.size == 0:
+        return 0.0
     return float(np.max(np.where(abs_terms > 0, err / np.maximum(abs_terms, 1e-300), 0.0)))
 
 
