@@ -55,11 +55,18 @@ struct I8Layout {
   }
 };
 
+// p·V records in flight per warp.  With one, p of the record in flight waits in
+// registers; with more, each stage also holds its record's p slices (bulk-copied with it).
+#ifndef PACKKV_PV_STAGES
+#define PACKKV_PV_STAGES 1
+#endif
+
 template <int BITS, int G, bool PV>
 struct Cfg {
   static constexpr int kRecBytes = raw_record_bytes(BITS);
   static constexpr int kStageRec = kRecBytes;                  // >= every record, staged in one piece
-  static constexpr int kStageBytes = kStageRec;
+  static constexpr bool kStagedP = PV && PACKKV_PV_STAGES > 1;  // p slices [G][128] fp32 after the record
+  static constexpr int kStageBytes = kStageRec + (kStagedP ? 512 * G : 0);
   // int8 tensor-core B table: columns n = 4*head + digit (digit 3 = 0), NT n-tiles of 8
   static constexpr int kNT = I8Layout<G>::kNT;
   static constexpr int kNH = I8Layout<G>::kNH;
@@ -68,8 +75,7 @@ struct Cfg {
   static constexpr int kSumBytes = PV ? 512 * G : 0;          // p·V: [G][128] channel sums
   static constexpr int kFixed = kTableBytes + kSumBytes;
   static constexpr int kStages0 = (kWarpSmemBudget - kFixed - 64) / kStageBytes;
-  // p·V keeps the p of its in-flight record in registers, one record deep: one stage
-  static constexpr int kStages = PV ? 1 : (kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0));
+  static constexpr int kStages = PV ? PACKKV_PV_STAGES : (kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0));
   static constexpr int kWarpSmem = ((kStages * kStageBytes + kFixed + kStages * 16) + 127) / 128 * 128;
   static_assert(kStageBytes % 16 == 0 && kFixed % 16 == 0, "stage alignment");
 };
@@ -262,11 +268,13 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, cons
   }
   unsigned char* st = m.stage(s);
   const unsigned char* src = a.arena + off16 * 16;
+  const bool with_p = C::kStagedP && (kind == kKindRaw || kind == kKindPacked);
   if (lane == 0) {
     *m.kind(s) = kind | (int)(len16 << 8);  // kind in bits 0..7, record length (16-B units) above
     uint32_t bytes = 0;
     if (kind == kKindRaw) bytes = C::kRecBytes;
     if (kind == kKindPacked) bytes = len16 * 16u;
+    if (with_p) bytes += 512u * G;
     fence_async_smem();
     if (bytes)
       mbar_arrive_expect_tx(m.bar(s), bytes);
@@ -278,6 +286,11 @@ __device__ __forceinline__ void issue_item(const GemvArgs& a, const Mem& m, cons
     if (lane == 16) bulk_g2s(st, src, C::kRecBytes, m.bar(s));
   } else if (kind == kKindPacked) {
     if (lane == 16) bulk_g2s(st, src, len16 * 16u, m.bar(s));
+  }
+  if (with_p && lane < G) {  // the record's p slices: 128 fp32 of each query head
+    const long b = c.bh / a.kv_heads, h = c.bh % a.kv_heads;
+    const float* prow = a.p + head_row(a, b, h, lane) * a.ld + (size_t)c.j * 128;
+    bulk_g2s(st + C::kStageRec + 512 * lane, prow, 512u, m.bar(s));
   }
 }
 

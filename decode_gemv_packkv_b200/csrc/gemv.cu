@@ -303,12 +303,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
       for (int hd = 0; hd < G; ++hd) pn[hd] = __ldcs(reinterpret_cast<const float4*>(prow + hd * a.ld) + lane);
     }
   };
-  static_assert(C::kStages == 1, "one record in flight per warp");
-  if (prod < hi) {
-    issue_item<BITS, G, true>(a, m, pc, win.get(prod), 0, lane);
-    load_p(pc);
-    ++prod;
-    cursor_next(a, plan, pc);
+  for (int s0 = 0; s0 < C::kStages && prod < hi; ++s0, ++prod, cursor_next(a, plan, pc)) {
+    issue_item<BITS, G, true>(a, m, pc, win.get(prod), s0, lane);
+    if (!C::kStagedP) load_p(pc);
   }
 
   float mp[G];  // sum over the warp's records of p * mn (lane: slots 4*lane .. +3)
@@ -358,7 +355,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
       float mpr[G];
 #pragma unroll
       for (int hd = 0; hd < G; ++hd) {
-        const float4 p4 = pn[hd];
+        const float4 p4 = C::kStagedP ? reinterpret_cast<const float4*>(st + C::kStageRec + 512 * hd)[lane] : pn[hd];
         const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
         mpr[hd] = 0.f;
 #pragma unroll
@@ -387,7 +384,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
     if (prod < hi) {
       if (prod - win.base >= 32) win.load(a, plan, prod, hi, lane);
       issue_item<BITS, G, true>(a, m, pc, win.get(prod), s, lane);
-      load_p(pc);
+      if (!C::kStagedP) load_p(pc);
       ++prod;
       cursor_next(a, plan, pc);
     }

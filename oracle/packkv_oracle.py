@@ -393,6 +393,49 @@ def parse_record(rec: bytes) -> ParsedRecord:
 
 
 # ----------------------------------------------------------------------------
+# Format variants, for the compression ablation only ([Fig. 2] step 2 and [Fig. 3]:
+# the packing exploits quantized codes that concentrate on few values).  The
+# library writes format v1 (frame-of-reference units, fp16 parameters, one meta
+# byte per unit); these give the record size the alternatives would have.
+# ----------------------------------------------------------------------------
+VARIANT_V1 = "v1"                      # frame of reference (base = min), fp16 params, 8-bit meta
+VARIANT_WIDTH_ONLY = "width-only"      # no base: w = bitlen(max code), meta holds w only
+VARIANT_FP32_PARAMS = "fp32-params"    # min and scale stored as fp32 (1024 B instead of 512)
+VARIANT_META4 = "meta4"                # b = 2: base and width in 2 bits each, 4-bit meta (256 B)
+
+
+def record_bytes_variant(codes_slot: np.ndarray, bits: int, variant: str) -> int:
+    """Bytes of one record of codes [slot, channel] under a format variant: the packed
+    size, or the raw size of that variant when packing does not make it smaller."""
+    codes_slot = np.asarray(codes_slot, dtype=np.int64)
+    params = 1024 if variant == VARIANT_FP32_PARAMS else 512
+    meta = 256 if variant == VARIANT_META4 else 512
+    if variant == VARIANT_META4 and bits != 2:
+        raise ValueError("the 4-bit meta variant is for 2-bit codes")
+    wsum = 0
+    for g in range(GROUPS_PER_BLOCK):
+        for c in range(HEAD_DIM):
+            unit = codes_slot[32 * g:32 * g + 32, c]
+            if variant == VARIANT_WIDTH_ONLY:
+                wsum += int(unit.max()).bit_length()
+            else:
+                wsum += unit_base_width(unit)[1]
+    packed = _ceil16(16 + params + meta + 4 * wsum)
+    raw = 16 + params + 2048 * bits
+    return min(packed, raw)
+
+
+def block_codes(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int = KEY_K_SUM):
+    """Codes of one block in storage order (K [slot, channel], V [slot, channel])."""
+    ck, _, _ = quantize_block_k(k_blk, bits)
+    cv, _, _ = quantize_block_v(v_blk, bits)
+    rank = stable_rank(reorder_keys(ck, cv, key_kind))
+    perm = np.empty(BLOCK_TOKENS, dtype=np.int64)
+    perm[rank] = np.arange(BLOCK_TOKENS)
+    return ck[perm], cv[perm]
+
+
+# ----------------------------------------------------------------------------
 # One block: quantize -> reorder -> pack
 # ----------------------------------------------------------------------------
 def encode_block(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int = KEY_K_SUM):
