@@ -669,7 +669,8 @@ def ragged_attention(cache: RaggedOracleCache, q: np.ndarray, scale: float):
     p = np.zeros_like(scores)
     for b in range(B):
         Tb = cache.seq_tokens(b)
-        p[b, :, :Tb] = softmax(scores[b, :, :Tb])
+        if Tb:  # a sequence with no tokens attends to nothing: its output is zero
+            p[b, :, :Tb] = softmax(scores[b, :, :Tb])
     return ragged_pv(cache, p)
 
 

@@ -140,3 +140,20 @@ def test_ragged_products_reduce_to_uniform_products():
         assert np.array_equal(o[b:b + 1], uo)
         ua, _ = O.cache_attention(u, q[b:b + 1], SCALE)
         assert np.allclose(a[b:b + 1], ua, rtol=0, atol=1e-12)
+
+
+def test_empty_sequence_attends_to_nothing():
+    """A sequence that never took a token has zero attention output (an empty softmax
+    weights nothing); the other sequences are unaffected."""
+    B, H, bits = 2, 2, 4
+    k, v = _streams(B, H, 140, 23)
+    r = O.RaggedOracleCache(B, H, 2, bits)
+    for t in range(140):
+        r.append_token_ragged(k[:, :, t], v[:, :, t], active=[0])
+    assert r.seq_tokens(1) == 0
+    q = np.random.default_rng(3).standard_normal((B, H, 128)).astype(np.float16)
+    a, terms = O.ragged_attention(r, q, SCALE)
+    assert np.array_equal(a[1], np.zeros((H, 128))) and np.array_equal(terms[1], np.zeros((H, 128)))
+    u = _uniform_of(k[0], v[0], 140, bits, 2)
+    ua, _ = O.cache_attention(u, q[:1], SCALE)
+    assert np.allclose(a[:1], ua, rtol=0, atol=1e-12)
