@@ -51,7 +51,7 @@ struct AttnCfg {
   static constexpr int kI8Tab = C::kI8Tab;
   static constexpr int kTableBytes = (kI8Tab + 15) / 16 * 16;
   static constexpr int kScoreBytes = 512 * G;  // [G][128] scores, then probabilities
-  static constexpr int kSumBytes = 512 * G;    // [G][128] channel sums (CUDA-core and tail paths)
+  static constexpr int kSumBytes = 512 * G;    // [G][128] channel sums (compressed records and the tail)
   static constexpr int kFixed = kAttnStages * kStageRec + kTableBytes + kScoreBytes + kSumBytes;
   static constexpr int kWarpSmem = (kFixed + 32 + 127) / 128 * 128;
   static_assert(kStageRec % 16 == 0 && kFixed % 16 == 0, "stage alignment");
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, attn_min_ctas(BITS, G))
       if (kind_v == kKindRaw)
         pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
       else
-        ok = pv_packed_tc<BITS, G>(st, (uint32_t)(kind_len_v >> 8) * 16u, tab, pv4, invf, sacc, lane);
+        ok = pv_packed_nat<BITS, G>(st, (uint32_t)(kind_len_v >> 8) * 16u, tab, invf, sacc, lane);
       if (ok) {
 #pragma unroll
         for (int hd = 0; hd < G; ++hd) mp[hd] += mpr[hd];

@@ -1,8 +1,8 @@
 // Device building blocks of the fused decode products over the packed cache:
 // record staging (bulk copies into warp-private shared-memory stages, bounded
 // mbarrier waits), the 8-bit integer tensor-core decode of raw records (2, 3 and
-// 4-bit) and of compressed records (units sorted by width; packed-cache format v1,
-// sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused attention kernel.
+// 4-bit) and of compressed records (q·Kᵀ: units sorted by width; p·V: every slice
+// kind decoded and masked by width; packed-cache format v1, sections 3-4).  Included by the q·Kᵀ / p·V kernels and by the fused attention kernel.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -688,21 +688,22 @@ __device__ __forceinline__ void pv_i8(const unsigned char* st, const uint32_t* t
 // ----------------------------------------------------------------------------
 // A compressed unit (pack group g, channel c) holds the 32 offsets of its slots in w
 // words: power-of-two slices of 4, 2 and 1 bits (packed-cache format v1, section 3).
-// A tensor-core A register takes four codes, so lanes must decode units with the same
-// instructions: the units of a group are sorted by width (classes 4, 3, 2, 1; a unit of
-// width 0 carries only its base and is left out), each class padded with dummy units to
-// a multiple of 16, and every run of 16 sorted units then has one width.
-//  * q·Kᵀ: a run is one k half (16 channels) of an m16n8k32 product.  Lane (g8, t) takes
-//    the channels at run positions 4t..4t+3 and slots 4g8..4g8+3 of the group (rows g8 and
-//    g8 + 8 of the group's two 16-slot tiles), joins the four units' slot runs with byte
-//    permutes and separates the codes with masks.  The B operand (q' digits, in natural
-//    channel order in the table of build_i8tab) is gathered through the sort.
-//  * p·V: a run is one 16-row tile (rows = channels, k = the group's 32 slots).  Lane t
-//    decodes 8 slots of two units with shifts and masks.  The rows change from group to
-//    group, so a group's tile results are added into the warp's channel sums.
-// The sorted descriptors (word start | tag << 16) live in the stage: the prologue reads
-// the record's meta into registers, after which bytes [0, 1040) of the stage (header,
-// params, meta) are free.  Words [1024, 1040) are zeroed; a dummy unit starts there
+// A tensor-core register takes four codes, and lanes must decode with the same
+// instructions whatever the widths of their units:
+//  * q·Kᵀ (contraction over channels): a register holds four channels of one slot, so
+//    four units are joined per register.  The units of a group are sorted by width
+//    (classes 4, 3, 2, 1; a unit of width 0 carries only its base and is left out), each
+//    class padded with dummy units to a multiple of 16, so every run of 16 sorted units
+//    has one width and is one k half (16 channels) of an m16n8k32 product.  Lane (g8, t)
+//    takes the channels at run positions 4t..4t+3 and slots 4g8..4g8+3 of the group (rows
+//    g8 and g8 + 8 of the group's two 16-slot tiles), joins the four units' slot runs with
+//    byte permutes and separates the codes with masks.  The B operand (q' digits, in
+//    natural channel order in the table of build_i8tab) is gathered through the sort.
+//  * p·V (contraction over slots, along the units): natural channel order, every slice
+//    kind decoded by every lane and masked by the unit's width (pv_packed_nat).
+// The prologue reads the record's meta into registers, after which bytes [0, 1040) of
+// the stage (header, params, meta) are free for descriptors.  q·Kᵀ: sorted descriptors
+// (word start | tag << 16); words [1024, 1040) are zeroed and a dummy unit starts there
 // (word index -4 of the word area), so it decodes to zero codes.
 constexpr int kZeroUnitStart = -4;
 
@@ -986,55 +987,12 @@ __device__ __forceinline__ void qk_tail(const GemvArgs& a, long bh, int nb, int 
   }
 }
 
-// p·V: A registers (rows = two units, k = the group's 32 slots) of lane t from a unit
-// of width W starting at word s.  The k position (kh, t, e) of a register holds
-//   slot 8t + 2e + kh  (order A: one word per lane for the 4-bit slice), or
-//   slot t + 8e + 4kh  (order B: one shift and mask per register for 2- and 1-bit slices).
-// a[0] / a[1]: the kh = 0 / kh = 1 registers.
-template <int W, bool kOrderA>
-__device__ __forceinline__ void pv_unit(const uint32_t* words, int s, int t, uint32_t (&a)[2]) {
-  if constexpr (kOrderA) {
-    if constexpr (W == 4) {
-      const uint32_t x = words[s + t];  // slots 8t .. 8t+7, a nibble each
-      a[0] = x & 0x0F0F0F0Fu;
-      a[1] = (x >> 4) & 0x0F0F0F0Fu;
-    } else {
-      uint32_t r0 = 0u, r1 = 0u;
-      if constexpr (W == 2 || W == 3) {  // slots 8t .. 8t+7: bits 16(t & 1) .. +15 of word t >> 1
-        const uint32_t z = __byte_perm(words[s + (t >> 1)], 0u, (t & 1) ? 0x3322u : 0x1100u);
-        r0 = (z & 0x00030003u) | ((z >> 4) & 0x03000300u);
-        r1 = ((z >> 2) & 0x00030003u) | ((z >> 6) & 0x03000300u);
-      }
-      if constexpr (W == 1 || W == 3) {  // slots 8t .. 8t+7: byte t; bit 2e -> byte e by one multiply
-        const uint32_t x = words[s + (W == 3 ? 2 : 0)] >> (8 * t);
-        const uint32_t b0 = ((x & 0x55u) * 0x41041u) & 0x01010101u;
-        const uint32_t b1 = (((x >> 1) & 0x55u) * 0x41041u) & 0x01010101u;
-        r0 |= W == 3 ? b0 << 2 : b0;
-        r1 |= W == 3 ? b1 << 2 : b1;
-      }
-      a[0] = r0;
-      a[1] = r1;
-    }
-  } else {
-    static_assert(W != 4, "order B serves widths 1 to 3");
-    uint32_t r0 = 0u, r1 = 0u;
-    if constexpr (W == 2 || W == 3) {  // slot t + 8e + 4kh: byte 2(e & 1) + kh of word e >> 1, bits 2t
-      const uint32_t w0 = words[s], w1 = words[s + 1];
-      r0 = (__byte_perm(w0, w1, 0x6420u) >> (2 * t)) & 0x03030303u;
-      r1 = (__byte_perm(w0, w1, 0x7531u) >> (2 * t)) & 0x03030303u;
-    }
-    if constexpr (W == 1 || W == 3) {  // bit t + 8e + 4kh
-      const uint32_t x = words[s + (W == 3 ? 2 : 0)] >> t;
-      const uint32_t b0 = x & 0x01010101u, b1 = (x >> 4) & 0x01010101u;
-      r0 |= W == 3 ? b0 << 2 : b0;
-      r1 |= W == 3 ? b1 << 2 : b1;
-    }
-    a[0] = r0;
-    a[1] = r1;
-  }
-}
+// p·V k orders: the k position (kh, t, e) of an A or B register of lane t (kh: the
+// register's k half, e: its byte) holds
+//   slot 8t + 2e + kh  (order A: a 4-bit slice gives a register per mask of word t), or
+//   slot t + 8e + 4kh  (order B: 2- and 1-bit slices give a register per shift and mask).
 
-// B fragments of group g in the two k orders of pv_unit, gathered from the int8 B table
+// B fragments of group g in the two k orders, gathered from the int8 B table
 // of p' (build_i8tab, natural slot order: byte k & 3 of word i8tab_word(k >> 5,
 // (k >> 4) & 1, (k >> 2) & 3, n) holds slot k).  bA/bB[kh][j] for n-tile j.
 template <int NT>
@@ -1060,97 +1018,128 @@ __device__ __forceinline__ void pv_group_frags(const uint32_t* tab, int g, int l
   }
 }
 
-// One 16-unit run of width W as a p·V tile: rows g8 / g8 + 8 = the units at run positions
-// g8 / g8 + 8; adds each row's products, digits joined and times invf, into sacc (the
-// warp's [G][128] channel sums).
-template <int W, int G>
-__device__ __forceinline__ void pv_run(const uint32_t* words, const uint32_t* desc, int blk,
-                                       const uint32_t (&bA)[2][I8Layout<G>::kNT],
-                                       const uint32_t (&bB)[2][I8Layout<G>::kNT], const float (&f_t)[I8Layout<G>::kNH],
-                                       const PairW& pw, float* sacc, int lane) {
-  using L = I8Layout<G>;
-  constexpr int NT = L::kNT;
-  constexpr bool kA = W == 4;
-  const int g8 = lane >> 2, t = lane & 3;
-  const uint32_t dlo = desc[16 * blk + g8], dhi = desc[16 * blk + 8 + g8];
-  uint32_t alo[2], ahi[2];
-  pv_unit<W, kA>(words, desc_start(dlo), t, alo);
-  pv_unit<W, kA>(words, desc_start(dhi), t, ahi);
-  const uint32_t a[4] = {alo[0], ahi[0], alo[1], ahi[1]};
-  int d[NT][4];
-#pragma unroll
-  for (int j = 0; j < NT; ++j) {
-    d[j][0] = d[j][1] = d[j][2] = d[j][3] = kRoundBits;
-    imma16832(d[j], a, kA ? bA[0][j] : bB[0][j], kA ? bA[1][j] : bB[1][j]);
-  }
-  const uint32_t clo = dlo >> 16, chi = dhi >> 16;  // channels (0xFFFF: dummy)
-  auto emit = [&](int, int jh, float lo, float hi) {
-    if (L::owns(jh, t)) {
-      float* row = sacc + L::head(jh, t) * 128;
-      if (clo < 128u) row[clo] = fmaf(lo, f_t[jh], row[clo]);
-      if (chi < 128u) row[chi] = fmaf(hi, f_t[jh], row[chi]);
-    }
-  };
-  emit_tile<G>(0, d, 1.f, 1.f, pw, emit);
+// p·V in natural channel order.  Row tile T = channels 16T .. 16T+15 (the tiles of raw
+// records), k-step g = pack group g.  Every lane decodes its two units of a tile with
+// the same instructions whatever their widths: a 4-bit slice in k order A,
+// the 2- and 1-bit slices and the unit's base in k order B, a slice the unit lacks
+// masked to zero.  Two products per tile, one per order, add into the same
+// accumulators, so a tile ends with sum_r p'_r (base + offset) of its channels.  No
+// sort: every tile's rows are fixed channels.
+//
+// Descriptor of unit (g, c): group-relative word start | width << 9 | base << 12 (the
+// start is at most 127 * 4, the base at most 15); word 64g + 8T + (c & 7) of the stage's
+// free bytes holds channel 16T + (c & 7) in its low half and channel 16T + (c & 7) + 8
+// in its high half, so a lane reads both of its rows with one load.  The loads do not
+// depend on the width (no divergence); a word read past a unit's end still lies in the
+// staged record or the stage's slack (a compressed record is at least 16 bytes shorter
+// than a raw one) and is masked off.
+#ifndef PACKKV_NAT_FRAG_NT
+#define PACKKV_NAT_FRAG_NT 2
+#endif
+__device__ __forceinline__ void pv_nat_unit(const uint32_t* words, int gs, uint32_t dsc, int t, uint32_t& a0,
+                                            uint32_t& a1, uint32_t& b0, uint32_t& b1) {
+  const int s = gs + (int)(dsc & 511u);
+  const uint32_t w = (dsc >> 9) & 7u;
+  const uint32_t bb = (dsc >> 12) * 0x01010101u;
+  const uint32_t m4 = w == 4u ? 0x0F0F0F0Fu : 0u;
+  const uint32_t m2 = (w & 2u) ? 0x03030303u : 0u;
+  const uint32_t m1 = (w & 1u) ? 0x01010101u : 0u;
+  const uint32_t x4 = words[s + t];  // 4-bit slice: slots 8t .. 8t+7, a nibble each
+  const uint32_t x20 = words[s], x21 = words[s + 1];  // 2-bit slice: bits 0-1 of the offsets
+  const uint32_t x1 = words[s + (int)(w & 2u)];       // 1-bit slice: bit 0 (width 1) or bit 2 (width 3)
+  a0 = x4 & m4;
+  a1 = (x4 >> 4) & m4;
+  const uint32_t k1 = (w & 2u) ? 4u : 1u;
+  const uint32_t y = x1 >> t;  // bit t + 8e + 4kh -> bit 8e (kh = 0) / 8e + 4 (kh = 1)
+  b0 = ((__byte_perm(x20, x21, 0x6420u) >> (2 * t)) & m2) + (y & m1) * k1 + bb;
+  b1 = ((__byte_perm(x20, x21, 0x7531u) >> (2 * t)) & m2) + ((y >> 4) & m1) * k1 + bb;
 }
 
-// p·V of one compressed V record on the tensor cores.  tab: the int8 B table of p'
-// (build_i8tab, natural slot order); pv4: this lane's p' = p * scale_r for slots
-// 4*lane .. +3; invf: per head.  Adds sum_r p'_r code[r][c] into sacc.  Returns false
-// (nothing added) if the record fails the prologue's checks.
+// p·V of one compressed V record in natural channel order (see pv_nat_unit): adds
+// sum_r p'_r code[r][c], digits joined and times invf, into sacc (the warp's [G][128]
+// channel sums).  tab: the int8 B table of p' in natural slot order (build_i8tab).
+// Returns false (nothing added) if the record fails the prologue's checks.
 template <int BITS, int G>
-__device__ __forceinline__ bool pv_packed_tc(unsigned char* st, uint32_t len, const uint32_t* tab,
-                                             const float (&pv4)[G][4], const float (&invf)[G], float* sacc, int lane) {
+__device__ __forceinline__ bool pv_packed_nat(unsigned char* st, uint32_t len, const uint32_t* tab,
+                                              const float (&invf)[G], float* sacc, int lane) {
   using L = I8Layout<G>;
   constexpr int NT = L::kNT;
+  constexpr bool kFragRegs = NT <= PACKKV_NAT_FRAG_NT;  // B fragments of all four groups in registers
   uint32_t m4[4];
   if (!packed_prologue<BITS>(st, len, m4, lane)) return false;
-  const int t = lane & 3;
-  uint32_t* desc = reinterpret_cast<uint32_t*>(st);
+  const int g8 = lane >> 2, t = lane & 3;
+  // word starts: lane sums of the widths, two groups per 16-bit half, scanned over the warp
+  uint32_t ls[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) ls[g] = __dp4a((m4[g] >> 4) & 0x0F0F0F0Fu, 0x01010101u, 0u);
+  uint32_t inc0 = ls[0] | (ls[1] << 16), inc1 = ls[2] | (ls[3] << 16);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y0 = __shfl_up_sync(0xffffffffu, inc0, o), y1 = __shfl_up_sync(0xffffffffu, inc1, o);
+    if (lane >= o) {
+      inc0 += y0;
+      inc1 += y1;
+    }
+  }
+  const uint32_t tot0 = __shfl_sync(0xffffffffu, inc0, 31), tot1 = __shfl_sync(0xffffffffu, inc1, 31);
+  const int gs1 = (int)(tot0 & 0xFFFFu), gs2 = gs1 + (int)(tot0 >> 16), gs3 = gs2 + (int)(tot1 & 0xFFFFu);
+  const uint32_t ex0 = inc0 - (ls[0] | (ls[1] << 16)), ex1 = inc1 - (ls[2] | (ls[3] << 16));
+  const uint32_t ex[4] = {ex0 & 0xFFFFu, ex0 >> 16, ex1 & 0xFFFFu, ex1 >> 16};
+  uint16_t* d16 = reinterpret_cast<uint16_t*>(st);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t rel = ex[g];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t mb = (m4[g] >> (8 * i)) & 0xFFu;  // base | width << 4
+      const uint32_t w = mb >> 4;
+      d16[2 * (64 * g + 8 * (lane >> 2) + 4 * (lane & 1) + i) + ((lane >> 1) & 1)] =
+          (uint16_t)(rel | (w << 9) | ((mb & 15u) << 12));
+      rel += w;
+    }
+  }
+  uint32_t bA[kFragRegs ? 4 : 1][2][NT], bB[kFragRegs ? 4 : 1][2][NT];
+  if constexpr (kFragRegs) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) pv_group_frags<NT>(tab, g, lane, bA[g], bB[g]);
+  }
+  __syncwarp();  // descriptors written
   const uint32_t* words = reinterpret_cast<const uint32_t*>(st + kPackedWordOffset);
-  const uint32_t dummy = ((uint32_t)kZeroUnitStart & 0xFFFFu) | 0xFFFF0000u;
+  const uint32_t* dsc = reinterpret_cast<const uint32_t*>(st) + g8;
   const PairW pw = pair_weights(t);
   float f_t[L::kNH];
 #pragma unroll
   for (int jh = 0; jh < L::kNH; ++jh) f_t[jh] = head_sel<G>(invf, L::head(jh, t));
-  // base terms first: channel c gets sum_g base_gc * (sum of p' over group g); lanes
-  // 8g .. 8g+7 hold group g.  (Every later addition into sacc commutes with these.)
+#pragma unroll 1
+  for (int T = 0; T < 8; ++T) {
+    int d[NT][4];
 #pragma unroll
-  for (int hd = 0; hd < G; ++hd) {
-    float ps = (pv4[hd][0] + pv4[hd][1]) + (pv4[hd][2] + pv4[hd][3]);
-    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
-    ps += __shfl_xor_sync(0xffffffffu, ps, 2);
-    ps += __shfl_xor_sync(0xffffffffu, ps, 4);
-    float bacc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < NT; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = kRoundBits;
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      const float pg = __shfl_sync(0xffffffffu, ps, 8 * g);
+      const uint32_t x = dsc[64 * g + 8 * T];
+      const int gs = g == 0 ? 0 : (g == 1 ? gs1 : (g == 2 ? gs2 : gs3));
+      uint32_t aA[4], aB[4];  // rows g8 / g8 + 8 at kh 0, then kh 1
+      pv_nat_unit(words, gs, x & 0xFFFFu, t, aA[0], aA[2], aB[0], aB[2]);
+      pv_nat_unit(words, gs, x >> 16, t, aA[1], aA[3], aB[1], aB[3]);
+      const int gi = kFragRegs ? g : 0;
+      if constexpr (!kFragRegs) pv_group_frags<NT>(tab, g, lane, bA[0], bB[0]);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) bacc[i] = fmaf(small_u2f((m4[g] >> (8 * i)) & 15u), pg, bacc[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sacc[hd * 128 + 4 * lane + i] += bacc[i];
-  }
-  int wbase = 0;
-#pragma unroll 1
-  for (int g = 0; g < 4; ++g) {
-    __syncwarp();  // the previous group's runs are done: desc may be rewritten
-    const SortedGroup sg = sort_group(m4[g], wbase, desc, dummy, [](int c) { return (uint32_t)c; }, lane);
-    uint32_t bA[2][NT], bB[2][NT];
-    pv_group_frags<NT>(tab, g, lane, bA, bB);
-    __syncwarp();  // desc of this group written
-#pragma unroll 1
-    for (int blk = 0; blk < sg.nblk; ++blk) {
-      switch (sg.width(blk)) {  // warp-uniform
-        case 4: pv_run<4, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
-        case 3: pv_run<3, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
-        case 2: pv_run<2, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
-        default: pv_run<1, G>(words, desc, blk, bA, bB, f_t, pw, sacc, lane); break;
+      for (int j = 0; j < NT; ++j) {
+        imma16832(d[j], aA, bA[gi][0][j], bA[gi][1][j]);
+        imma16832(d[j], aB, bB[gi][0][j], bB[gi][1][j]);
       }
-      __syncwarp();  // a run's sums are added before the next run (rows of one group differ, but
-                     // a lane adds rows it does not own across runs only through sacc)
     }
+    auto emit = [&](int TT, int jh, float lo, float hi) {
+      if (L::owns(jh, t)) {
+        float* row = sacc + L::head(jh, t) * 128 + 16 * TT + g8;
+        row[0] = fmaf(lo, f_t[jh], row[0]);
+        row[8] = fmaf(hi, f_t[jh], row[8]);
+      }
+    };
+    emit_tile<G>(T, d, 1.f, 1.f, pw, emit);
   }
+  __syncwarp();  // sums added before other lanes read or add them
   return true;
 }
 

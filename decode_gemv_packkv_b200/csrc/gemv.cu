@@ -24,9 +24,11 @@
 //    (u8 x s8 -> s32, exact) multiplies them by q' or p' written as three
 //    base-128 digits of q'*f (f = 127 / max|q'| per record and head; about 22
 //    significant bits, the digits in three B columns).
-//  * Compressed (frame-of-reference) records also run on the int8 tensor cores: the
-//    units of each pack group are sorted by width so that every run of 16 units is
-//    decoded with one instruction sequence (decode.cuh, "Compressed records").
+//  * Compressed (frame-of-reference) records also run on the int8 tensor cores
+//    (decode.cuh, "Compressed records"): for q·Kᵀ the units of each pack group are
+//    sorted by width so that every run of 16 units is decoded with one instruction
+//    sequence; for p·V every lane decodes its units in natural channel order with the
+//    same instructions whatever their widths.
 //  * p·V: a warp sums its item range into per-channel fp32 partials and writes
 //    them to the workspace at every (sequence, head) boundary (split-K over the
 //    sequence); a second-pass kernel, launched as a programmatic dependent so
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, pv_min_ctas(BITS, G))
       if (kind == kKindRaw)
         pv_i8<BITS, G>(st, tab, invf, acc_lo, acc_hi, lane);
       else
-        ok = pv_packed_tc<BITS, G>(st, (uint32_t)(kind_len >> 8) * 16u, tab, pv4, invf, sacc, lane);
+        ok = pv_packed_nat<BITS, G>(st, (uint32_t)(kind_len >> 8) * 16u, tab, invf, sacc, lane);
       if (ok) {
 #pragma unroll
         for (int hd = 0; hd < G; ++hd) mp[hd] += mpr[hd];

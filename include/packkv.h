@@ -228,7 +228,7 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
  * (sequence, kv head) pairs fit.  A call that needs more returns
  * PACKKV_ERR_CAPACITY without launching anything.
  * The first call on a device looks up the array's device address (a one-time
- * set-up, cached per device); make that first call before any stream capture.
+ * set-up, cached per device).
  * The cached address belongs to the device's current context: after a
  * cudaDeviceReset in the same process this entry point must not be used again.
  * All calls share the one array, and it keeps the last call's partials: calls
