@@ -57,15 +57,18 @@ struct I8Layout {
 
 // p·V records in flight per warp.  With one, p of the record in flight waits in
 // registers; with more, each stage also holds its record's p slices (bulk-copied with it).
+// 0 (default): two for 2- and 4-bit records, one for 3-bit records (measured: two stages
+// took 5% off the GQA p·V and added 5% to the batched 3-bit one; three were slower).
 #ifndef PACKKV_PV_STAGES
-#define PACKKV_PV_STAGES 1
+#define PACKKV_PV_STAGES 0
 #endif
+constexpr int pv_stages(int bits) { return PACKKV_PV_STAGES > 0 ? PACKKV_PV_STAGES : (bits == 3 ? 1 : 2); }
 
 template <int BITS, int G, bool PV>
 struct Cfg {
   static constexpr int kRecBytes = raw_record_bytes(BITS);
   static constexpr int kStageRec = kRecBytes;                  // >= every record, staged in one piece
-  static constexpr bool kStagedP = PV && PACKKV_PV_STAGES > 1;  // p slices [G][128] fp32 after the record
+  static constexpr bool kStagedP = PV && pv_stages(BITS) > 1;  // p slices [G][128] fp32 after the record
   static constexpr int kStageBytes = kStageRec + (kStagedP ? 512 * G : 0);
   // int8 tensor-core B table: columns n = 4*head + digit (digit 3 = 0), NT n-tiles of 8
   static constexpr int kNT = I8Layout<G>::kNT;
@@ -75,7 +78,7 @@ struct Cfg {
   static constexpr int kSumBytes = PV ? 512 * G : 0;          // p·V: [G][128] channel sums
   static constexpr int kFixed = kTableBytes + kSumBytes;
   static constexpr int kStages0 = (kWarpSmemBudget - kFixed - 64) / kStageBytes;
-  static constexpr int kStages = PV ? PACKKV_PV_STAGES : (kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0));
+  static constexpr int kStages = PV ? pv_stages(BITS) : (kStages0 > 4 ? 4 : (kStages0 < 1 ? 1 : kStages0));
   static constexpr int kWarpSmem = ((kStages * kStageBytes + kFixed + kStages * 16) + 127) / 128 * 128;
   static_assert(kStageBytes % 16 == 0 && kFixed % 16 == 0, "stage alignment");
 };

@@ -223,9 +223,9 @@ packkv_status packkv_pv_gemv(const packkv_cache* cache, const float* p, int64_t 
  * the call allocates nothing.  It needs
  *     (W + batch*kv_heads) * G * 512 bytes,
  * W = the warps it launches = min(batch*kv_heads*items per pair, resident warps
- * of the p·V kernel: SMs x CTAs per SM x 4); e.g. on a B200 with G = 4 (4 CTAs
- * per SM, W = 2368 once the cache has that many items) about 1700
- * (sequence, kv head) pairs fit.  A call that needs more returns
+ * of the p·V kernel: SMs x CTAs per SM x 4); e.g. on a B200 with 4-bit records
+ * and G = 4 (2 CTAs per SM, W = 1184 once the cache has that many items) about
+ * 2900 (sequence, kv head) pairs fit.  A call that needs more returns
  * PACKKV_ERR_CAPACITY without launching anything.
  * The first call on a device looks up the array's device address (a one-time
  * set-up, cached per device).
