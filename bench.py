@@ -143,9 +143,14 @@ def measured_peaks():
 
 # DRAM bytes (read + write) per launch of pv_kernel, the first pass of packkv_pv_gemv,
 # measured by ncu on this build's kernels (dram__bytes_read.sum + dram__bytes_write.sum,
-# one capture of the 32-head 32k-token 4-bit cache; summary in profiles/).  None for
+# mean of two launches on the 32-head 32k-token 4-bit cache; summary in
+# profiles/launches__bench_mha32_seq32k_b4.md).  The q·Kᵀ entry serves when q·Kᵀ is the
+# dominant kernel.  None for
 # other workloads, and None whenever the kernel has changed since the capture.
-DRAM_TRAFFIC = {}
+DRAM_TRAFFIC = {
+    ("llama7b-decode mha b1 h32 d128 seq32768 4-bit", 4, "pv"): 75_790_848,
+    ("llama7b-decode mha b1 h32 d128 seq32768 4-bit", 4, "qk"): 72_169_088,
+}
 
 
 # ------------------------------------------------------------------ the CUDA path: helpers
