@@ -53,7 +53,7 @@ struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
   uint16_t vmin[kBlockTokens], vscale[kBlockTokens];  // per token (original order)
   float krcp[kHeadDim], vrcp[kBlockTokens];      // 1 / scale (rounded), 0 for a zero scale
   float red[4][kEncodeThreads];        // min / max partials
-  int key[kBlockTokens];
+  alignas(16) int key[kBlockTokens];  // reorder key * 128 + token
   int rank_part[kParts][kBlockTokens];
   uint8_t perm[kBlockTokens];          // perm[slot] = token
   uint8_t base[2][kGroups][kHeadDim];
@@ -72,6 +72,14 @@ struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
 static_assert(sizeof(EncodeSmem) <= 113 * 1024, "two encoder CTAs per SM");
 
 __device__ __forceinline__ int bitlen(uint32_t x) { return x == 0 ? 0 : 32 - __clz(x); }
+
+constexpr float kEncRound = 12582912.0f;  // 1.5 * 2^23: y + kEncRound keeps rint(y) in the low bits
+
+// The low bytes of four floats, packed in order.
+__device__ __forceinline__ uint32_t low_bytes4(float2 lo, float2 hi) {
+  return __byte_perm(__byte_perm(__float_as_uint(lo.x), __float_as_uint(lo.y), 0x0040u),
+                     __byte_perm(__float_as_uint(hi.x), __float_as_uint(hi.y), 0x0040u), 0x5410u);
+}
 
 // code = clamp(rint(fl(d / s)), 0, qmax) for d = fl(x - mn) >= 0 and scale s > 0, with
 // r = 1/s rounded to nearest.  q1 = fl(d * r) lies within 2^-18 of fl(d / s) (both are
@@ -211,53 +219,61 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   if (!input_ok) s.failed = 1;  // every writer writes 1
   __syncthreads();
 
-  // ---- non-finite values ------------------------------------------------------
+  // ---- quantization ranges (K per channel, V per token) and non-finite values ---
+  // fp16 pairs: min / max of fp16 values are exact in fp16 (NaN is passed over, as fminf
+  // does; a signed zero is normalised below).  A value whose exponent field is all ones
+  // (inf or NaN) carries into bit 15 of its half when 0x0400 is added to that field.
   {
-    const uint4* kin = reinterpret_cast<const uint4*>(&s.kx[0][0]);
-    const uint4* vin = reinterpret_cast<const uint4*>(&s.vx[0][0]);
-    int bad = 0;
-    for (int i = tid; i < kBlockTokens * kHeadDim / 8; i += blockDim.x) {
-      const uint4 kk = kin[i], vv = vin[i];
-      const uint32_t w[8] = {kk.x, kk.y, kk.z, kk.w, vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        bad |= ((w[j] & 0x7C00u) == 0x7C00u) | ((w[j] & 0x7C000000u) == 0x7C000000u);
-      }
-    }
-    if (bad) s.nonfinite = 1;
-  }
-
-  // ---- quantization parameters: K per channel, V per token -------------------
-  {
-    // kParts threads per channel (K) and per token (V), each over a slice of the block
-    constexpr int kSlice = kBlockTokens / kParts;
-    const int part = tid / kBlockTokens, idx = tid % kBlockTokens;
-    float mn = 3.4e38f, mx = -3.4e38f, vmn = 3.4e38f, vmx = -3.4e38f;
+    const __half2* k2 = reinterpret_cast<const __half2*>(&s.kx[0][0]);  // [token][channel pair]
+    const __half2* v2 = reinterpret_cast<const __half2*>(&s.vx[0][0]);
+    constexpr int kPairs = kHeadDim / 2;
+    constexpr int kKParts = kEncodeThreads / kPairs;      // token slices per K channel pair
+    constexpr int kKSlice = kBlockTokens / kKParts;
+    constexpr int kVSlice = kPairs / kParts;              // channel pairs per V token slice
+    const int cp = tid % kPairs, kpart = tid / kPairs;
+    const int t = tid % kBlockTokens, vpart = tid / kBlockTokens;
+    uint32_t bad = 0u;
+    __half2 kmn = k2[kKSlice * kpart * kPairs + cp], kmx = kmn;
 #pragma unroll 8
-    for (int i = 0; i < kSlice; ++i) {
-      const float xk = __half2float(s.kx[kSlice * part + i][idx]);
-      mn = fminf(mn, xk);
-      mx = fmaxf(mx, xk);
-      const float xv = __half2float(s.vx[idx][(kSlice * part + i + idx) & (kHeadDim - 1)]);  // rotated: banks
-      vmn = fminf(vmn, xv);
-      vmx = fmaxf(vmx, xv);
+    for (int i = 0; i < kKSlice; ++i) {
+      const __half2 h = k2[(kKSlice * kpart + i) * kPairs + cp];
+      kmn = __hmin2(kmn, h);
+      kmx = __hmax2(kmx, h);
+      bad |= (*reinterpret_cast<const uint32_t*>(&h) & 0x7C007C00u) + 0x04000400u;
     }
-    s.red[0][tid] = mn;
-    s.red[1][tid] = mx;
-    s.red[2][tid] = vmn;
-    s.red[3][tid] = vmx;
+    // a token's pairs from a rotated start: the 32 tokens of a warp hit 32 banks
+    const int p0 = kVSlice * vpart + t;
+    __half2 vmn = v2[t * kPairs + (p0 & (kPairs - 1))], vmx = vmn;
+#pragma unroll 8
+    for (int j = 0; j < kVSlice; ++j) {
+      const __half2 h = v2[t * kPairs + ((p0 + j) & (kPairs - 1))];
+      vmn = __hmin2(vmn, h);
+      vmx = __hmax2(vmx, h);
+      bad |= (*reinterpret_cast<const uint32_t*>(&h) & 0x7C007C00u) + 0x04000400u;
+    }
+    __half2* redk = reinterpret_cast<__half2*>(&s.red[0][0]);  // [min, max][kKParts][kPairs]
+    __half* redv = reinterpret_cast<__half*>(&s.red[2][0]);    // [min, max][kParts][kBlockTokens]
+    redk[kpart * kPairs + cp] = kmn;
+    redk[(kKParts + kpart) * kPairs + cp] = kmx;
+    redv[vpart * kBlockTokens + t] = __hmin(__low2half(vmn), __high2half(vmn));
+    redv[(kParts + vpart) * kBlockTokens + t] = __hmax(__low2half(vmx), __high2half(vmx));
+    if (bad & 0x80008000u) s.nonfinite = 1;
   }
   __syncthreads();
   if (tid == 0 && s.nonfinite) set_status(a.ctrl, PACKKV_DEV_NONFINITE);
   if (tid < 2 * kBlockTokens) {
     const bool is_k = tid < kBlockTokens;
-    const int i = tid % kBlockTokens, r0 = is_k ? 0 : 2;
-    float lo = s.red[r0][i], hi = s.red[r0 + 1][i];
-#pragma unroll
-    for (int q = 1; q < kParts; ++q) {
-      lo = fminf(lo, s.red[r0][q * kBlockTokens + i]);
-      hi = fmaxf(hi, s.red[r0 + 1][q * kBlockTokens + i]);
+    const int i = tid % kBlockTokens;
+    // K: the halves of channel i over the token slices; V: token i over the pair slices
+    const __half* red = reinterpret_cast<const __half*>(is_k ? &s.red[0][0] : &s.red[2][0]);
+    const int nq = is_k ? kEncodeThreads / (kHeadDim / 2) : kParts;
+    __half hlo = red[i], hhi = red[nq * kBlockTokens + i];
+    for (int q = 1; q < nq; ++q) {
+      hlo = __hmin(hlo, red[q * kBlockTokens + i]);
+      hhi = __hmax(hhi, red[(nq + q) * kBlockTokens + i]);
     }
+    float lo = __half2float(hlo);
+    const float hi = __half2float(hhi);
     if (lo == 0.0f) lo = 0.0f;  // -0 is stored as +0
     const float range = __fsub_rn(hi, lo);
     uint16_t sc = 0;
@@ -277,20 +293,65 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   __syncthreads();
 
   // ---- codes -----------------------------------------------------------------
-  // A thread keeps one channel (its K parameters in registers) and walks tokens.
+  // A thread keeps four channels (their K parameters in registers) and walks tokens;
+  // the four codes of a tensor go to shared memory as one word.  Fast path in pairs:
+  // q = fl(x - mn) * RN(1/scale), rint(q) by adding and removing 1.5 * 2^23 (ties to
+  // even), e = q - rint(q) exactly.  quant_code takes the correctly rounded quotient
+  // where it can differ, |e| >= 0.5 - 2^-17; where q is not finite or not below
+  // qmax + 0.5 (no clamp needed on the fast path), it takes the element too.
   {
-    static_assert(kEncodeThreads % kHeadDim == 0, "a thread keeps its channel");
-    const int c = tid & (kHeadDim - 1);
-    const float kmn = half_bits_to_float(s.kmin[c]), ksc = half_bits_to_float(s.kscale[c]), kr = s.krcp[c];
-    for (int t = tid >> 7; t < kBlockTokens; t += kEncodeThreads / kHeadDim) {
-      int code = 0;
-      if (ksc > 0.0f) code = quant_code(__fsub_rn(__half2float(s.kx[t][c]), kmn), ksc, kr, qmax);
-      s.ck[t][c] = (uint8_t)code;
-      const float vsc = half_bits_to_float(s.vscale[t]);
-      code = 0;
-      if (vsc > 0.0f)
-        code = quant_code(__fsub_rn(__half2float(s.vx[t][c]), half_bits_to_float(s.vmin[t])), vsc, s.vrcp[t], qmax);
-      s.cv[t][c] = (uint8_t)code;
+    static_assert(kEncodeThreads % (kHeadDim / 4) == 0, "a thread keeps its channels");
+    constexpr int kQuads = kHeadDim / 4, kRows = kEncodeThreads / kQuads;
+    const int j = tid % kQuads;
+    const float2 R = make_float2(kEncRound, kEncRound), nR = make_float2(-kEncRound, -kEncRound);
+    const float lim = (float)qmax + 0.5f;
+    constexpr float kTie = 0.5f - 7.62939453125e-06f;  // 0.5 - 2^-17
+    float2 nkmn[2], kr[2];
+    float ksc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ksc[i] = half_bits_to_float(s.kscale[4 * j + i]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      nkmn[h] = make_float2(-half_bits_to_float(s.kmin[4 * j + 2 * h]), -half_bits_to_float(s.kmin[4 * j + 2 * h + 1]));
+      kr[h] = make_float2(s.krcp[4 * j + 2 * h], s.krcp[4 * j + 2 * h + 1]);
+    }
+    // the four codes of x[0..3] (pairs x[h]) for minus-min nm, reciprocals r, scales sc
+    auto codes4 = [&](const float2 (&x)[2], const float2 (&nm)[2], const float2 (&r)[2],
+                      const float (&sc)[4]) -> uint32_t {
+      float2 d[2], q[2], u[2];
+      bool fast = true;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        d[h] = __fadd2_rn(x[h], nm[h]);
+        q[h] = __fmul2_rn(d[h], r[h]);
+        u[h] = __fadd2_rn(q[h], R);
+        const float2 e = __ffma2_rn(__fadd2_rn(u[h], nR), make_float2(-1.f, -1.f), q[h]);  // exact
+        fast = fast && q[h].x < lim && q[h].y < lim && fabsf(e.x) < kTie && fabsf(e.y) < kTie;
+      }
+      if (fast) return low_bytes4(u[0], u[1]);  // of 1.5 * 2^23 + rint(q): rint(q)
+      uint32_t w = 0u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float di = (i & 1) ? d[i >> 1].y : d[i >> 1].x;
+        const float ri = (i & 1) ? r[i >> 1].y : r[i >> 1].x;
+        const int c = sc[i] > 0.0f ? quant_code(di, sc[i], ri, qmax) : 0;
+        w |= (uint32_t)c << (8 * i);
+      }
+      return w;
+    };
+    for (int t = tid / kQuads; t < kBlockTokens; t += kRows) {
+      const uint2 kw = *reinterpret_cast<const uint2*>(&s.kx[t][4 * j]);
+      const float2 xk[2] = {__half22float2(*reinterpret_cast<const __half2*>(&kw.x)),
+                            __half22float2(*reinterpret_cast<const __half2*>(&kw.y))};
+      *reinterpret_cast<uint32_t*>(&s.ck[t][4 * j]) = codes4(xk, nkmn, kr, ksc);
+      const uint2 vw = *reinterpret_cast<const uint2*>(&s.vx[t][4 * j]);
+      const float2 xv[2] = {__half22float2(*reinterpret_cast<const __half2*>(&vw.x)),
+                            __half22float2(*reinterpret_cast<const __half2*>(&vw.y))};
+      const float nvm = -half_bits_to_float(s.vmin[t]), vr = s.vrcp[t], vs = half_bits_to_float(s.vscale[t]);
+      const float2 nvm2[2] = {make_float2(nvm, nvm), make_float2(nvm, nvm)};
+      const float2 vr2[2] = {make_float2(vr, vr), make_float2(vr, vr)};
+      const float vsc[4] = {vs, vs, vs, vs};
+      *reinterpret_cast<uint32_t*>(&s.cv[t][4 * j]) = codes4(xv, nvm2, vr2, vsc);
     }
   }
   __syncthreads();
@@ -305,24 +366,24 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
         if (a.key_kind == PACKKV_KEY_KV_SUM)
           sum = __dp4a(reinterpret_cast<const uint32_t*>(s.cv[t])[lane], 0x01010101u, sum);
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) s.key[t] = (int)sum;
+      sum = __reduce_add_sync(0xffffffffu, sum);
+      if (lane == 0) s.key[t] = (int)sum * kBlockTokens + t;  // key, then index: all distinct
     }
   }
   __syncthreads();
   {
-    // rank of token t = #{u : key[u] < key[t] or (key[u] == key[t] and u < t)};
+    // rank of token t = #{u : key[u] < key[t] or (key[u] == key[t] and u < t)}: with the
+    // index below the key (key * 128 + u), #{u : composite[u] < composite[t]};
     // kParts threads per token, each counting over a slice of the tokens
     constexpr int kSlice = kBlockTokens / kParts;
     const int t = tid % kBlockTokens, part = tid / kBlockTokens;
     const int kt = s.key[t];
+    const int4* k4 = reinterpret_cast<const int4*>(&s.key[kSlice * part]);
     int r = 0;
-#pragma unroll 8
-    for (int i = 0; i < kSlice; ++i) {
-      const int u = kSlice * part + i;
-      const int ku = s.key[u];
-      r += (ku < kt) | ((ku == kt) & (u < t));
+#pragma unroll
+    for (int i = 0; i < kSlice / 4; ++i) {
+      const int4 ku = k4[i];
+      r += (ku.x < kt) + (ku.y < kt) + (ku.z < kt) + (ku.w < kt);
     }
     s.rank_part[part][t] = r;
   }
@@ -352,14 +413,20 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     *reinterpret_cast<uint32_t*>(vt + c * kVtPitch + r4) = w;
   }
 
+  __syncthreads();  // the storage-order copies are complete
+
+  // code of storage slot r, channel c: K from the row copies, V from the transposed ones
+  auto slot_code = [&](int tensor, int r, int c) -> int {
+    return tensor ? vt[c * kVtPitch + r] : kp[r * kHeadDim + c];
+  };
+
   // ---- frame of reference and width of every (group, channel) unit ----------
   for (int u = tid; u < 2 * kGroups * kHeadDim; u += blockDim.x) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
-    const uint8_t(*cx)[kHeadDim] = tensor ? s.cv : s.ck;
     int lo = 255, hi = 0;
 #pragma unroll 8
     for (int j = 0; j < kGroupTokens; ++j) {
-      const int code = cx[s.perm[g * kGroupTokens + j]][c];
+      const int code = slot_code(tensor, g * kGroupTokens + j, c);
       lo = min(lo, code);
       hi = max(hi, code);
     }
@@ -495,7 +562,6 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   for (int u = tid; u < 2 * kGroups * kHeadDim; u += blockDim.x) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
     if (raw[tensor]) continue;  // written above
-    const uint8_t(*cx)[kHeadDim] = tensor ? s.cv : s.ck;
     const int w = raw[tensor] ? a.bits : s.width[tensor][g][c];
     const int base = raw[tensor] ? 0 : s.base[tensor][g][c];
     if (w == 0) continue;
@@ -514,7 +580,7 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
         const int per = 32 / p;
         for (int f = 0; f < per; ++f) {
           const int j = q * per + f;
-          const uint32_t off = (uint32_t)(cx[s.perm[g * kGroupTokens + j]][c] - base);
+          const uint32_t off = (uint32_t)(slot_code(tensor, g * kGroupTokens + j, c) - base);
           word |= ((off >> lo) & mask) << ((j * p) & 31);
         }
         words[at + q] = word;

@@ -25,7 +25,8 @@
  *   - Errors found on the host are returned before anything is launched, and
  *     nothing is written.  Errors found on the device (arena full, non-finite
  *     input, corrupt index entry, a wait that gave up) set sticky bits in the
- *     cache's status word; packkv_get_status reads and clears them.
+ *     cache's status word; packkv_get_status reads and clears them.  A block
+ *     holding a NaN or Inf is still encoded, but its records are unspecified.
  *   - Thread safety: calls on one cache must be serialised by the caller.
  */
 #ifndef PACKKV_H
