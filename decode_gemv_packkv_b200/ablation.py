@@ -1,6 +1,7 @@
-"""Encoder ablation on one GPU: reorder key x code width x input kind.
+"""Encoder ablation on one GPU: reorder key x unit mode x code width x input kind.
 
-For each combination this encodes a (1 sequence x H heads x T tokens) cache and
+For each combination (every reorder key with frame-of-reference units, and the
+default key with width-only units) this encodes a (1 sequence x H heads x T tokens) cache and
 reports the K and V compression ratios (fp16 bytes / (record + index bytes); plain
 b-bit quantization, codes plus fp16 min and scale, for comparison), the share of
 blocks stored raw, and the CUDA-event time of one packkv_qk_gemv and one
@@ -14,7 +15,7 @@ than L2, are rotated so that every launch reads HBM.
 
     python -m decode_gemv_packkv_b200.ablation [--heads 32] [--tokens 32768]
 
-prints one JSON line per (input kind, bits, reorder key).
+prints one JSON line per (input kind, bits, reorder key, unit mode).
 """
 import argparse
 import json
@@ -87,22 +88,28 @@ def run(heads: int, tokens: int, bits_list, reps: int, seed: int):
     for kind in ("iid", "structured"):
         kd, vd = _inputs(heads, T, kind == "structured", seed, dev)
         for bits in bits_list:
-            for key_name, key in KEYS.items():
-                first = pk.PackKVCache(1, heads, nb, bits, reorder_key=key)
+            # every reorder key with frame-of-reference units, then width-only units (base
+            # 0) with the default key: the width-only variant of the packing
+            combos = [(kn, kv, "frame-of-reference", pk.UNITS_FOR) for kn, kv in KEYS.items()]
+            combos.append(("k-code-sum", pk.KEY_K_SUM, "width-only", pk.UNITS_WIDTH_ONLY))
+            for key_name, key, unit_name, unit_mode in combos:
+                first = pk.PackKVCache(1, heads, nb, bits, reorder_key=key, unit_mode=unit_mode)
                 pk.packkv_encode_block(first, kd, vd, nb)
                 k_used, v_used = first.arena_used()
                 raw_k, raw_v = _raw_share(first, bits)
                 copies = max(3, int(np.ceil(2.5 * L2_BYTES / (k_used + v_used + 2 * index_bytes))))
                 caches = [first]
                 for _ in range(copies - 1):
-                    c = pk.PackKVCache(1, heads, nb, bits, reorder_key=key, arena_bytes=max(k_used, v_used) + 16)
+                    c = pk.PackKVCache(1, heads, nb, bits, reorder_key=key, arena_bytes=max(k_used, v_used) + 16,
+                                       unit_mode=unit_mode)
                     pk.packkv_encode_block(c, kd, vd, nb)
                     caches.append(c)
                 qk_us = _time(lambda i: pk.packkv_qk_gemv(caches[i], q, scale, scores), copies, reps)
                 pv_us = _time(lambda i: pk.packkv_pv_gemv(caches[i], p, out), copies, reps)
                 bad = [pk.packkv_get_status(c) for c in caches if pk.packkv_get_status(c) != 0]
                 print(json.dumps({
-                    "inputs": kind, "bits": bits, "reorder_key": key_name, "heads": heads, "tokens": T,
+                    "inputs": kind, "bits": bits, "reorder_key": key_name, "units": unit_name, "heads": heads,
+                    "tokens": T,
                     "cr_k": fp16_bytes / (k_used + index_bytes), "cr_v": fp16_bytes / (v_used + index_bytes),
                     "plain_quant_cr": 128 * 128 * 2 / (128 * 128 * bits / 8 + 512),  # codes + fp16 min/scale
                     "raw_share_k": raw_k, "raw_share_v": raw_v,

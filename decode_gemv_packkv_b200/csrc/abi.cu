@@ -34,6 +34,7 @@ packkv_status check_cache(const packkv_cache* c) {
     return PACKKV_ERR_UNSUPPORTED;
   if (f.bits < 2 || f.bits > 4) return PACKKV_ERR_UNSUPPORTED;
   if (f.reorder_key > PACKKV_KEY_KV_SUM) return PACKKV_ERR_UNSUPPORTED;
+  if (f.unit_mode > PACKKV_UNITS_WIDTH_ONLY) return PACKKV_ERR_UNSUPPORTED;
   if (c->batch < 1 || c->kv_heads < 1 || c->max_blocks < 1) return PACKKV_ERR_INVALID_ARG;
   if ((int64_t)c->batch * c->kv_heads > (1 << 24) || (int64_t)c->max_blocks > (1 << 24))
     return PACKKV_ERR_INVALID_ARG;
@@ -116,6 +117,7 @@ EncodeArgs encode_args(const packkv_cache* c, const uint16_t* k, const uint16_t*
   a.max_blocks = c->max_blocks;
   a.bits = (int)c->fmt.bits;
   a.key_kind = (int)c->fmt.reorder_key;
+  a.unit_mode = (int)c->fmt.unit_mode;
   a.k_index = c->k_index;
   a.v_index = c->v_index;
   a.k_arena = c->k_arena;

@@ -406,11 +406,20 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     const int r = i >> 3, q = i & 7;
     reinterpret_cast<uint4*>(kp + r * kHeadDim)[q] = reinterpret_cast<const uint4*>(s.ck[s.perm[r]])[q];
   }
-  for (int i = tid; i < kHeadDim * kBlockTokens / 4; i += blockDim.x) {
-    const int c = i & (kHeadDim - 1), r4 = (i >> 7) * 4;  // lanes take consecutive channels
-    const uint32_t w = (uint32_t)s.cv[s.perm[r4]][c] | ((uint32_t)s.cv[s.perm[r4 + 1]][c] << 8) |
-                       ((uint32_t)s.cv[s.perm[r4 + 2]][c] << 16) | ((uint32_t)s.cv[s.perm[r4 + 3]][c] << 24);
-    *reinterpret_cast<uint32_t*>(vt + c * kVtPitch + r4) = w;
+  // V: four slots x four channels per task, a 4x4 byte transpose of four row words
+  for (int i = tid; i < kHeadDim * kBlockTokens / 16; i += blockDim.x) {
+    const int cq = i & (kHeadDim / 4 - 1), r4 = (i >> 5) * 4;  // lanes take consecutive channel quads
+    const uint32_t w0 = reinterpret_cast<const uint32_t*>(s.cv[s.perm[r4]])[cq];
+    const uint32_t w1 = reinterpret_cast<const uint32_t*>(s.cv[s.perm[r4 + 1]])[cq];
+    const uint32_t w2 = reinterpret_cast<const uint32_t*>(s.cv[s.perm[r4 + 2]])[cq];
+    const uint32_t w3 = reinterpret_cast<const uint32_t*>(s.cv[s.perm[r4 + 3]])[cq];
+    const uint32_t lo01 = __byte_perm(w0, w1, 0x5140u), hi01 = __byte_perm(w0, w1, 0x7362u);  // b0 b4 b1 b5 / b2 b6 b3 b7
+    const uint32_t lo23 = __byte_perm(w2, w3, 0x5140u), hi23 = __byte_perm(w2, w3, 0x7362u);
+    uint8_t* dst = vt + 4 * cq * kVtPitch + r4;
+    *reinterpret_cast<uint32_t*>(dst) = __byte_perm(lo01, lo23, 0x5410u);                // channel 4cq
+    *reinterpret_cast<uint32_t*>(dst + kVtPitch) = __byte_perm(lo01, lo23, 0x7632u);     // 4cq + 1
+    *reinterpret_cast<uint32_t*>(dst + 2 * kVtPitch) = __byte_perm(hi01, hi23, 0x5410u); // 4cq + 2
+    *reinterpret_cast<uint32_t*>(dst + 3 * kVtPitch) = __byte_perm(hi01, hi23, 0x7632u); // 4cq + 3
   }
 
   __syncthreads();  // the storage-order copies are complete
@@ -430,9 +439,13 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
       lo = min(lo, code);
       hi = max(hi, code);
     }
+    if (a.unit_mode == (int)PACKKV_UNITS_WIDTH_ONLY) lo = 0;  // no frame of reference
+    const int w = bitlen((uint32_t)(hi - lo));
     s.base[tensor][g][c] = (uint8_t)lo;
-    s.width[tensor][g][c] = (uint8_t)bitlen((uint32_t)(hi - lo));
-    atomicAdd(&s.wsum[tensor], bitlen((uint32_t)(hi - lo)));
+    s.width[tensor][g][c] = (uint8_t)w;
+    // a warp's 32 units belong to one tensor (512 units per tensor, warps of 32)
+    const int wsum = (int)__reduce_add_sync(0xffffffffu, (unsigned)w);
+    if ((tid & 31) == 0) atomicAdd(&s.wsum[tensor], wsum);
   }
   __syncthreads();
 
@@ -483,17 +496,32 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   }
   __syncthreads();
 
-  // ---- assemble both records in shared memory (reusing the input buffers) ---
-  uint32_t* rec32[2] = {reinterpret_cast<uint32_t*>(&s.kx[0][0]), reinterpret_cast<uint32_t*>(&s.vx[0][0])};
-  for (int i = tid; i < raw_bytes / 16; i += blockDim.x) {
-    reinterpret_cast<uint4*>(rec32[0])[i] = make_uint4(0u, 0u, 0u, 0u);
-    reinterpret_cast<uint4*>(rec32[1])[i] = make_uint4(0u, 0u, 0u, 0u);
+  // ---- look-back: arena offsets (warp 0: K, warp 1: V), while warps 2.. assemble ----
+  if (tid < 64) {
+    const int tensor = tid >> 5, lane = tid & 31;
+    uint32_t* index = tensor ? a.v_index : a.k_index;
+    const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
+    unsigned long long excl = 0;
+    const bool ok = look_back(index, a, plan, t_call, end0, &excl, lane);
+    if (lane == 0) {
+      if (!ok) s.failed = 1;
+      s.prefix[tensor] = excl;
+      // final entry {offset16, length16}; a failed call is invalidated by the last CTA
+      const unsigned long long fin = (unsigned long long)(uint32_t)(end0 + excl) |
+                                     ((unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) << 32);
+      atomicExch(entry64(index, a, plan, t_call), fin);
+    }
   }
-  __syncthreads();
+  // ---- assemble both records in shared memory (reusing the input buffers) ---
+  // Threads 64.. (asm = tid - 64) write every byte of both records: header, parameters,
+  // meta, each word by exactly one thread, and the zero padding to 16 bytes.
+  uint32_t* rec32[2] = {reinterpret_cast<uint32_t*>(&s.kx[0][0]), reinterpret_cast<uint32_t*>(&s.vx[0][0])};
+  constexpr int kAsmFirst = 64;
+  const int asm_id = tid - kAsmFirst, n_asm = (int)blockDim.x - kAsmFirst;
 #pragma unroll
   for (int tensor = 0; tensor < 2; ++tensor) {
     unsigned char* rec = reinterpret_cast<unsigned char*>(rec32[tensor]);
-    if (tid == 0) {
+    if (asm_id == 0) {
       uint16_t* gws = reinterpret_cast<uint16_t*>(rec);
       int acc = 0;
       for (int g = 0; g < kGroups; ++g) {
@@ -504,20 +532,23 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
                              (PACKKV_FORMAT_VERSION << 8) | ((uint32_t)a.bits << 16);
       reinterpret_cast<uint32_t*>(rec)[2] = flags;
       reinterpret_cast<uint32_t*>(rec)[3] = (uint32_t)acc;
+      // zero padding after the last word (compressed records; raw ones end on 16 bytes)
+      const int end_words = (raw[tensor] ? kRawWordOffset / 4 + 512 * a.bits : kPackedWordOffset / 4 + acc);
+      for (int wpad = end_words; wpad < rec_bytes[tensor] / 4; ++wpad) rec32[tensor][wpad] = 0u;
     }
-    if (tid < kHeadDim) {
+    if (asm_id >= 0 && asm_id < kHeadDim) {
       uint16_t* mn = reinterpret_cast<uint16_t*>(rec + kParamOffset);
       uint16_t* sc = mn + kHeadDim;
       if (tensor == 0) {
-        mn[tid] = s.kmin[tid];
-        sc[tid] = s.kscale[tid];
+        mn[asm_id] = s.kmin[asm_id];
+        sc[asm_id] = s.kscale[asm_id];
       } else {
-        mn[tid] = s.vmin[s.perm[tid]];
-        sc[tid] = s.vscale[s.perm[tid]];
+        mn[asm_id] = s.vmin[s.perm[asm_id]];
+        sc[asm_id] = s.vscale[s.perm[asm_id]];
       }
     }
-    if (!raw[tensor]) {
-      for (int u = tid; u < kGroups * kHeadDim; u += blockDim.x) {
+    if (!raw[tensor] && asm_id >= 0) {
+      for (int u = asm_id; u < kGroups * kHeadDim; u += n_asm) {
         const int g = u >> 7, c = u & 127;
         rec[kMetaOffset + u] = (uint8_t)(s.base[tensor][g][c] | (s.width[tensor][g][c] << 4));
       }
@@ -528,38 +559,45 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   // m).  A word's byte e holds column k0 + e of rows (16T + 8rh + g): one 32-bit load
   // of a storage-order row gives the four codes of a (row, byte) field set, placed by
   // one shift.  b = 3: bits 0-1 in words 0..1023 (the b = 2 order), bit 2 in 1024..1535.
+  // Word wj = ((row group * 2 + J) * 32 + 4g + t) * 4 + 2 Q2 + kh, kappa = 2J + Q2; the row
+  // group is the tile (b = 4), the tile pair (b = 2, low plane of b = 3) or the tile quad
+  // (bit-2 plane).  A task is one (row group, J, t, Q2, kh) and walks g = 0..7: the lanes
+  // of a warp then read 32 different banks.
+  {
+    const int n_tasks = 512 * a.bits / 8;  // per tensor
+    for (int task = asm_id; asm_id >= 0 && task < 2 * n_tasks; task += n_asm) {
+      const int tensor = task >= n_tasks ? 1 : 0;
+      if (!raw[tensor]) continue;
+      const int tk = task - tensor * n_tasks;
+      uint32_t* words = rec32[tensor] + kRawWordOffset / 4;
+      const uint8_t* rows = tensor ? vt : kp;
+      const int pitch = tensor ? kVtPitch : kHeadDim;
+      const bool plane1 = a.bits == 3 && tk >= 128;
+      const int tj = plane1 ? tk - 128 : tk;
+      const int i = tj & 3, t = (tj >> 2) & 3, jj = (tj >> 4) & 1, tp = tj >> 5;
+      const uint8_t* col = rows + 32 * (2 * jj + (i >> 1)) + 16 * (i & 1) + 4 * t;
+      uint32_t* wout = words + (plane1 ? 1024 : 0) + ((tp * 2 + jj) * 32 + t) * 4 + i;
+#pragma unroll 2
+      for (int g = 0; g < 8; ++g, col += pitch) {
+        auto row4 = [&](int m8) { return *reinterpret_cast<const uint32_t*>(col + m8 * 8 * pitch); };
+        uint32_t word;
+        if (a.bits == 4) {
+          word = row4(2 * tp) | (row4(2 * tp + 1) << 4);  // rows 16T + g, 16T + 8 + g
+        } else if (!plane1) {
+          const uint32_t m3 = a.bits == 3 ? 0x03030303u : 0xFFFFFFFFu;
+          word = (row4(4 * tp) & m3) | ((row4(4 * tp + 1) & m3) << 2) | ((row4(4 * tp + 2) & m3) << 4) |
+                 ((row4(4 * tp + 3) & m3) << 6);
+        } else {
+          word = 0u;
 #pragma unroll
-  for (int tensor = 0; tensor < 2; ++tensor) {
-    if (!raw[tensor]) continue;
-    uint32_t* words = rec32[tensor] + kRawWordOffset / 4;
-    const uint8_t* rows = tensor ? vt : kp;
-    const int pitch = tensor ? kVtPitch : kHeadDim;
-    for (int wi = tid; wi < 512 * a.bits; wi += blockDim.x) {
-      const bool plane1 = a.bits == 3 && wi >= 1024;
-      const int wj = plane1 ? wi - 1024 : wi;
-      // wj = ((row group)*2 + J)*32 + lane)*4 + 2*Q2 + kh, kappa = 2J + Q2; the row group is
-      // the tile (b = 4), the tile pair (b = 2, low plane of b = 3) or the tile quad (bit-2 plane)
-      const int kh = wj & 1, q2 = (wj >> 1) & 1, lane = (wj >> 2) & 31, jj = (wj >> 7) & 1, tp = wj >> 8;
-      const int g = lane >> 2, t = lane & 3;
-      const uint8_t* col = rows + 32 * (2 * jj + q2) + 16 * kh + 4 * t + g * pitch;
-      auto row4 = [&](int m8) { return *reinterpret_cast<const uint32_t*>(col + m8 * 8 * pitch); };  // row 8*m8 + g
-      uint32_t word;
-      if (a.bits == 4) {
-        word = row4(2 * tp) | (row4(2 * tp + 1) << 4);  // rows 16T + g, 16T + 8 + g
-      } else if (!plane1) {
-        const uint32_t m3 = a.bits == 3 ? 0x03030303u : 0xFFFFFFFFu;
-        word = (row4(4 * tp) & m3) | ((row4(4 * tp + 1) & m3) << 2) | ((row4(4 * tp + 2) & m3) << 4) |
-               ((row4(4 * tp + 3) & m3) << 6);
-      } else {
-        word = 0u;
-#pragma unroll
-        for (int sg = 0; sg < 8; ++sg) word |= ((row4(8 * tp + sg) >> 2) & 0x01010101u) << sg;
+          for (int sg = 0; sg < 8; ++sg) word |= ((row4(8 * tp + sg) >> 2) & 0x01010101u) << sg;
+        }
+        wout[16 * g] = word;
       }
-      words[wi] = word;
     }
   }
   // pack the units: every word is owned by exactly one thread
-  for (int u = tid; u < 2 * kGroups * kHeadDim; u += blockDim.x) {
+  for (int u = asm_id; asm_id >= 0 && u < 2 * kGroups * kHeadDim; u += n_asm) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
     if (raw[tensor]) continue;  // written above
     const int w = raw[tensor] ? a.bits : s.width[tensor][g][c];
@@ -591,23 +629,7 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     }
   }
 
-  // ---- look-back: arena offsets (warp 0: K, warp 1: V) -------------------------
-  if (tid < 64) {
-    const int tensor = tid >> 5, lane = tid & 31;
-    uint32_t* index = tensor ? a.v_index : a.k_index;
-    const unsigned long long end0 = a.ctrl[tensor ? kCtrlVEnd : kCtrlKEnd];
-    unsigned long long excl = 0;
-    const bool ok = look_back(index, a, plan, t_call, end0, &excl, lane);
-    if (lane == 0) {
-      if (!ok) s.failed = 1;
-      s.prefix[tensor] = excl;
-      // final entry {offset16, length16}; a failed call is invalidated by the last CTA
-      const unsigned long long fin = (unsigned long long)(uint32_t)(end0 + excl) |
-                                     ((unsigned long long)(uint32_t)(rec_bytes[tensor] >> 4) << 32);
-      atomicExch(entry64(index, a, plan, t_call), fin);
-    }
-  }
-  __syncthreads();
+  __syncthreads();  // records assembled, arena offsets known
 
   // ---- write the records that fit and the permutation ------------------------
   bool fits_all = !s.failed;

@@ -32,6 +32,7 @@ struct EncodeArgs {
   const uint16_t* k;  // [batch][heads][nb*128][128] fp16
   const uint16_t* v;
   int batch, heads, nb, n_old, max_blocks, bits, key_kind;
+  int unit_mode;  // PACKKV_UNITS_*: unit base = smallest code, or 0
   uint32_t* k_index;
   uint32_t* v_index;
   uint8_t* k_arena;

@@ -25,6 +25,7 @@ FORMAT_VERSION = 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_DEVICE = range(6)
 DEV_CAPACITY, DEV_NONFINITE, DEV_BAD_RECORD, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 KEY_IDENTITY, KEY_K_SUM, KEY_KV_SUM = 0, 1, 2
+UNITS_FOR, UNITS_WIDTH_ONLY = 0, 1      # how the encoder sizes a unit (base = min, or 0)
 
 EXPORTED = [
     "packkv_abi_version", "packkv_cache_struct_size", "packkv_status_string", "packkv_record_bytes_max",
@@ -45,7 +46,8 @@ class PackKVError(RuntimeError):
 
 class Format(ctypes.Structure):
     _fields_ = [("version", ctypes.c_uint32), ("bits", ctypes.c_uint32), ("block_tokens", ctypes.c_uint32),
-                ("group_tokens", ctypes.c_uint32), ("head_dim", ctypes.c_uint32), ("reorder_key", ctypes.c_uint32)]
+                ("group_tokens", ctypes.c_uint32), ("head_dim", ctypes.c_uint32), ("reorder_key", ctypes.c_uint32),
+                ("unit_mode", ctypes.c_uint32)]
 
 
 class CacheStruct(ctypes.Structure):
@@ -126,7 +128,7 @@ class PackKVCache:
 
     def __init__(self, batch: int, kv_heads: int, max_blocks: int, bits: int, reorder_key: int = KEY_K_SUM,
                  arena_bytes: int | None = None, keep_perm: bool = False, device="cuda", ragged: bool = False,
-                 block_table: torch.Tensor | None = None):
+                 block_table: torch.Tensor | None = None, unit_mode: int = 0):
         dev = torch.device(device)
         if arena_bytes is None:
             arena_bytes = batch * kv_heads * max_blocks * record_bytes_max(bits)
@@ -141,7 +143,7 @@ class PackKVCache:
         self.perm = (torch.zeros((batch, kv_heads, max_blocks, BLOCK_TOKENS), dtype=torch.uint8, device=dev)
                      if keep_perm else None)
         self.s = CacheStruct()
-        self.s.fmt = Format(FORMAT_VERSION, bits, BLOCK_TOKENS, 32, HEAD_DIM, reorder_key)
+        self.s.fmt = Format(FORMAT_VERSION, bits, BLOCK_TOKENS, 32, HEAD_DIM, reorder_key, unit_mode)
         self.s.batch, self.s.kv_heads, self.s.max_blocks = batch, kv_heads, max_blocks
         self.s.n_blocks = self.s.tail_len = 0
         self.s.k_arena, self.s.v_arena = self.k_arena.data_ptr(), self.v_arena.data_ptr()

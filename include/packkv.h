@@ -39,7 +39,7 @@
 extern "C" {
 #endif
 
-#define PACKKV_ABI_VERSION 2u
+#define PACKKV_ABI_VERSION 3u
 #define PACKKV_FORMAT_VERSION 1u
 #define PACKKV_BLOCK_TOKENS 128
 #define PACKKV_GROUP_TOKENS 32
@@ -66,6 +66,15 @@ typedef enum {
 #define PACKKV_KEY_K_SUM 1u
 #define PACKKV_KEY_KV_SUM 2u
 
+/* How the encoder sizes a pack unit (packed-cache format v1, section 3; the PackKV
+ * paper page, Figure 3: quantized codes concentrate on few values).  Both give format
+ * v1 units (meta byte = base | width << 4) that every decode path reads alike:
+ *   FOR:        frame of reference, base = the unit's smallest code, width = bit length
+ *               of (largest - smallest);
+ *   WIDTH_ONLY: base = 0, width = bit length of the largest code (for the ablation). */
+#define PACKKV_UNITS_FOR 0u
+#define PACKKV_UNITS_WIDTH_ONLY 1u
+
 typedef struct {
   uint32_t version;      /* PACKKV_FORMAT_VERSION */
   uint32_t bits;         /* code width: 2, 3 or 4 */
@@ -73,6 +82,7 @@ typedef struct {
   uint32_t group_tokens; /* 32 */
   uint32_t head_dim;     /* 128 */
   uint32_t reorder_key;  /* PACKKV_KEY_* */
+  uint32_t unit_mode;    /* PACKKV_UNITS_*: encoder only */
 } packkv_format;
 
 /*

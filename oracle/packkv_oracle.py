@@ -167,10 +167,16 @@ def slices_of_width(w: int):
     return {0: [], 1: [(1, 0)], 2: [(2, 0)], 3: [(2, 0), (1, 2)], 4: [(4, 0)]}[w]
 
 
-def unit_base_width(codes32: np.ndarray):
-    """Frame of reference of one (group, channel) unit: base = min, w = bitlen(max - min)."""
+UNITS_FOR = 0          # frame of reference: base = min of the unit's codes (format v1 default)
+UNITS_WIDTH_ONLY = 1   # no base: base = 0, the width covers the largest code ([Fig. 3] ablation)
+
+
+def unit_base_width(codes32: np.ndarray, unit_mode: int = UNITS_FOR):
+    """Base and width of one (group, channel) unit: frame of reference (base = min,
+    w = bitlen(max - min)) or, width-only, base = 0 and w = bitlen(max).  Both are
+    format v1 units: the record stores base | w << 4 either way."""
     c = np.asarray(codes32, dtype=np.int64)
-    base = int(c.min())
+    base = int(c.min()) if unit_mode == UNITS_FOR else 0
     w = int(c.max() - base).bit_length()
     return base, w
 
@@ -296,15 +302,16 @@ def _ceil16(n: int) -> int:
 
 
 def build_record(codes_slot: np.ndarray, mn16: np.ndarray, sc16: np.ndarray,
-                 bits: int, is_v: bool) -> bytes:
-    """Assemble one record from codes in storage order [slot, channel] and params."""
+                 bits: int, is_v: bool, unit_mode: int = UNITS_FOR) -> bytes:
+    """Assemble one record from codes in storage order [slot, channel] and params
+    (units sized by unit_base_width in `unit_mode`)."""
     codes_slot = np.asarray(codes_slot, dtype=np.int64)
     assert codes_slot.shape == (BLOCK_TOKENS, HEAD_DIM)
     base = np.zeros((GROUPS_PER_BLOCK, HEAD_DIM), dtype=np.int64)
     width = np.zeros((GROUPS_PER_BLOCK, HEAD_DIM), dtype=np.int64)
     for g in range(GROUPS_PER_BLOCK):
         for c in range(HEAD_DIM):
-            base[g, c], width[g, c] = unit_base_width(codes_slot[32 * g:32 * g + 32, c])
+            base[g, c], width[g, c] = unit_base_width(codes_slot[32 * g:32 * g + 32, c], unit_mode)
     compressed_size = _ceil16(1040 + 4 * int(width.sum()))
     raw = compressed_size >= raw_record_bytes(bits)
     if raw:
@@ -438,7 +445,8 @@ def block_codes(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int =
 # ----------------------------------------------------------------------------
 # One block: quantize -> reorder -> pack
 # ----------------------------------------------------------------------------
-def encode_block(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int = KEY_K_SUM):
+def encode_block(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int = KEY_K_SUM,
+                 unit_mode: int = UNITS_FOR):
     """Encode one 128-token block of K and V.  Returns (k_record, v_record, perm)
     where perm[slot] = original token index within the block."""
     ck, k_mn, k_sc = quantize_block_k(k_blk, bits)
@@ -446,8 +454,8 @@ def encode_block(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int 
     rank = stable_rank(reorder_keys(ck, cv, key_kind))
     perm = np.empty(BLOCK_TOKENS, dtype=np.int64)
     perm[rank] = np.arange(BLOCK_TOKENS)
-    k_rec = build_record(ck[perm], k_mn, k_sc, bits, is_v=False)
-    v_rec = build_record(cv[perm], v_mn[perm], v_sc[perm], bits, is_v=True)
+    k_rec = build_record(ck[perm], k_mn, k_sc, bits, is_v=False, unit_mode=unit_mode)
+    v_rec = build_record(cv[perm], v_mn[perm], v_sc[perm], bits, is_v=True, unit_mode=unit_mode)
     return k_rec, v_rec, perm
 
 
@@ -467,10 +475,11 @@ def dequant_v(rec: ParsedRecord) -> np.ndarray:
 class OracleCache:
     """Mirror of the packed cache state: two arenas, two index tables, the tail."""
 
-    def __init__(self, batch, kv_heads, max_blocks, bits, key_kind=KEY_K_SUM, head_dim=HEAD_DIM):
+    def __init__(self, batch, kv_heads, max_blocks, bits, key_kind=KEY_K_SUM, head_dim=HEAD_DIM,
+                 unit_mode=UNITS_FOR):
         assert head_dim == HEAD_DIM
         self.batch, self.kv_heads, self.max_blocks = batch, kv_heads, max_blocks
-        self.bits, self.key_kind = bits, key_kind
+        self.bits, self.key_kind, self.unit_mode = bits, key_kind, unit_mode
         self.k_arena = bytearray()
         self.v_arena = bytearray()
         self.k_index = np.zeros((batch, kv_heads, max_blocks, 2), np.uint32)
@@ -495,7 +504,8 @@ class OracleCache:
                     if blocks is not None and (b, h, i) not in blocks:
                         continue
                     sl = slice(i * BLOCK_TOKENS, (i + 1) * BLOCK_TOKENS)
-                    k_rec, v_rec, perm = encode_block(k[b, h, sl], v[b, h, sl], self.bits, self.key_kind)
+                    k_rec, v_rec, perm = encode_block(k[b, h, sl], v[b, h, sl], self.bits, self.key_kind,
+                                                      self.unit_mode)
                     j = self.n_blocks + i
                     self.k_index[b, h, j] = (len(self.k_arena) // 16, len(k_rec) // 16)
                     self.v_index[b, h, j] = (len(self.v_arena) // 16, len(v_rec) // 16)
@@ -551,8 +561,8 @@ class RaggedOracleCache(OracleCache):
     block) order of the sequences they touch, as the uniform cache does.
     """
 
-    def __init__(self, batch, kv_heads, max_blocks, bits, key_kind=KEY_K_SUM, table=None):
-        super().__init__(batch, kv_heads, max_blocks, bits, key_kind)
+    def __init__(self, batch, kv_heads, max_blocks, bits, key_kind=KEY_K_SUM, table=None, unit_mode=UNITS_FOR):
+        super().__init__(batch, kv_heads, max_blocks, bits, key_kind, unit_mode=unit_mode)
         self.seq_blocks = [0] * batch
         self.seq_tail = [0] * batch
         ids = np.arange(batch * max_blocks, dtype=np.int64).reshape(batch, max_blocks)
@@ -563,7 +573,7 @@ class RaggedOracleCache(OracleCache):
         return divmod(int(self.table[b, j]), self.max_blocks)
 
     def _encode_one(self, b, h, j, k_blk, v_blk):
-        k_rec, v_rec, perm = encode_block(k_blk, v_blk, self.bits, self.key_kind)
+        k_rec, v_rec, perm = encode_block(k_blk, v_blk, self.bits, self.key_kind, self.unit_mode)
         rb, jb = self.physical(b, j)
         self.k_index[rb, h, jb] = (len(self.k_arena) // 16, len(k_rec) // 16)
         self.v_index[rb, h, jb] = (len(self.v_arena) // 16, len(v_rec) // 16)

@@ -58,7 +58,7 @@ def test_library_exports_every_declared_symbol(pk):
 
 def test_abi_constants(pk):
     lib = pk._lib
-    assert lib.packkv_abi_version() == 2
+    assert lib.packkv_abi_version() == 3
     assert lib.packkv_cache_struct_size() == ctypes.sizeof(pk.CacheStruct)
     assert [lib.packkv_record_bytes_max(b) for b in (1, 2, 3, 4, 5)] == [0, 4624, 6672, 8720, 0]
     assert lib.packkv_status_string(3) == b"capacity exceeded"
@@ -73,7 +73,7 @@ def _fake_cache(pk, **over):
         setattr(s, f, base + i * 0x100000)
     s.arena_bytes = 1 << 20
     for k, v in over.items():
-        if k in ("bits", "version", "reorder_key", "head_dim"):
+        if k in ("bits", "version", "reorder_key", "head_dim", "unit_mode"):
             setattr(s.fmt, k, v)
         else:
             setattr(s, k, v)
@@ -84,11 +84,13 @@ def test_host_checks_reject_before_launch(pk):
     lib = pk._lib
     ok = _fake_cache(pk)
     assert lib.packkv_cache_check(ctypes.byref(ok)) == pk.OK
+    assert lib.packkv_cache_check(ctypes.byref(_fake_cache(pk, unit_mode=pk.UNITS_WIDTH_ONLY))) == pk.OK
     bad_cases = {
         "bits": (dict(bits=5), pk.ERR_UNSUPPORTED),
         "version": (dict(version=2), pk.ERR_UNSUPPORTED),
         "head_dim": (dict(head_dim=64), pk.ERR_UNSUPPORTED),
         "key": (dict(reorder_key=7), pk.ERR_UNSUPPORTED),
+        "unit mode": (dict(unit_mode=2), pk.ERR_UNSUPPORTED),
         "misaligned": (dict(k_arena=0x10000008), pk.ERR_INVALID_ARG),
         "null": (dict(ctrl=0), pk.ERR_INVALID_ARG),
         "arena": (dict(arena_bytes=1000), pk.ERR_INVALID_ARG),

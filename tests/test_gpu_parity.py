@@ -27,13 +27,15 @@ def pk():
     return packkv
 
 
-def _build(pk, k, v, bits, key=O.KEY_K_SUM, max_blocks=None, keep_perm=True, arena_bytes=None):
+def _build(pk, k, v, bits, key=O.KEY_K_SUM, max_blocks=None, keep_perm=True, arena_bytes=None,
+           unit_mode=O.UNITS_FOR):
     B, H, T, _ = k.shape
     nb_total = T // 128
     mb = max_blocks or max(1, nb_total + 1)
-    cache = pk.PackKVCache(B, H, mb, bits, reorder_key=key, keep_perm=keep_perm, arena_bytes=arena_bytes)
+    cache = pk.PackKVCache(B, H, mb, bits, reorder_key=key, keep_perm=keep_perm, arena_bytes=arena_bytes,
+                           unit_mode=unit_mode)
     pk.prefill(cache, to_dev(k), to_dev(v))
-    ocache = O.OracleCache(B, H, mb, bits, key)
+    ocache = O.OracleCache(B, H, mb, bits, key, unit_mode=unit_mode)
     ocache.encode_blocks(k[:, :, :nb_total * 128], v[:, :, :nb_total * 128], nb_total)
     for t in range(nb_total * 128, T):
         ocache.append_token(k[:, :, t], v[:, :, t])
@@ -68,6 +70,28 @@ def test_encoder_bit_exact(pk, bits, structured, key):
     k, v, _ = synth.small_case(100 + bits + 3 * key, 2, 3, 1, 512, structured=structured)
     cache, ocache = _build(pk, k, v, bits, key)
     compare_encoder(cache, ocache)
+    assert pk.packkv_get_status(cache) == 0
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_width_only_units(pk, bits):
+    """The width-only unit mode (base 0, width of the largest code): records bit-exact
+    with the oracle, and the products over them (every decode path reads them as the
+    v1 units they are) within 1e-3 * sum|terms|."""
+    k, v, q = synth.small_case(150 + bits, 3, 4, 2, 5 * 128 + 21, structured=True)
+    cache, ocache = _build(pk, k, v, bits, unit_mode=O.UNITS_WIDTH_ONLY)
+    compare_encoder(cache, ocache)
+    got = _qk(pk, cache, q)
+    ref, terms = O.cache_qk(ocache, q, SCALE)
+    T = ocache.tokens
+    assert_within_terms(got[:, :, :T], ref, terms, "scores, width-only units")
+    p = O.softmax(ref)
+    ref_o, terms_o = O.cache_pv(ocache, p)
+    assert_within_terms(_pv(pk, cache, p), ref_o, terms_o, "p·V, width-only units")
+    att = torch.zeros((3, 8, 128), device="cuda")
+    pk.packkv_attention_decode(cache, to_dev(q), SCALE, att)
+    ref_a, terms_a = O.cache_attention(ocache, q, SCALE)
+    assert_within_terms(att.cpu().numpy(), ref_a, terms_a, "attention, width-only units")
     assert pk.packkv_get_status(cache) == 0
 
 

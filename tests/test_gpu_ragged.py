@@ -157,10 +157,12 @@ def test_ragged_many_sequences(pk, monkeypatch):
     import oracle.packkv_oracle as OM
     B, H, bits = 512, 4, 4
     real_enc, real_parse = OM.encode_block, OM.parse_record
-    enc = functools.lru_cache(maxsize=None)(lambda kb, vb, b_, key: real_enc(
-        np.frombuffer(kb, np.float16).reshape(128, 128), np.frombuffer(vb, np.float16).reshape(128, 128), b_, key))
-    monkeypatch.setattr(OM, "encode_block", lambda k_, v_, b_, key=O.KEY_K_SUM: enc(
-        np.ascontiguousarray(k_, np.float16).tobytes(), np.ascontiguousarray(v_, np.float16).tobytes(), b_, key))
+    enc = functools.lru_cache(maxsize=None)(lambda kb, vb, b_, key, mode: real_enc(
+        np.frombuffer(kb, np.float16).reshape(128, 128), np.frombuffer(vb, np.float16).reshape(128, 128), b_, key,
+        mode))
+    monkeypatch.setattr(OM, "encode_block", lambda k_, v_, b_, key=O.KEY_K_SUM, mode=O.UNITS_FOR: enc(
+        np.ascontiguousarray(k_, np.float16).tobytes(), np.ascontiguousarray(v_, np.float16).tobytes(), b_, key,
+        mode))
     monkeypatch.setattr(OM, "parse_record", functools.lru_cache(maxsize=None)(real_parse))
     pool_k, pool_v, _ = synth.small_case(94, 1, 4, 1, 128)
     rng = np.random.default_rng(4)

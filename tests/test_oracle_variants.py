@@ -47,6 +47,44 @@ def test_variant_sizes_by_hand():
         O.record_bytes_variant(ck4, 4, O.VARIANT_META4)
 
 
+def test_width_only_records():
+    """The encoder's width-only unit mode writes format v1 records (base 0, the width
+    of the largest code): their lengths are the size model's, they decode to the
+    same codes as the frame-of-reference records, and on block K1 of the record
+    goldens (0.5 everywhere, channel 0 = t % 2, K-sum key, 4-bit) the two units of
+    channel 0 in groups 2 and 3 carry meta byte 0x40 and four words 0xFFFFFFFF
+    (frame of reference: meta 0x0F and no words)."""
+    for bits in (2, 3, 4):
+        for structured in (False, True):
+            k, v, _ = synth.small_case(90 + bits, 1, 1, 1, 256, structured=structured)
+            for i in range(2):
+                kb, vb = k[0, 0, 128 * i:128 * (i + 1)], v[0, 0, 128 * i:128 * (i + 1)]
+                kw, vw, pw = O.encode_block(kb, vb, bits, unit_mode=O.UNITS_WIDTH_ONLY)
+                kf, vf, pf = O.encode_block(kb, vb, bits)
+                assert np.array_equal(pw, pf)
+                ck, cv = O.block_codes(kb, vb, bits)
+                assert len(kw) == O.record_bytes_variant(ck, bits, O.VARIANT_WIDTH_ONLY)
+                assert len(vw) == O.record_bytes_variant(cv, bits, O.VARIANT_WIDTH_ONLY)
+                for a, b in ((kw, kf), (vw, vf)):
+                    ra, rb = O.parse_record(a), O.parse_record(b)
+                    assert np.array_equal(ra.codes, rb.codes)
+                    if not ra.raw:
+                        assert np.all(ra.base == 0)
+    k = np.full((128, 128), np.float16(0.5))
+    k[:, 0] = (np.arange(128) % 2).astype(np.float16)
+    v = np.zeros((128, 128), np.float16)
+    kw, _, _ = O.encode_block(k, v, 4, unit_mode=O.UNITS_WIDTH_ONLY)
+    kf, _, _ = O.encode_block(k, v, 4)
+    assert len(kw) == 1072 and len(kf) == 1040
+    meta_w, meta_f = kw[528:1040], kf[528:1040]
+    for g in range(4):
+        assert meta_w[g * 128] == (0x40 if g >= 2 else 0x00)
+        assert meta_f[g * 128] == (0x0F if g >= 2 else 0x00)
+        assert all(meta_w[g * 128 + c] == 0 for c in range(1, 128))
+    words = np.frombuffer(kw, "<u4", 8, 1040)
+    assert np.all(words == 0xFFFFFFFF)
+
+
 def test_variant_invariants():
     """Width-only units are never narrower than frame-of-reference ones; fp32 params
     add exactly 512 B to a packed record and to the raw size; 4-bit meta saves 256 B
