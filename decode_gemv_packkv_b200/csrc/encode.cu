@@ -220,9 +220,10 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   __syncthreads();
 
   // ---- quantization ranges (K per channel, V per token) and non-finite values ---
-  // fp16 pairs: min / max of fp16 values are exact in fp16 (NaN is passed over, as fminf
-  // does; a signed zero is normalised below).  A value whose exponent field is all ones
-  // (inf or NaN) carries into bit 15 of its half when 0x0400 is added to that field.
+  // fp16 pairs: min / max of fp16 values are exact in fp16 (a signed zero is normalised
+  // below).  The NaN-propagating forms carry a NaN, and min / max carry an infinity, to
+  // the slice results, so one test of those finds every non-finite input: a value whose
+  // exponent field is all ones carries into bit 15 of its half when 0x0400 is added.
   {
     const __half2* k2 = reinterpret_cast<const __half2*>(&s.kx[0][0]);  // [token][channel pair]
     const __half2* v2 = reinterpret_cast<const __half2*>(&s.vx[0][0]);
@@ -232,14 +233,12 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     constexpr int kVSlice = kPairs / kParts;              // channel pairs per V token slice
     const int cp = tid % kPairs, kpart = tid / kPairs;
     const int t = tid % kBlockTokens, vpart = tid / kBlockTokens;
-    uint32_t bad = 0u;
     __half2 kmn = k2[kKSlice * kpart * kPairs + cp], kmx = kmn;
 #pragma unroll 8
     for (int i = 0; i < kKSlice; ++i) {
       const __half2 h = k2[(kKSlice * kpart + i) * kPairs + cp];
-      kmn = __hmin2(kmn, h);
-      kmx = __hmax2(kmx, h);
-      bad |= (*reinterpret_cast<const uint32_t*>(&h) & 0x7C007C00u) + 0x04000400u;
+      kmn = __hmin2_nan(kmn, h);
+      kmx = __hmax2_nan(kmx, h);
     }
     // a token's pairs from a rotated start: the 32 tokens of a warp hit 32 banks
     const int p0 = kVSlice * vpart + t;
@@ -247,17 +246,20 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
 #pragma unroll 8
     for (int j = 0; j < kVSlice; ++j) {
       const __half2 h = v2[t * kPairs + ((p0 + j) & (kPairs - 1))];
-      vmn = __hmin2(vmn, h);
-      vmx = __hmax2(vmx, h);
-      bad |= (*reinterpret_cast<const uint32_t*>(&h) & 0x7C007C00u) + 0x04000400u;
+      vmn = __hmin2_nan(vmn, h);
+      vmx = __hmax2_nan(vmx, h);
     }
+    auto nonfinite2 = [](__half2 x) {
+      return ((*reinterpret_cast<const uint32_t*>(&x) & 0x7C007C00u) + 0x04000400u) & 0x80008000u;
+    };
+    const uint32_t bad = nonfinite2(kmn) | nonfinite2(kmx) | nonfinite2(vmn) | nonfinite2(vmx);
     __half2* redk = reinterpret_cast<__half2*>(&s.red[0][0]);  // [min, max][kKParts][kPairs]
     __half* redv = reinterpret_cast<__half*>(&s.red[2][0]);    // [min, max][kParts][kBlockTokens]
     redk[kpart * kPairs + cp] = kmn;
     redk[(kKParts + kpart) * kPairs + cp] = kmx;
     redv[vpart * kBlockTokens + t] = __hmin(__low2half(vmn), __high2half(vmn));
     redv[(kParts + vpart) * kBlockTokens + t] = __hmax(__low2half(vmx), __high2half(vmx));
-    if (bad & 0x80008000u) s.nonfinite = 1;
+    if (bad) s.nonfinite = 1;
   }
   __syncthreads();
   if (tid == 0 && s.nonfinite) set_status(a.ctrl, PACKKV_DEV_NONFINITE);
@@ -596,36 +598,66 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
       }
     }
   }
-  // pack the units: every word is owned by exactly one thread
+  // pack the units: every word is owned by exactly one thread.  A unit's 32 offsets are
+  // held as eight words of four bytes (slots 4k .. 4k+3 in word k); each slice is then
+  // gathered with shifts, masks and byte permutes (field j of a p-bit slice at bit
+  // (j p) mod 32 of word (j p) / 32, packed-cache format v1, section 3).
   for (int u = asm_id; asm_id >= 0 && u < 2 * kGroups * kHeadDim; u += n_asm) {
     const int tensor = u >> 9, g = (u >> 7) & 3, c = u & 127;
     if (raw[tensor]) continue;  // written above
-    const int w = raw[tensor] ? a.bits : s.width[tensor][g][c];
-    const int base = raw[tensor] ? 0 : s.base[tensor][g][c];
+    const int w = s.width[tensor][g][c];
     if (w == 0) continue;
+    const uint32_t base4 = (uint32_t)s.base[tensor][g][c] * 0x01010101u;
     int gstart = 0;
     for (int gg = 0; gg < g; ++gg) gstart += s.group_total[tensor][gg];
-    uint32_t* words = rec32[tensor] + (raw[tensor] ? kRawWordOffset : kPackedWordOffset) / 4 + gstart +
-                      s.ustart[tensor][g][c];
-    // slices in descending size: 4 | 2 then 1 | 2 | 1
-    int lo = 0, at = 0;
-    int rem = w;
-    while (rem > 0) {
-      const int p = rem >= 4 ? 4 : (rem >= 2 ? 2 : 1);
-      const uint32_t mask = (1u << p) - 1u;
-      for (int q = 0; q < p; ++q) {
-        uint32_t word = 0;
-        const int per = 32 / p;
-        for (int f = 0; f < per; ++f) {
-          const int j = q * per + f;
-          const uint32_t off = (uint32_t)(slot_code(tensor, g * kGroupTokens + j, c) - base);
-          word |= ((off >> lo) & mask) << ((j * p) & 31);
-        }
-        words[at + q] = word;
+    uint32_t* words = rec32[tensor] + kPackedWordOffset / 4 + gstart + s.ustart[tensor][g][c];
+    uint32_t ow[8];  // offsets (code - base, no borrow between bytes)
+    if (tensor) {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(vt + c * kVtPitch + g * kGroupTokens);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ow[k] = src[k] - base4;
+    } else {
+      const uint8_t* src = kp + g * kGroupTokens * kHeadDim + c;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t b0 = src[(4 * k) * kHeadDim], b1 = src[(4 * k + 1) * kHeadDim];
+        const uint32_t b2 = src[(4 * k + 2) * kHeadDim], b3 = src[(4 * k + 3) * kHeadDim];
+        ow[k] = __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u) - base4;
       }
-      at += p;
-      lo += p;
-      rem -= p;
+    }
+    // slices in descending size: 4 | 2 then 1 | 2 | 1
+    int at = 0, lo = 0;
+    if (w == 4) {  // word q: slots 8q .. 8q+7, a nibble each
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t y0 = ow[2 * q] | (ow[2 * q] >> 4), y1 = ow[2 * q + 1] | (ow[2 * q + 1] >> 4);
+        words[q] = __byte_perm(y0, y1, 0x6420u);
+      }
+      at = 4;
+    }
+    if (w & 2) {  // word q: slots 16q .. 16q+15, two bits each, from bits 0-1
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        uint32_t z[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t x = ow[4 * q + k] & 0x03030303u;
+          const uint32_t y = x | (x >> 6);  // bytes 0 and 2: two fields each
+          z[k] = y | (y >> 12);             // byte 0: slots 4k .. 4k+3
+        }
+        words[at + q] = __byte_perm(__byte_perm(z[0], z[1], 0x0040u), __byte_perm(z[2], z[3], 0x0040u), 0x5410u);
+      }
+      at += 2;
+      lo = 2;
+    }
+    if (w & 1) {  // one word: slot j at bit j, from bit lo
+      uint32_t word = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t x = (ow[k] >> lo) & 0x01010101u;
+        word |= ((x * 0x10204080u) >> 28) << (4 * k);  // bit of byte e -> bit 28 + e
+      }
+      words[at] = word;
     }
   }
 

@@ -239,12 +239,18 @@ def test_arena_overflow_is_detected_on_device(pk):
     assert pk.packkv_get_status(cache) == 0     # read-and-clear
 
 
-def test_nonfinite_input_sets_status(pk):
-    k, v, _ = synth.small_case(78, 1, 1, 1, 128)
-    k[0, 0, 5, 7] = np.inf
-    cache = pk.PackKVCache(1, 1, 2, 4)
-    pk.packkv_encode_block(cache, to_dev(k), to_dev(v), 1)
+@pytest.mark.parametrize("where,value", [("k", np.inf), ("k", -np.inf), ("v", np.nan), ("k", np.nan),
+                                         ("v", -np.inf)])
+def test_nonfinite_input_sets_status(pk, where, value):
+    """A NaN or an infinity anywhere in a block sets the sticky non-finite bit; a clean
+    block after it does not."""
+    k, v, _ = synth.small_case(78, 1, 1, 1, 256)
+    (k if where == "k" else v)[0, 0, 5, 7] = value
+    cache = pk.PackKVCache(1, 1, 3, 4)
+    pk.packkv_encode_block(cache, to_dev(k[:, :, :128].copy()), to_dev(v[:, :, :128].copy()), 1)
     assert pk.packkv_get_status(cache) & pk.DEV_NONFINITE
+    pk.packkv_encode_block(cache, to_dev(k[:, :, 128:].copy()), to_dev(v[:, :, 128:].copy()), 1)
+    assert pk.packkv_get_status(cache) == 0
 
 
 # ----------------------------------------------------------------------------- full workload sizes
