@@ -47,12 +47,12 @@ constexpr int kParts = kEncodeThreads / kBlockTokens;  // threads per channel / 
 struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
   __half kx[kBlockTokens][kHeadDim];   // input K block; later the K record buffer
   __half vx[kBlockTokens][kHeadDim];   // input V block; later the V record buffer
-  uint8_t ck[kBlockTokens][kHeadDim];  // K codes [token][channel]
+  uint8_t ck[kBlockTokens][kHeadDim];  // K codes [token][channel]; before them, the range partials
   uint8_t cv[kBlockTokens][kHeadDim];  // V codes [token][channel]
   uint16_t kmin[kHeadDim], kscale[kHeadDim];     // per channel
   uint16_t vmin[kBlockTokens], vscale[kBlockTokens];  // per token (original order)
-  float krcp[kHeadDim], vrcp[kBlockTokens];      // 1 / scale (rounded), 0 for a zero scale
-  float red[4][kEncodeThreads];        // min / max partials
+  float krcp[kHeadDim];                          // 1 / scale (rounded), 0 for a zero scale
+  float4 vq[kBlockTokens];  // per token: -min, 1 / scale (rounded, 0 for a zero scale), scale
   alignas(16) int key[kBlockTokens];  // reorder key * 128 + token
   int rank_part[kParts][kBlockTokens];
   uint8_t perm[kBlockTokens];          // perm[slot] = token
@@ -253,8 +253,8 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
       return ((*reinterpret_cast<const uint32_t*>(&x) & 0x7C007C00u) + 0x04000400u) & 0x80008000u;
     };
     const uint32_t bad = nonfinite2(kmn) | nonfinite2(kmx) | nonfinite2(vmn) | nonfinite2(vmx);
-    __half2* redk = reinterpret_cast<__half2*>(&s.red[0][0]);  // [min, max][kKParts][kPairs]
-    __half* redv = reinterpret_cast<__half*>(&s.red[2][0]);    // [min, max][kParts][kBlockTokens]
+    __half2* redk = reinterpret_cast<__half2*>(&s.ck[0][0]);  // [min, max][kKParts][kPairs]
+    __half* redv = reinterpret_cast<__half*>(&s.ck[0][0]) + 2 * 2 * kEncodeThreads;  // [min, max][kParts][128]
     redk[kpart * kPairs + cp] = kmn;
     redk[(kKParts + kpart) * kPairs + cp] = kmx;
     redv[vpart * kBlockTokens + t] = __hmin(__low2half(vmn), __high2half(vmn));
@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     const bool is_k = tid < kBlockTokens;
     const int i = tid % kBlockTokens;
     // K: the halves of channel i over the token slices; V: token i over the pair slices
-    const __half* red = reinterpret_cast<const __half*>(is_k ? &s.red[0][0] : &s.red[2][0]);
+    const __half* red = reinterpret_cast<const __half*>(&s.ck[0][0]) + (is_k ? 0 : 2 * 2 * kEncodeThreads);
     const int nq = is_k ? kEncodeThreads / (kHeadDim / 2) : kParts;
     __half hlo = red[i], hhi = red[nq * kBlockTokens + i];
     for (int q = 1; q < nq; ++q) {
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
     } else {
       s.vmin[i] = mnb;
       s.vscale[i] = sc;
-      s.vrcp[i] = rcp;
+      s.vq[i] = make_float4(-half_bits_to_float(mnb), rcp, half_bits_to_float(sc), 0.0f);
     }
   }
   __syncthreads();
@@ -349,7 +349,8 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
       const uint2 vw = *reinterpret_cast<const uint2*>(&s.vx[t][4 * j]);
       const float2 xv[2] = {__half22float2(*reinterpret_cast<const __half2*>(&vw.x)),
                             __half22float2(*reinterpret_cast<const __half2*>(&vw.y))};
-      const float nvm = -half_bits_to_float(s.vmin[t]), vr = s.vrcp[t], vs = half_bits_to_float(s.vscale[t]);
+      const float4 pq = s.vq[t];
+      const float nvm = pq.x, vr = pq.y, vs = pq.z;
       const float2 nvm2[2] = {make_float2(nvm, nvm), make_float2(nvm, nvm)};
       const float2 vr2[2] = {make_float2(vr, vr), make_float2(vr, vr)};
       const float vsc[4] = {vs, vs, vs, vs};
