@@ -4,7 +4,8 @@
 //
 // One encode call is one pass over the input: a CTA per (sequence, head, block)
 // quantizes the K and V blocks, ranks the tokens, sizes the units, assembles both
-// records in shared memory and writes them at their arena offsets.  The offsets
+// records in shared memory (while two warps find the arena offsets) and writes them
+// at their arena offsets.  The offsets
 // follow ascending (sequence, head, block) order, so they are prefix sums of
 // the record lengths; a CTA learns its prefix by decoupled look-back over the
 // index entries of the blocks before it:
@@ -47,7 +48,7 @@ constexpr int kParts = kEncodeThreads / kBlockTokens;  // threads per channel / 
 struct EncodeSmem {  // two CTAs per SM: at most about 113 KB
   __half kx[kBlockTokens][kHeadDim];   // input K block; later the K record buffer
   __half vx[kBlockTokens][kHeadDim];   // input V block; later the V record buffer
-  uint8_t ck[kBlockTokens][kHeadDim];  // K codes [token][channel]; before them, the range partials
+  uint8_t ck[kBlockTokens][kHeadDim];  // K codes [token][channel] (first the range partials)
   uint8_t cv[kBlockTokens][kHeadDim];  // V codes [token][channel]
   uint16_t kmin[kHeadDim], kscale[kHeadDim];     // per channel
   uint16_t vmin[kBlockTokens], vscale[kBlockTokens];  // per token (original order)
