@@ -295,9 +295,10 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
   }
   __syncthreads();
 
-  // ---- codes -----------------------------------------------------------------
+  // ---- codes and reorder keys ---------------------------------------------------
   // A thread keeps four channels (their K parameters in registers) and walks tokens;
-  // the four codes of a tensor go to shared memory as one word.  Fast path in pairs:
+  // the four codes of a tensor go to shared memory as one word, and a warp's 32 lanes
+  // (all channels of one token) sum the token's reorder key.  Fast path in pairs:
   // q = fl(x - mn) * RN(1/scale), rint(q) by adding and removing 1.5 * 2^23 (ties to
   // even), e = q - rint(q) exactly.  quant_code takes the correctly rounded quotient
   // where it can differ, |e| >= 0.5 - 2^-17; where q is not finite or not below
@@ -346,7 +347,8 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
       const uint2 kw = *reinterpret_cast<const uint2*>(&s.kx[t][4 * j]);
       const float2 xk[2] = {__half22float2(*reinterpret_cast<const __half2*>(&kw.x)),
                             __half22float2(*reinterpret_cast<const __half2*>(&kw.y))};
-      *reinterpret_cast<uint32_t*>(&s.ck[t][4 * j]) = codes4(xk, nkmn, kr, ksc);
+      const uint32_t kcodes = codes4(xk, nkmn, kr, ksc);
+      *reinterpret_cast<uint32_t*>(&s.ck[t][4 * j]) = kcodes;
       const uint2 vw = *reinterpret_cast<const uint2*>(&s.vx[t][4 * j]);
       const float2 xv[2] = {__half22float2(*reinterpret_cast<const __half2*>(&vw.x)),
                             __half22float2(*reinterpret_cast<const __half2*>(&vw.y))};
@@ -355,26 +357,23 @@ __global__ void __launch_bounds__(kEncodeThreads) encode_kernel(const EncodeArgs
       const float2 nvm2[2] = {make_float2(nvm, nvm), make_float2(nvm, nvm)};
       const float2 vr2[2] = {make_float2(vr, vr), make_float2(vr, vr)};
       const float vsc[4] = {vs, vs, vs, vs};
-      *reinterpret_cast<uint32_t*>(&s.cv[t][4 * j]) = codes4(xv, nvm2, vr2, vsc);
+      const uint32_t vcodes = codes4(xv, nvm2, vr2, vsc);
+      *reinterpret_cast<uint32_t*>(&s.cv[t][4 * j]) = vcodes;
+      // the reorder key of token t (the warp holds all its channels): the sum of its K
+      // codes (plus its V codes for the K+V key), then the token index below it, so
+      // that all keys differ and a plain count gives the stable rank
+      uint32_t sum = 0u;
+      if (a.key_kind != PACKKV_KEY_IDENTITY) {
+        sum = __dp4a(kcodes, 0x01010101u, 0u);
+        if (a.key_kind == PACKKV_KEY_KV_SUM) sum = __dp4a(vcodes, 0x01010101u, sum);
+      }
+      sum = __reduce_add_sync(0xffffffffu, sum);
+      if (j == 0) s.key[t] = (int)sum * kBlockTokens + t;
     }
   }
   __syncthreads();
 
-  // ---- reorder key per token, then stable rank ------------------------------
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int t = warp; t < kBlockTokens; t += blockDim.x / 32) {
-      uint32_t sum = 0;
-      if (a.key_kind != PACKKV_KEY_IDENTITY) {
-        sum = __dp4a(reinterpret_cast<const uint32_t*>(s.ck[t])[lane], 0x01010101u, 0u);
-        if (a.key_kind == PACKKV_KEY_KV_SUM)
-          sum = __dp4a(reinterpret_cast<const uint32_t*>(s.cv[t])[lane], 0x01010101u, sum);
-      }
-      sum = __reduce_add_sync(0xffffffffu, sum);
-      if (lane == 0) s.key[t] = (int)sum * kBlockTokens + t;  // key, then index: all distinct
-    }
-  }
-  __syncthreads();
+  // ---- stable rank -------------------------------------------------------------
   {
     // rank of token t = #{u : key[u] < key[t] or (key[u] == key[t] and u < t)}: with the
     // index below the key (key * 128 + u), #{u : composite[u] < composite[t]};
