@@ -151,6 +151,7 @@ packkv_status packkv_cache_reset(packkv_cache* cache, void* stream);
  * (quantize, joint token reorder, channel-direction bit-packing: packed-cache format v1,
  * sections 1-4; paper page Figures 2 and 5).
  *   k, v: device fp16 [batch][kv_heads][n_blocks*128][128], row-major.
+ * Pack units are sized as cache->fmt.unit_mode says (PACKKV_UNITS_*).
  * Records go to the arenas in ascending (sequence, head, block) order.
  * Requires tail_len == 0 and n_blocks + cache->n_blocks <= max_blocks
  * (else PACKKV_ERR_INVALID_ARG / PACKKV_ERR_CAPACITY, nothing launched).
