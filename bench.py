@@ -188,6 +188,11 @@ def timed_ms(dev, fn, pre_sleep=True) -> float:
     return a.elapsed_time(b_)
 
 
+def median_ms(dev, fn, reps: int = 5) -> float:
+    """Median of `reps` CUDA-event timings of fn() (per-kernel sub-record times)."""
+    return statistics.median(timed_ms(dev, fn) for _ in range(reps))
+
+
 def capture(dev, fn):
     """A CUDA graph of fn() (run once eagerly on a side stream first)."""
     import torch
@@ -263,7 +268,8 @@ class CacheSet:
         return capture(self.dev, body)
 
     def per_launch_ms(self, kind, min_launches=60):
-        """Average time of one launch of `kind` over whole rotations of the copies."""
+        """Average time of one launch of `kind` over whole rotations of the copies (the
+        median of five such timings)."""
         g = self.graph(kind)
         g.replay()
         reps = max(1, int(np.ceil(min_launches / self.R)))
@@ -271,7 +277,7 @@ class CacheSet:
         def run():
             for _ in range(reps):
                 g.replay()
-        return timed_ms(self.dev, run) / (reps * self.R)
+        return median_ms(self.dev, run) / (reps * self.R)
 
     def bytes(self):
         B, Hq, T = self.B, self.Hq, self.T
@@ -485,7 +491,7 @@ def ragged_record(pk, dev, peak, bits=3):
         g = capture(dev, lambda: [fn(i) for i in range(R)])
         g.replay()
         reps = max(1, int(np.ceil(60 / R)))
-        return timed_ms(dev, lambda: [g.replay() for _ in range(reps)]) / (reps * R)
+        return median_ms(dev, lambda: [g.replay() for _ in range(reps)]) / (reps * R)
     qk_ms = per_launch(lambda i: pk.packkv_qk_gemv(caches[i], q[i], SCALE, scores))
     pv_ms = per_launch(lambda i: pk.packkv_pv_gemv(caches[i], p, out, ws))
     at_ms = per_launch(lambda i: pk.packkv_attention_decode(caches[i], q[i], SCALE, out, wsa))

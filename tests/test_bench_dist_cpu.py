@@ -93,3 +93,13 @@ def test_reference_arm_line(monkeypatch, capsys):
     assert line["impl"] == "reference" and line["unit"] == bench.UNIT and line["higher_is_better"] is True
     assert line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_median_ms_takes_the_median_of_five_timings(monkeypatch):
+    """Sub-record kernel times are the median of five CUDA-event timings."""
+    import bench
+    seq = iter([5.0, 1.0, 9.0, 3.0, 7.0])
+    calls = []
+    monkeypatch.setattr(bench, "timed_ms", lambda dev, fn: calls.append(fn) or next(seq))
+    assert bench.median_ms(None, "f") == 5.0
+    assert calls == ["f"] * 5
