@@ -366,6 +366,8 @@ def parse_record(rec: bytes) -> ParsedRecord:
     bits = (flags >> 16) & 0xF
     if version != FORMAT_VERSION:
         raise ValueError("unknown record version")
+    if flags >> 24:
+        raise ValueError("a layout-variant record (parse_record_variant reads those)")
     mn = np.frombuffer(rec, dtype="<f2", count=128, offset=16).astype(np.float16)
     sc = np.frombuffer(rec, dtype="<f2", count=128, offset=272).astype(np.float16)
     if raw:
@@ -430,6 +432,103 @@ def record_bytes_variant(codes_slot: np.ndarray, bits: int, variant: str) -> int
     packed = _ceil16(16 + params + meta + 4 * wsum)
     raw = 16 + params + 2048 * bits
     return min(packed, raw)
+
+
+# Records of the two layout variants (ablation only; the library writes and reads v1).
+# The header is v1's with a variant id in flags bits 24-27; then
+#   fp32 parameters: min[128] and scale[128] as fp32 (the fp16 values widened, so codes
+#     and decoded values equal v1's), meta at 1040, words at 1552 (raw: words at 1040);
+#   4-bit meta (b = 2): unit (g, c) in the 4-bit entry (byte (128 g + c) / 2, low
+#     nibble for even c) = base | w << 2, meta at 528 (256 B), words at 784 (raw: as v1).
+# Units, slices, the raw fragment order and the raw rule (packed >= raw size) are v1's.
+VARIANT_IDS = {VARIANT_FP32_PARAMS: 1, VARIANT_META4: 2}
+
+
+def build_record_variant(codes_slot: np.ndarray, mn16: np.ndarray, sc16: np.ndarray, bits: int,
+                         is_v: bool, variant: str) -> bytes:
+    """One record of a layout variant (v1 and width-only: build_record)."""
+    if variant == VARIANT_V1:
+        return build_record(codes_slot, mn16, sc16, bits, is_v)
+    if variant == VARIANT_WIDTH_ONLY:
+        return build_record(codes_slot, mn16, sc16, bits, is_v, UNITS_WIDTH_ONLY)
+    if variant == VARIANT_META4 and bits != 2:
+        raise ValueError("the 4-bit meta variant is for 2-bit codes")
+    codes_slot = np.asarray(codes_slot, dtype=np.int64)
+    fp32 = variant == VARIANT_FP32_PARAMS
+    params = 1024 if fp32 else 512
+    meta_bytes = 256 if variant == VARIANT_META4 else 512
+    base = np.zeros((GROUPS_PER_BLOCK, HEAD_DIM), dtype=np.int64)
+    width = np.zeros((GROUPS_PER_BLOCK, HEAD_DIM), dtype=np.int64)
+    for g in range(GROUPS_PER_BLOCK):
+        for c in range(HEAD_DIM):
+            base[g, c], width[g, c] = unit_base_width(codes_slot[32 * g:32 * g + 32, c])
+    raw_size = 16 + params + 2048 * bits
+    raw = _ceil16(16 + params + meta_bytes + 4 * int(width.sum())) >= raw_size
+    if raw:
+        base[:] = 0
+        width[:] = bits
+        words = pack_raw_fragment(codes_slot.T if is_v else codes_slot, bits)
+    else:
+        words = np.concatenate([pack_unit(codes_slot[32 * g:32 * g + 32, c] - base[g, c], int(width[g, c]))
+                                for g in range(GROUPS_PER_BLOCK) for c in range(HEAD_DIM)]).astype(np.uint32)
+    group_start = [int(width[:g].sum()) for g in range(GROUPS_PER_BLOCK)]
+    flags = ((RAW_FLAG if raw else 0) | (V_FLAG if is_v else 0) | (FORMAT_VERSION << 8) | (bits << 16)
+             | (VARIANT_IDS[variant] << 24))
+    out = bytearray()
+    out += struct.pack("<4H", *group_start)
+    out += struct.pack("<II", flags, int(words.size))
+    pdt = np.float32 if fp32 else np.float16
+    out += np.asarray(mn16, np.float16).astype(pdt).tobytes()
+    out += np.asarray(sc16, np.float16).astype(pdt).tobytes()
+    if not raw:
+        if variant == VARIANT_META4:
+            e = (base | (width << 2)).reshape(-1)
+            out += (e[0::2] | (e[1::2] << 4)).astype(np.uint8).tobytes()
+        else:
+            out += (base | (width << 4)).astype(np.uint8).tobytes()
+    out += words.astype("<u4").tobytes()
+    out += b"\x00" * (_ceil16(len(out)) - len(out))
+    assert raw == (len(out) == raw_size)
+    return bytes(out)
+
+
+def parse_record_variant(rec: bytes) -> ParsedRecord:
+    """Inverse of build_record_variant for the two layout variants."""
+    gws = list(struct.unpack_from("<4H", rec, 0))
+    flags, total_words = struct.unpack_from("<II", rec, 8)
+    vid = flags >> 24
+    variant = {i: v for v, i in VARIANT_IDS.items()}.get(vid)
+    if variant is None or (flags >> 8) & 0xFF != FORMAT_VERSION:
+        raise ValueError("not a layout-variant record")
+    raw, is_v, bits = bool(flags & RAW_FLAG), bool(flags & V_FLAG), (flags >> 16) & 0xF
+    fp32 = variant == VARIANT_FP32_PARAMS
+    pdt, params = ("<f4", 1024) if fp32 else ("<f2", 512)
+    mn = np.frombuffer(rec, dtype=pdt, count=128, offset=16).astype(np.float16)
+    sc = np.frombuffer(rec, dtype=pdt, count=128, offset=16 + params // 2).astype(np.float16)
+    if raw:
+        words = np.frombuffer(rec, dtype="<u4", count=total_words, offset=16 + params).astype(np.uint64)
+        a = unpack_raw_fragment(words, bits)
+        codes = a.T.copy() if is_v else a
+        return ParsedRecord(raw, is_v, bits, mn, sc, np.zeros((4, 128), np.int64), np.full((4, 128), bits, np.int64),
+                            codes, gws)
+    if variant == VARIANT_META4:
+        m = np.frombuffer(rec, dtype=np.uint8, count=256, offset=16 + params).astype(np.int64)
+        e = np.stack([m & 0xF, m >> 4], axis=1).reshape(4, 128)
+        base, width, word_at = e & 3, e >> 2, 16 + params + 256
+    else:
+        meta = np.frombuffer(rec, dtype=np.uint8, count=512, offset=16 + params).astype(np.int64).reshape(4, 128)
+        base, width, word_at = meta & 0xF, meta >> 4, 16 + params + 512
+    words = np.frombuffer(rec, dtype="<u4", count=total_words, offset=word_at).astype(np.uint64)
+    codes = np.zeros((128, 128), np.int64)
+    at = 0
+    for g in range(4):
+        if at != gws[g]:
+            raise ValueError("group_word_start does not match the unit widths")
+        for c in range(128):
+            w = int(width[g, c])
+            codes[32 * g:32 * g + 32, c] = base[g, c] + unpack_unit(words[at:at + w], w)
+            at += w
+    return ParsedRecord(raw, is_v, bits, mn, sc, base, width, codes, gws)
 
 
 def block_codes(k_blk: np.ndarray, v_blk: np.ndarray, bits: int, key_kind: int = KEY_K_SUM):

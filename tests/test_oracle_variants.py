@@ -7,6 +7,8 @@ reference units and narrow meta exploit).  The oracle's size model of each
 variant is pinned to the real v1 records and to record sizes derived by hand;
 the ratios it gives on the synthetic workloads are reported by the last test.
 """
+import struct
+
 import numpy as np
 import pytest
 
@@ -83,6 +85,55 @@ def test_width_only_records():
         assert all(meta_w[g * 128 + c] == 0 for c in range(1, 128))
     words = np.frombuffer(kw, "<u4", 8, 1040)
     assert np.all(words == 0xFFFFFFFF)
+
+
+def test_layout_variant_records():
+    """Records of the fp32-parameter and 4-bit-meta layouts: their lengths are the size
+    model's, they parse back to the v1 codes and parameters, and v1's parser refuses
+    them.  By hand, on block K1 of the record goldens (0.5 everywhere, channel 0 =
+    t % 2, K-sum key): at 2 bits the units of channel 0 in groups 2 and 3 hold code 3,
+    so their 4-bit entries (low nibble of meta bytes 128 and 192) are base 3 | w 0 << 2
+    = 0x3 and the record is 784 bytes; at 4 bits the fp32 record is 1552 bytes with
+    min[1] = 0.5f (0x3F000000) and meta byte 0x0F for those units."""
+    for bits in (2, 3, 4):
+        for structured in (False, True):
+            k, v, _ = synth.small_case(110 + bits, 1, 1, 1, 128, structured=structured)
+            kb, vb = k[0, 0], v[0, 0]
+            ck, k_mn, k_sc = O.quantize_block_k(kb, bits)
+            cv, v_mn, v_sc = O.quantize_block_v(vb, bits)
+            rank = O.stable_rank(O.reorder_keys(ck, cv, O.KEY_K_SUM))
+            perm = np.empty(128, np.int64)
+            perm[rank] = np.arange(128)
+            variants = [O.VARIANT_FP32_PARAMS] + ([O.VARIANT_META4] if bits == 2 else [])
+            for codes, mn, sc, is_v in ((ck[perm], k_mn, k_sc, False), (cv[perm], v_mn[perm], v_sc[perm], True)):
+                v1 = O.parse_record(O.build_record(codes, mn, sc, bits, is_v))
+                for var in variants:
+                    rec = O.build_record_variant(codes, mn, sc, bits, is_v, var)
+                    assert len(rec) == O.record_bytes_variant(codes, bits, var)
+                    p = O.parse_record_variant(rec)
+                    assert np.array_equal(p.codes, codes) and np.array_equal(p.codes, v1.codes)
+                    assert np.array_equal(p.mn, v1.mn) and np.array_equal(p.scale, v1.scale)
+                    assert p.raw == v1.raw and p.is_v == is_v
+                    with pytest.raises(ValueError):
+                        O.parse_record(rec)
+    k = np.full((128, 128), np.float16(0.5))
+    k[:, 0] = (np.arange(128) % 2).astype(np.float16)
+    ck, mn, sc = O.quantize_block_k(k, 2)
+    rank = O.stable_rank(O.reorder_keys(ck, ck, O.KEY_K_SUM))
+    perm = np.empty(128, np.int64)
+    perm[rank] = np.arange(128)
+    rec = O.build_record_variant(ck[perm], mn, sc, 2, False, O.VARIANT_META4)
+    assert len(rec) == 784
+    meta = rec[528:784]
+    assert meta[128] == 0x03 and meta[192] == 0x03 and meta[0] == 0 and meta[64] == 0
+    assert all(b == 0 for i, b in enumerate(meta) if i not in (128, 192))
+    ck4, mn4, sc4 = O.quantize_block_k(k, 4)
+    rank = O.stable_rank(O.reorder_keys(ck4, ck4, O.KEY_K_SUM))
+    perm[rank] = np.arange(128)
+    rec = O.build_record_variant(ck4[perm], mn4, sc4, 4, False, O.VARIANT_FP32_PARAMS)
+    assert len(rec) == 1552
+    assert struct.unpack_from("<I", rec, 16 + 4)[0] == 0x3F000000
+    assert rec[1040 + 256] == 0x0F and rec[1040 + 384] == 0x0F
 
 
 def test_variant_invariants():
